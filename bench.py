@@ -1,0 +1,405 @@
+#!/usr/bin/env python
+"""Benchmark: one GQA decode step (one layer) per step, on N GPUs.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one gqa_decode call (split-KV kernel + LSE combine kernel) over one
+batch of the workload, with q, the KV cache and seq_lens resident in HBM.
+The default workload is the Llama-2-70B-shaped ragged batch (B=32, 64 query /
+8 KV heads, head_dim 128, lengths U[1, 32768]); its KV bytes per step
+(~2.15 GB) exceed the 126 MB L2, so no flush is needed between steps.
+
+Printed metric: achieved HBM GB/s of algorithmic traffic (K and V rows of
+the live tokens, plus Q and the fp32 output) -- whole-job over N GPUs, each
+GPU running its own independent batch (weak scaling, no collective on the
+data path).  Timing: CUDA events on the launching stream, barrier and
+synchronize around exactly K steps, max over ranks.
+
+--impl reference times the fp64 CPU oracle on the host cores on a bounded
+sample of the same workload (the slow reference arm).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from gqa_mqa_kv_b200.workloads import WORKLOADS, algorithmic_bytes, make_inputs  # noqa: E402
+
+METRIC = "decode-attention achieved HBM GB/s (% of B200 peak) and µs per decode step"
+FALLBACK_HBM_GBS = 6650.0
+CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+REASON_NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3000)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama2_70b_ragged", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--soak-seconds", type=float, default=1.5,
+                    help="untimed steps before the timed region so clocks settle and are sampled")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    if dist is None:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- peaks, clocks, profiles
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            v = float(json.load(f)["hbm_gbs"])
+        return v, "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background (200 ms period)."""
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.file = None
+
+    def __enter__(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.file is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        self.file.flush()
+        with open(self.file.name) as f:
+            rows = [r.split(",") for r in f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.file.name)
+        sm, smax, power, reasons = [], [], [], set()
+        for r in rows:
+            r = [c.strip() for c in r]
+            if len(r) < 9 or r[0] != str(self.gpu_index):
+                continue
+            try:
+                sm.append(float(r[1]))
+                smax.append(float(r[2]))
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for name, val in zip(REASON_NAMES, r[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "power_w_max": max(power), "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gqa_mqa_kv_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per split-kernel launch from the committed ncu summary, if it
+    was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        ent = rec.get(workload)
+        if ent and ent.get("kernel_source_hash") == kernel_source_hash():
+            return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+def cpu_oracle_sample(w, inp, seconds: float):
+    """Time the fp64 oracle on the first sequences of the batch (all query
+    heads), sized to take about `seconds` of wall clock."""
+    import oracle
+
+    lens = inp["seq_lens"]
+    H_Q = w.H_Q
+    # calibrate on one (b, h) pair of the first non-empty sequence
+    b0 = int(torch.nonzero(lens > 0)[0])
+    t0 = time.perf_counter()
+    oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=[(b0, 0)], n_threads=1)
+    per_token_head = max((time.perf_counter() - t0) / max(int(lens[b0]), 1), 1e-9)
+    threads = oracle.hardware_threads()
+    budget = seconds * threads / per_token_head  # token-heads the sample may cover
+    pairs, tok_heads, b = [], 0, 0
+    while b < w.B and (tok_heads < budget or not pairs):
+        pairs += [(b, h) for h in range(H_Q)]
+        tok_heads += int(lens[b]) * H_Q
+        b += 1
+    t0 = time.perf_counter()
+    oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=pairs, n_threads=0)
+    dt = time.perf_counter() - t0
+    e = 2 if w.dtype == "bf16" else 4
+    nb = b
+    sample_bytes = (int(lens[:nb].to(torch.int64).sum()) * w.H_KV * w.D * e * 2
+                    + nb * H_Q * w.D * e + nb * H_Q * w.D * 4)
+    return {
+        "value": sample_bytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+        "sample": f"sequences 0..{nb - 1} of {w.B} (all {H_Q} query heads, "
+                  f"{int(lens[:nb].sum())} cached tokens), fp64, {dt:.2f} s wall",
+        "seconds": dt, "us_per_full_step_equiv": dt * 1e6 * (algorithmic_bytes(w, lens) / sample_bytes),
+    }
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    step_results = []
+    for _ in range(args.warmup):
+        pass  # the oracle has no warm state; warm-up steps are no-ops by construction
+    t_start = time.perf_counter()
+    last = None
+    for _ in range(args.steps):
+        last = cpu_oracle_sample(w, inp, args.cpu_sample_seconds / max(args.steps, 1))
+        step_results.append(last)
+    total = time.perf_counter() - t_start
+    value = statistics.median(r["value"] for r in step_results)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": total * 1e3 / max(args.steps, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(w, args.gpus),
+        "cpu_baseline": {k: last[k] for k in ("kind", "cores", "sample")} | {"value": value, "unit": "GB/s"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU arm
+
+def workload_config(w, n):
+    return {"workload": w.name, "B": w.B, "H_Q": w.H_Q, "H_KV": w.H_KV, "head_dim": w.D,
+            "seq_len": w.seq_len, "ragged": w.ragged, "page_size": w.page_size,
+            "kv_dtype": w.dtype, "global_batch": w.B * n,
+            "l2": "inputs larger than L2 (no flush)" if w.seq_len * w.B * w.H_KV * w.D * 4 > 2 * 126e6
+                  else "L2 flushed before every step",
+            "parallelism": f"dp{n} (independent batch per GPU, no collective)"}
+
+
+def run_ours(args):
+    import gqa_mqa_kv_b200 as gq
+
+    world, rank, local = dist_env()
+    if world != args.gpus and world > 1:
+        print(f"WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    w = WORKLOADS[args.workload]
+    inp = make_inputs(w)
+    lens_host = inp["seq_lens"]
+    step_bytes = algorithmic_bytes(w, lens_host)
+    paged = bool(w.page_size)
+    kk = inp["k_paged"] if paged else inp["k"]
+    vv = inp["v_paged"] if paged else inp["v"]
+    q = inp["q"].to(dev)
+    k = kk.to(dev)
+    v = vv.to(dev)
+    lens = lens_host.to(dev)
+    table = inp["block_table"].to(dev) if paged else None
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    params = gq.make_params(q, k, lens, table)
+    ws = torch.zeros(gq.workspace_bytes(params), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    big = w.seq_len * w.B * w.H_KV * w.D * 4 > 2 * 126e6
+    flush = None if big else torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        if flush is not None:
+            flush.zero_()
+        gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+
+    with ClockSampler(local) as clocks:
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < args.soak_seconds:
+            for _ in range(50):
+                step()
+            torch.cuda.synchronize(dev)
+        # ------------------------------------------------ timed region
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        ev_begin = torch.cuda.Event(enable_timing=True)
+        ev_end = torch.cuda.Event(enable_timing=True)
+        split_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)]
+        step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(args.steps)] if flush is not None else None
+        ev_begin.record(stream)
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+                step_ev[i][0].record(stream)
+            gq.gqa_decode_timed(split_ev[i], q, k, v, lens, table, scale=w.softmax_scale, out=out,
+                                workspace=ws, stream=stream)
+            if flush is not None:
+                step_ev[i][1].record(stream)
+        ev_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        # ------------------------------------------------ end of timed region
+    # Whole region when nothing else runs in it; per-step sums when an L2 flush
+    # sits between the steps.
+    elapsed_ms = (ev_begin.elapsed_time(ev_end) if step_ev is None
+                  else sum(a.elapsed_time(b) for a, b in step_ev))
+    split_ms = statistics.mean(a.elapsed_time(b) for a, b in split_ev)
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
+    split_ms_max = max_over_ranks(split_ms, dist, dev)
+    status = gq.read_status(ws)
+
+    # ---------------------------------------------------- end to end through the public API
+    q_host = inp["q"].pin_memory()
+    lens_pin = lens_host.pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = q_host.numel() * q_host.element_size() + lens_pin.numel() * 4
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        q.copy_(q_host, non_blocking=True)
+        lens.copy_(lens_pin, non_blocking=True)
+        gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws, stream=stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / args.e2e_steps
+
+    peak, peak_kind = hbm_peak()
+    ms_per_step = elapsed_ms / args.steps
+    value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
+    achieved = step_bytes / (split_ms_max * 1e-3) / 1e9
+    traffic = recorded_traffic(w.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
+        "pct_of_hbm_peak": 100.0 * (value / world) / peak, "peak_kind": peak_kind,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": workload_config(w, world),
+        "algorithmic_bytes_per_step_per_gpu": step_bytes,
+        "clocks": clocks.summary(),
+        "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                "us_per_step": e2e_ms * 1e3, "h2d_bytes_per_step": world * h2d,
+                "d2h_bytes_per_step": world * d2h,
+                "path": "pinned q and seq_lens copied in, gqa_decode, out copied back, every step; "
+                        "KV cache resident in HBM"},
+        "gpu_launches": 2 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": traffic,
+                     "kernel": "split-KV decode kernel (combine excluded)",
+                     "split_kernel_us": split_ms_max * 1e3,
+                     "peak_note": f"{peak_kind} HBM copy bandwidth"},
+        "device_status_flags": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w, inp, args.cpu_sample_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,381 @@
+// gqa_decode.cu -- host side of the C ABI declared in include/gqa_decode.h.
+//
+// Validates arguments, picks the kernel (tensor-core split kernel for bf16
+// with groups of up to 64 query heads, CUDA-core split kernel otherwise),
+// encodes the TMA tensor maps, and enqueues split + combine on the caller's
+// stream with programmatic dependent launch so the combine grid's launch
+// overlaps the split grid's tail.  No allocation, no host synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <set>
+#include <utility>
+
+#include "gqa_decode.h"
+#include "combine.cuh"
+#include "split_mma.cuh"
+#include "split_simt.cuh"
+
+namespace {
+
+using namespace gqa;
+
+constexpr size_t kHeaderBytes = 256;  // status word lives at offset 0
+constexpr int kSimtCtasPerSm = 4;
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+    int sms = 0;
+    int smem_optin = 0;
+};
+
+gqa_status device_info(DeviceInfo* info) {
+    static std::mutex mu;
+    static DeviceInfo cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev].sms == 0) {
+        DeviceInfo d;
+        if (cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+                cudaSuccess)
+            return GQA_ERR_CUDA;
+        cache[dev] = d;
+    }
+    *info = cache[dev];
+    return GQA_OK;
+}
+
+bool aligned(const void* p, size_t n) { return reinterpret_cast<uintptr_t>(p) % n == 0; }
+
+size_t round_up(size_t x, size_t m) { return (x + m - 1) / m * m; }
+
+gqa_status validate_params(const gqa_decode_params* p) {
+    if (p == nullptr) return GQA_ERR_INVALID;
+    if (p->B < 0 || p->H_Q <= 0 || p->H_KV <= 0 || p->max_seq_len < 0) return GQA_ERR_INVALID;
+    if (p->H_Q % p->H_KV != 0) return GQA_ERR_INVALID;
+    if (p->qkv_dtype != GQA_BF16 && p->qkv_dtype != GQA_F32) return GQA_ERR_INVALID;
+    if (p->out_dtype != GQA_BF16 && p->out_dtype != GQA_F32) return GQA_ERR_INVALID;
+    if (p->page_size != 0 && p->page_size != kTile) return GQA_ERR_UNSUPPORTED;
+    if (p->head_dim != 64 && p->head_dim != 128) return GQA_ERR_UNSUPPORTED;
+    if (p->page_size == 0) {
+        if (p->max_blocks_per_seq != 0 || p->num_blocks != 0) return GQA_ERR_INVALID;
+    } else {
+        if (p->max_blocks_per_seq <= 0 || p->num_blocks <= 0) return GQA_ERR_INVALID;
+        if (static_cast<int64_t>(p->max_seq_len) > static_cast<int64_t>(p->max_blocks_per_seq) * kTile)
+            return GQA_ERR_INVALID;
+    }
+    // 64-bit element offsets are used throughout; keep 32-bit grid / head math safe.
+    if (static_cast<int64_t>(p->B) * p->H_Q > (int64_t(1) << 30)) return GQA_ERR_UNSUPPORTED;
+    return GQA_OK;
+}
+
+bool use_tensor_cores(const gqa_decode_params* p) {
+    return p->qkv_dtype == GQA_BF16 && p->H_Q / p->H_KV <= 64;
+}
+
+int grid_for(const gqa_decode_params* p, const DeviceInfo& dev) {
+    return use_tensor_cores(p) ? dev.sms : dev.sms * kSimtCtasPerSm;
+}
+
+size_t workspace_for(const gqa_decode_params* p, int grid) {
+    const size_t R = static_cast<size_t>(p->H_Q / p->H_KV);
+    const size_t slots = 2 * static_cast<size_t>(grid);
+    return kHeaderBytes + round_up(slots * R * p->head_dim * sizeof(float), 256) +
+           round_up(slots * R * sizeof(float), 256);
+}
+
+// ------------------------------------------------------------------ TMA maps
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault,
+                                             &qr) == cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    });
+    return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
+bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                 const uint64_t* strides_bytes, const uint32_t* box) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t bx[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) s[i] = strides_bytes[i];
+    }
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+              const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launches
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_chained(void (*kernel)(KArgs...), int grid, int block, size_t smem,
+                           cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(block));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_smem(const void* kernel, int bytes) {
+    static std::mutex mu;
+    static std::set<std::pair<const void*, int>> done;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count({kernel, dev})) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) done.insert({kernel, dev});
+    return e;
+}
+
+struct Buffers {
+    const void* q;
+    const void* k;
+    const void* v;
+};
+
+template <int D, int HG, bool PAGED, bool OUTB>
+cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArgs args,
+                       const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
+    using C = MmaCfg<D, HG>;
+    const int R = p->H_Q / p->H_KV;
+    int stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
+    if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    args.n_stages = stages;
+    args.q_rows = R < 16 ? R : 16;
+    args.q_groups = (R + 15) / 16;
+
+    CUtensorMap tmQ, tmK, tmV;
+    const uint64_t row = static_cast<uint64_t>(D) * 2;
+    {
+        const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(p->H_Q),
+                                  static_cast<uint64_t>(p->B)};
+        const uint64_t strides[2] = {row, row * p->H_Q};
+        const uint32_t box[3] = {64, static_cast<uint32_t>(args.q_rows), 1};
+        *encode_ok = encode_bf16(&tmQ, buf.q, 3, dims, strides, box);
+    }
+    const uint32_t box4[4] = {64, 1, static_cast<uint32_t>(kTile), 1};
+    if (*encode_ok) {
+        uint64_t dims[4], strides[3];
+        dims[0] = D;
+        dims[1] = p->H_KV;
+        strides[0] = row;
+        strides[1] = row * p->H_KV;
+        if (PAGED) {
+            dims[2] = kTile;
+            dims[3] = p->num_blocks;
+        } else {
+            dims[2] = p->max_seq_len > 0 ? p->max_seq_len : 1;
+            dims[3] = p->B;
+        }
+        strides[2] = strides[1] * dims[2];
+        *encode_ok = encode_bf16(&tmK, buf.k, 4, dims, strides, box4) &&
+                     encode_bf16(&tmV, buf.v, 4, dims, strides, box4);
+    }
+    if (!*encode_ok) return cudaErrorInvalidValue;
+    auto kernel = split_mma_kernel<D, HG, PAGED, OUTB>;
+    const int smem = C::smem_bytes(stages);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), smem);
+    if (e != cudaSuccess) return e;
+    return launch_chained(kernel, grid, C::THREADS, smem, stream, tmQ, tmK, tmV, args);
+}
+
+template <int D, bool PAGED, bool OUTB>
+cudaError_t launch_mma_groups(const gqa_decode_params* p, const Buffers& buf,
+                              const KernelArgs& args, const DeviceInfo& dev, int grid,
+                              cudaStream_t stream, bool* encode_ok) {
+    const int R = p->H_Q / p->H_KV;
+    if (R <= 16) return launch_mma<D, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (R <= 32) return launch_mma<D, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    return launch_mma<D, 4, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+}
+
+template <typename T, int D, bool PAGED, bool OUTB>
+cudaError_t launch_simt(const Buffers& buf, const KernelArgs& args, int grid, cudaStream_t stream) {
+    return launch_chained(split_simt_kernel<T, D, PAGED, OUTB>, grid, 32 * kSimtWarps, 0, stream,
+                          static_cast<const T*>(buf.q), static_cast<const T*>(buf.k),
+                          static_cast<const T*>(buf.v), args);
+}
+
+template <int D, bool PAGED, bool OUTB>
+cudaError_t launch_split(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
+                         const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
+    if (use_tensor_cores(p)) return launch_mma_groups<D, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (p->qkv_dtype == GQA_F32) return launch_simt<float, D, PAGED, OUTB>(buf, args, grid, stream);
+    return launch_simt<__nv_bfloat16, D, PAGED, OUTB>(buf, args, grid, stream);
+}
+
+template <int D, bool OUTB>
+cudaError_t launch_all(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
+                       const DeviceInfo& dev, int grid, cudaStream_t stream, cudaEvent_t ev0,
+                       cudaEvent_t ev1, bool* encode_ok) {
+    cudaError_t e;
+    if (ev0 && (e = cudaEventRecord(ev0, stream)) != cudaSuccess) return e;
+    e = p->page_size ? launch_split<D, true, OUTB>(p, buf, args, dev, grid, stream, encode_ok)
+                     : launch_split<D, false, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (e != cudaSuccess) return e;
+    if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return e;
+    return launch_chained(combine_kernel<D, OUTB>, p->B, 256, 0, stream, args, grid);
+}
+
+gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const void* v,
+               const int32_t* seq_lens, const int32_t* block_table, float scale, void* out,
+               void* workspace, size_t workspace_bytes, void* stream_ptr, void* ev0, void* ev1) {
+    gqa_status st = validate_params(p);
+    if (st != GQA_OK) return st;
+    if (p->B == 0) return GQA_OK;
+    if (!q || !k || !v || !seq_lens || !out) return GQA_ERR_INVALID;
+    if ((p->page_size != 0) != (block_table != nullptr)) return GQA_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 8) ||
+        !aligned(seq_lens, 4) || (block_table && !aligned(block_table, 4)))
+        return GQA_ERR_INVALID;
+    if (!(scale == scale)) return GQA_ERR_INVALID;  // NaN scale
+
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != GQA_OK) return st;
+    const int grid = grid_for(p, dev);
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < workspace_for(p, grid))
+        return GQA_ERR_WORKSPACE;
+
+    const int R = p->H_Q / p->H_KV;
+    const size_t slots = 2 * static_cast<size_t>(grid);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    KernelArgs args;
+    std::memset(&args, 0, sizeof args);
+    args.seq_lens = seq_lens;
+    args.block_table = block_table;
+    args.B = p->B;
+    args.H_Q = p->H_Q;
+    args.H_KV = p->H_KV;
+    args.R = R;
+    args.max_len = p->max_seq_len;
+    args.S_max = p->page_size ? 0 : p->max_seq_len;
+    args.max_blocks = p->max_blocks_per_seq;
+    args.num_blocks = p->num_blocks;
+    args.sl2 = scale * 1.4426950408889634f;  // log2(e): exponentials are taken base 2
+    args.out = out;
+    args.status = reinterpret_cast<uint32_t*>(ws);
+    args.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes);
+    args.ws_lse = reinterpret_cast<float*>(
+        ws + kHeaderBytes + round_up(slots * R * p->head_dim * sizeof(float), 256));
+
+    const Buffers buf{q, k, v};
+    cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
+    cudaEvent_t e0 = static_cast<cudaEvent_t>(ev0), e1 = static_cast<cudaEvent_t>(ev1);
+    bool encode_ok = true;
+    cudaError_t e;
+    const bool outb = p->out_dtype == GQA_BF16;
+    if (p->head_dim == 64)
+        e = outb ? launch_all<64, true>(p, buf, args, dev, grid, stream, e0, e1, &encode_ok)
+                 : launch_all<64, false>(p, buf, args, dev, grid, stream, e0, e1, &encode_ok);
+    else
+        e = outb ? launch_all<128, true>(p, buf, args, dev, grid, stream, e0, e1, &encode_ok)
+                 : launch_all<128, false>(p, buf, args, dev, grid, stream, e0, e1, &encode_ok);
+    if (!encode_ok) return GQA_ERR_INVALID;
+    return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes) {
+    if (bytes == nullptr) return GQA_ERR_INVALID;
+    gqa_status st = validate_params(params);
+    if (st != GQA_OK) return st;
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != GQA_OK) return st;
+    *bytes = workspace_for(params, grid_for(params, dev));
+    return GQA_OK;
+}
+
+gqa_status gqa_decode(const gqa_decode_params* params, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, const int32_t* block_table,
+                      float scale, void* out, void* workspace, size_t workspace_bytes,
+                      void* stream) {
+    return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, workspace,
+               workspace_bytes, stream, nullptr, nullptr);
+}
+
+gqa_status gqa_decode_timed(const gqa_decode_params* params, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* seq_lens,
+                            const int32_t* block_table, float scale, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream, void* split_begin,
+                            void* split_end) {
+    return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, workspace,
+               workspace_bytes, stream, split_begin, split_end);
+}
+
+gqa_status gqa_read_status(const void* workspace, void* stream, uint32_t* flags, int clear) {
+    if (workspace == nullptr || flags == nullptr) return GQA_ERR_INVALID;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t host = 0;
+    if (cudaMemcpyAsync(&host, workspace, sizeof host, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return GQA_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GQA_ERR_CUDA;
+    if (clear) {
+        if (cudaMemsetAsync(const_cast<void*>(workspace), 0, sizeof host, s) != cudaSuccess ||
+            cudaStreamSynchronize(s) != cudaSuccess)
+            return GQA_ERR_CUDA;
+    }
+    *flags = host;
+    return GQA_OK;
+}
+
+uint64_t gqa_kv_cache_bytes(int64_t layers, int64_t tokens, int64_t H_KV, int64_t head_dim,
+                            int64_t elem_bytes) {
+    if (layers < 0 || tokens < 0 || H_KV < 0 || head_dim < 0 || elem_bytes < 0) return 0;
+    return 2ull * static_cast<uint64_t>(layers) * static_cast<uint64_t>(tokens) *
+           static_cast<uint64_t>(H_KV) * static_cast<uint64_t>(head_dim) *
+           static_cast<uint64_t>(elem_bytes);
+}
+
+const char* gqa_status_string(gqa_status status) {
+    switch (status) {
+        case GQA_OK: return "ok";
+        case GQA_ERR_INVALID: return "invalid argument";
+        case GQA_ERR_UNSUPPORTED: return "unsupported configuration";
+        case GQA_ERR_CUDA: return "CUDA error";
+        case GQA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    }
+    return "unknown status";
+}
+
+int gqa_version(void) { return GQA_DECODE_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,153 @@
+// split_simt.cuh -- CUDA-core split-KV decode kernel (fp32 or bf16 inputs).
+//
+// The path for fp32 caches and for groups wider than 64 query heads, where
+// the tensor-core kernel does not apply.  Same tile schedule and outputs as
+// split_mma.cuh: every segment writes the final output or a partial
+// (o / l, m + log2 l).  Four warps take interleaved tokens; each lane holds
+// D/32 elements of every row; query heads are handled 8 at a time.  fp32
+// arithmetic throughout ("Grouped-Query Attention (GQA) and Multi-Query
+// Attention (MQA): Mathematical Foundations, ...", section 2, Head_i).
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+
+namespace gqa {
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+constexpr int kSimtWarps = 4;
+constexpr int kSimtHeads = 8;
+
+template <typename T, int D, bool PAGED, bool OUT_BF16>
+__global__ void __launch_bounds__(32 * kSimtWarps)
+    split_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                      const KernelArgs a) {
+    constexpr int DPL = D / 32;
+    constexpr int HC = kSimtHeads;
+    __shared__ Plan plan;
+    __shared__ float sm_m[kSimtWarps][HC];
+    __shared__ float sm_l[kSimtWarps][HC];
+    __shared__ float sm_o[kSimtWarps][HC][D];
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (warp == 0) make_plan(a, &plan);
+    __syncthreads();
+    const int64_t lo = plan.lo, hi = plan.hi;
+    if (lo >= hi) return;
+    Walk w{plan.b, plan.kv, plan.tile, plan.n_b, plan.L};
+
+    bool first = true;
+    int64_t gi = lo;
+    while (gi < hi) {
+        const int seg_tiles = static_cast<int>(min(static_cast<int64_t>(w.n_b - w.tile), hi - gi));
+        const bool whole = (w.tile == 0) && (seg_tiles == w.n_b);
+        const int64_t slot = first ? 2 * static_cast<int64_t>(blockIdx.x) : 2 * static_cast<int64_t>(blockIdx.x) + 1;
+        const int t_begin = w.tile * kTile;
+        const int t_end = min((w.tile + seg_tiles) * kTile, w.L);
+
+        for (int hc = 0; hc < a.R; hc += HC) {
+            const int nh = min(HC, a.R - hc);
+            float qr[HC][DPL], o[HC][DPL], m[HC], l[HC];
+#pragma unroll
+            for (int j = 0; j < HC; ++j) {
+                const int64_t qrow = static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + hc + j;
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) {
+                    qr[j][i] = j < nh ? to_f32(q[qrow * D + lane + 32 * i]) : 0.f;
+                    o[j][i] = 0.f;
+                }
+                m[j] = NEG_INF;
+                l[j] = 0.f;
+            }
+            for (int tok = t_begin + warp; tok < t_end; tok += kSimtWarps) {
+                float kr[DPL], vr[DPL];
+                int64_t row;
+                bool live = true;
+                if constexpr (PAGED) {
+                    const int page = __ldg(a.block_table + static_cast<int64_t>(w.b) * a.max_blocks + tok / kTile);
+                    live = page >= 0 && page < a.num_blocks;
+                    if (!live && lane == 0) atomicOr(a.status, kFlagBadBlock);
+                    row = (static_cast<int64_t>(live ? page : 0) * kTile + tok % kTile) * a.H_KV + w.kv;
+                } else {
+                    row = (static_cast<int64_t>(w.b) * a.S_max + tok) * a.H_KV + w.kv;
+                }
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) {
+                    kr[i] = live ? to_f32(k[row * D + lane + 32 * i]) : 0.f;  // a bad page reads as zeros
+                    vr[i] = live ? to_f32(v[row * D + lane + 32 * i]) : 0.f;
+                }
+#pragma unroll
+                for (int j = 0; j < HC; ++j) {
+                    float s = 0.f;
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) s = fmaf(qr[j][i], kr[i], s);
+#pragma unroll
+                    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+                    s *= a.sl2;
+                    const float mn = fmaxf(m[j], s);
+                    const float al = exp2f(m[j] - mn);
+                    const float p = exp2f(s - mn);
+                    l[j] = l[j] * al + p;
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) o[j][i] = fmaf(p, vr[i], o[j][i] * al);
+                    m[j] = mn;
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < HC; ++j) {
+                if (lane == 0) {
+                    sm_m[warp][j] = m[j];
+                    sm_l[warp][j] = l[j];
+                }
+#pragma unroll
+                for (int i = 0; i < DPL; ++i) sm_o[warp][j][lane + 32 * i] = o[j][i];
+            }
+            __syncthreads();
+            for (int idx = threadIdx.x; idx < nh * D; idx += blockDim.x) {
+                const int j = idx / D, d = idx % D;
+                float M = NEG_INF;
+#pragma unroll
+                for (int ww = 0; ww < kSimtWarps; ++ww) M = fmaxf(M, sm_m[ww][j]);
+                const float ref = M == NEG_INF ? 0.f : M;
+                float L = 0.f, O = 0.f;
+#pragma unroll
+                for (int ww = 0; ww < kSimtWarps; ++ww) {
+                    const float e = exp2f(sm_m[ww][j] - ref);
+                    L += sm_l[ww][j] * e;
+                    O += sm_o[ww][j][d] * e;
+                }
+                const int r = hc + j;
+                if (whole) {
+                    const int64_t oi = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + r) * D + d;
+                    if constexpr (OUT_BF16)
+                        static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(O / L);
+                    else
+                        static_cast<float*>(a.out)[oi] = O / L;
+                } else {
+                    a.ws_o[(slot * a.R + r) * D + d] = O / L;
+                    if (d == 0) a.ws_lse[slot * a.R + r] = M + log2f(L);
+                }
+            }
+            __syncthreads();
+        }
+        first = false;
+        gi += seg_tiles;
+        w.tile += seg_tiles - 1;
+        if (gi < hi) w.advance(a);
+    }
+}
+
+}  // namespace gqa

@@ -1,0 +1,173 @@
+/*
+ * gqa_decode.h -- C ABI of the B200 grouped-query attention decode library.
+ *
+ * One call computes one decode step of one attention layer: every query head
+ * of every sequence attends, with a single new query token, over that
+ * sequence's cached keys and values.  Key/value head g of the cache serves
+ * the R = H_Q / H_KV query heads h with g = floor(h / R) and is read from HBM
+ * once for all of them.
+ *
+ * Defining passages (cited by page title and section):
+ *   [LLMS] "Grouped-Query Attention (GQA) and Multi-Query Attention (MQA):
+ *          Mathematical Foundations, Arithmetic Intensity, and KV-Cache
+ *          Scaling Mechanics" (llms.blog)
+ *          - section 2, "Grouped-Query Attention": group size R = H_Q / G,
+ *            H_KV = G, group index g(i) = floor((i-1)/R) + 1 (1-based), and
+ *            Head_i = softmax(Q_i K_{g(i)}^T / sqrt(d_k) + M) V_{g(i)}.
+ *            G = H_Q is MHA, G = 1 is MQA.
+ *          - section 2, the K, V in R^{b x s x G x d_k} layout that the
+ *            contiguous cache below follows.
+ *          - section 1, "KV Cache Memory Footprint": the cache-size formula.
+ *          - Sources list: PagedAttention (vLLM), the origin of the paged
+ *            cache layout.
+ *   [AIT]  "Grouped-Query Attention Shares Keys Without Sharing Every Query"
+ *          (aitamer.news): the cache estimate 2 x layers x tokens x groups x
+ *          head dim x bytes per element, and "paging" as a serving layout.
+ *
+ * What one call computes, for b < B and h < H_Q, with g = h / R, L_b the
+ * clamped seq_lens[b], and t < L_b:
+ *     s_t = scale * <q[b,h,:], K_b[t,g,:]>
+ *     out[b,h,:] = sum_t softmax(s)_t * V_b[t,g,:]
+ * The single query is the newest position, so the causal mask keeps all L_b
+ * cached tokens (the current token's key/value already appended) and drops
+ * positions >= L_b.  L_b = 0 gives out[b,h,:] = 0.
+ *
+ * Ownership and threading: the caller allocates every buffer (inputs, out
+ * and workspace).  The library allocates no device memory, never
+ * synchronises the stream in gqa_decode, and enqueues its kernels on the
+ * caller's stream.  Calls on different streams must not share a workspace.
+ * All entry points are thread-safe.
+ */
+#ifndef GQA_DECODE_H
+#define GQA_DECODE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GQA_DECODE_VERSION 1
+
+typedef enum gqa_status {
+    GQA_OK = 0,
+    GQA_ERR_INVALID = 1,     /* an argument is invalid; nothing was launched */
+    GQA_ERR_UNSUPPORTED = 2, /* valid but not implemented (e.g. head_dim 96) */
+    GQA_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed */
+    GQA_ERR_WORKSPACE = 4    /* workspace missing, misaligned or too small */
+} gqa_status;
+
+typedef enum gqa_dtype {
+    GQA_BF16 = 0,
+    GQA_F32 = 1
+} gqa_dtype;
+
+/* Device status flags, accumulated (bitwise OR) in the workspace. */
+#define GQA_FLAG_SEQ_LEN_CLAMPED 1u   /* a seq_lens entry was < 0 or > max_seq_len */
+#define GQA_FLAG_BAD_BLOCK 2u         /* a live block_table entry was outside [0, num_blocks) */
+#define GQA_FLAG_TIMEOUT 4u           /* an internal pipeline wait gave up; outputs invalid */
+
+/*
+ * Problem description.  All counts are element counts.
+ *
+ *  B, H_Q, H_KV     batch rows, query heads, key/value heads.  H_Q % H_KV == 0
+ *                   ([LLMS] section 2: R = H_Q / G is a whole number).
+ *  head_dim         d_k = d_v; 64 or 128.
+ *  max_seq_len      contiguous cache: its sequence capacity S_max (the second
+ *                   dimension of k_cache/v_cache).  Paged cache: the largest
+ *                   allowed length, <= max_blocks_per_seq * page_size.
+ *                   seq_lens entries are clamped to [0, max_seq_len].
+ *  page_size        0 for a contiguous cache, 64 for a paged cache.
+ *  max_blocks_per_seq, num_blocks   paged cache only (else 0): columns of the
+ *                   block table, and pages held by k_cache/v_cache.
+ *  qkv_dtype        element type of q, k_cache and v_cache.
+ *  out_dtype        element type of out.  F32 keeps the fp32 accumulator.
+ */
+typedef struct gqa_decode_params {
+    int32_t B;
+    int32_t H_Q;
+    int32_t H_KV;
+    int32_t head_dim;
+    int32_t max_seq_len;
+    int32_t page_size;
+    int32_t max_blocks_per_seq;
+    int32_t num_blocks;
+    gqa_dtype qkv_dtype;
+    gqa_dtype out_dtype;
+} gqa_decode_params;
+
+/*
+ * Bytes of workspace gqa_decode needs for these parameters on the CURRENT
+ * CUDA device (the size depends on its SM count).  Writes *bytes.
+ * The workspace holds one status word and the split-KV partial results.
+ * Zero-fill it once after allocating it (the status word must start at 0);
+ * later calls need no clearing.
+ */
+gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes);
+
+/*
+ * One decode step, enqueued on `stream` (a cudaStream_t; NULL = legacy default).
+ *
+ * Device pointers, row-major, innermost dimension last:
+ *   q            [B, H_Q, head_dim]                       qkv_dtype, 16-byte aligned
+ *   k_cache,     contiguous: [B, max_seq_len, H_KV, head_dim]
+ *   v_cache      paged:      [num_blocks, 64, H_KV, head_dim]
+ *                qkv_dtype, 16-byte aligned.  Rows at positions >= L_b are
+ *                never used (they may hold anything, NaN included).
+ *   seq_lens     int32 [B], cached tokens per sequence including the newest.
+ *   block_table  int32 [B, max_blocks_per_seq] for a paged cache, else NULL.
+ *                Token t of sequence b lives in page block_table[b][t / 64],
+ *                slot t % 64.  Entries past ceil(L_b / 64) are not read.
+ *   scale        softmax scale, usually 1/sqrt(head_dim) ([LLMS] section 2).
+ *   out          [B, H_Q, head_dim] out_dtype, 8-byte aligned.
+ *   workspace    >= gqa_decode_workspace_size bytes, 256-byte aligned.
+ *
+ * Errors: argument errors return GQA_ERR_INVALID / GQA_ERR_UNSUPPORTED /
+ * GQA_ERR_WORKSPACE before anything is enqueued.  seq_lens and block_table
+ * are device data and are not read on the host: out-of-range lengths are
+ * clamped and out-of-range pages read as zeros, and both raise a flag in the
+ * workspace status word (see gqa_read_status).  The kernels never trap.
+ * A launch failure returns GQA_ERR_CUDA.
+ */
+gqa_status gqa_decode(const gqa_decode_params* params, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, const int32_t* block_table,
+                      float scale, void* out, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
+ * gqa_decode that also records `split_begin` just before and `split_end`
+ * just after the split-KV kernel (both cudaEvent_t, either may be NULL).
+ * For measuring the dominant kernel alone; the result equals gqa_decode's.
+ */
+gqa_status gqa_decode_timed(const gqa_decode_params* params, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* seq_lens,
+                            const int32_t* block_table, float scale, void* out, void* workspace,
+                            size_t workspace_bytes, void* stream, void* split_begin,
+                            void* split_end);
+
+/*
+ * Reads the workspace status word (GQA_FLAG_* bits) into *flags after
+ * synchronising `stream`; clears it when `clear` is non-zero.
+ */
+gqa_status gqa_read_status(const void* workspace, void* stream, uint32_t* flags, int clear);
+
+/*
+ * KV-cache size in bytes: 2 x layers x tokens x H_KV x head_dim x elem_bytes
+ * ([LLMS] section 1 "KV Cache Memory Footprint"; [AIT] cache estimate).
+ * tokens counts every cached token of every sequence.  Host-only, pure.
+ */
+uint64_t gqa_kv_cache_bytes(int64_t layers, int64_t tokens, int64_t H_KV, int64_t head_dim,
+                            int64_t elem_bytes);
+
+/* Static string for a status code. */
+const char* gqa_status_string(gqa_status status);
+
+/* GQA_DECODE_VERSION of the loaded library. */
+int gqa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GQA_DECODE_H */
