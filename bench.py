@@ -105,16 +105,20 @@ def hbm_peak():
 class ClockSampler:
     """nvidia-smi clock/throttle sampling in the background (200 ms period)."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu_index = gpu_index
+    def __init__(self, device: torch.device):
+        try:
+            self.uuid = "GPU-" + str(torch.cuda.get_device_properties(device).uuid)
+        except Exception:
+            self.uuid = None
         self.proc = None
         self.file = None
 
     def __enter__(self):
         try:
             self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            sel = ["-i", self.uuid] if self.uuid else []
             self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
+                ["nvidia-smi", *sel, f"--query-gpu={CLOCK_FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -138,7 +142,7 @@ class ClockSampler:
         sm, smax, power, reasons = [], [], [], set()
         for r in rows:
             r = [c.strip() for c in r]
-            if len(r) < 9 or r[0] != str(self.gpu_index):
+            if len(r) < 9:
                 continue
             try:
                 sm.append(float(r[1]))
@@ -188,29 +192,37 @@ def cpu_oracle_sample(w, inp, seconds: float):
 
     lens = inp["seq_lens"]
     H_Q = w.H_Q
-    # calibrate on one (b, h) pair of the first non-empty sequence
+    threads = oracle.hardware_threads()
+    # calibrate on all heads of the first non-empty sequence
     b0 = int(torch.nonzero(lens > 0)[0])
     t0 = time.perf_counter()
-    oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=[(b0, 0)], n_threads=1)
-    per_token_head = max((time.perf_counter() - t0) / max(int(lens[b0]), 1), 1e-9)
-    threads = oracle.hardware_threads()
-    budget = seconds * threads / per_token_head  # token-heads the sample may cover
-    pairs, tok_heads, b = [], 0, 0
-    while b < w.B and (tok_heads < budget or not pairs):
-        pairs += [(b, h) for h in range(H_Q)]
-        tok_heads += int(lens[b]) * H_Q
-        b += 1
-    t0 = time.perf_counter()
-    oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=pairs, n_threads=0)
-    dt = time.perf_counter() - t0
+    oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale,
+                      pairs=[(b0, h) for h in range(H_Q)], n_threads=0)
+    per_token = max((time.perf_counter() - t0) / max(int(lens[b0]), 1), 1e-12)  # all heads, all threads
+    est_full = per_token * int(lens.sum())
+    if est_full <= seconds:
+        nb, reps = w.B, max(1, min(3, int(seconds / max(est_full, 1e-3))))
+    else:
+        nb, acc = 0, 0.0
+        while nb < w.B and (acc < seconds or nb == 0):
+            acc += per_token * int(lens[nb])
+            nb += 1
+        reps = 1
+    pairs = [(b, h) for b in range(nb) for h in range(H_Q)]
+    times = []
+    for _ in range(reps):
+        t0 = time.perf_counter()
+        oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=pairs, n_threads=0)
+        times.append(time.perf_counter() - t0)
+    dt = statistics.median(times)
     e = 2 if w.dtype == "bf16" else 4
-    nb = b
     sample_bytes = (int(lens[:nb].to(torch.int64).sum()) * w.H_KV * w.D * e * 2
                     + nb * H_Q * w.D * e + nb * H_Q * w.D * 4)
+    what = "the whole step" if nb == w.B else f"sequences 0..{nb - 1} of {w.B}"
     return {
         "value": sample_bytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-        "sample": f"sequences 0..{nb - 1} of {w.B} (all {H_Q} query heads, "
-                  f"{int(lens[:nb].sum())} cached tokens), fp64, {dt:.2f} s wall",
+        "sample": f"{what} (all {H_Q} query heads, {int(lens[:nb].sum())} cached tokens), fp64, "
+                  f"median of {reps} run(s), {dt:.2f} s each",
         "seconds": dt, "us_per_full_step_equiv": dt * 1e6 * (algorithmic_bytes(w, lens) / sample_bytes),
     }
 
@@ -292,20 +304,18 @@ def run_ours(args):
         step()
     torch.cuda.synchronize(dev)
 
-    with ClockSampler(local) as clocks:
+    with ClockSampler(dev) as clocks:
         t_soak = time.perf_counter()
         while time.perf_counter() - t_soak < args.soak_seconds:
             for _ in range(50):
                 step()
             torch.cuda.synchronize(dev)
-        # ------------------------------------------------ timed region
+        # ------------------------------------------------ timed region: the headline
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
         ev_begin = torch.cuda.Event(enable_timing=True)
         ev_end = torch.cuda.Event(enable_timing=True)
-        split_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-                    for _ in range(args.steps)]
         step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                    for _ in range(args.steps)] if flush is not None else None
         ev_begin.record(stream)
@@ -313,11 +323,25 @@ def run_ours(args):
             if flush is not None:
                 flush.zero_()
                 step_ev[i][0].record(stream)
-            gq.gqa_decode_timed(split_ev[i], q, k, v, lens, table, scale=w.softmax_scale, out=out,
-                                workspace=ws, stream=stream)
+            gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws,
+                          stream=stream)
             if flush is not None:
                 step_ev[i][1].record(stream)
         ev_end.record(stream)
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+        # ------------------------------------------------ second pass: the split kernel alone
+        # Same K steps with events recorded just before and after the split-KV
+        # kernel of every step (the events break the launch chaining, so this
+        # pass is not the headline).
+        split_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                    for _ in range(args.steps)]
+        for i in range(args.steps):
+            if flush is not None:
+                flush.zero_()
+            gq.gqa_decode_timed(split_ev[i], q, k, v, lens, table, scale=w.softmax_scale, out=out,
+                                workspace=ws, stream=stream)
         torch.cuda.synchronize(dev)
         if dist is not None:
             dist.barrier()

@@ -212,6 +212,9 @@ def _call(q, k_cache, v_cache, seq_lens, block_table, scale, out, out_dtype, wor
     if events is None:
         st = lib.gqa_decode(*args)
     else:
+        for ev in events:  # torch creates the CUDA event on its first record
+            if ev.cuda_event == 0:
+                ev.record(stream)
         st = lib.gqa_decode_timed(*args, ctypes.c_void_p(events[0].cuda_event),
                                   ctypes.c_void_p(events[1].cuda_event))
     if st != 0:

@@ -9,7 +9,10 @@
 // section 2 (Head_i).  Units whose tiles stayed in one CTA were finished by
 // the split kernel; sequences with L_b = 0 get out = 0 here.
 //
-// One CTA per sequence b; partial slots follow schedule.cuh.
+// One CTA per unit.  Each thread owns (head, d) output elements; the partials'
+// log-sum-exps are staged in shared memory kCombineChunk at a time and folded
+// in with a running maximum, so any number of partials works and every
+// partial load of a chunk is independent of the others.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -19,14 +22,31 @@
 
 namespace gqa {
 
-template <int D, bool OUT_BF16>
-__global__ void __launch_bounds__(256) combine_kernel(const KernelArgs a, int grid) {
-    __shared__ int64_t red_total[8], red_before[8];
-    grid_dependency_wait();
-    grid_launch_dependents();
+constexpr int kCombineThreads = 256;
+constexpr int kCombineChunk = 8;  // partials staged per pass
+constexpr int kMaxR = 1024;       // widest group the combine supports (shared memory bound)
 
-    const int b = blockIdx.x;
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ void store_out(void* out, int64_t i, float x) {
+    if constexpr (OUT_BF16)
+        static_cast<__nv_bfloat16*>(out)[i] = __float2bfloat16_rn(x);
+    else
+        static_cast<float*>(out)[i] = x;
+}
+
+template <int D, bool OUT_BF16>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const KernelArgs a, int grid) {
+    extern __shared__ float s_lse[];  // [kCombineChunk][R]
+    __shared__ int64_t red_total[kCombineThreads / 32], red_before[kCombineThreads / 32];
+
+    grid_launch_dependents();
+    const int b = blockIdx.x / a.H_KV;
+    const int kv = blockIdx.x % a.H_KV;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int R = a.R;
+
+    // seq_lens were final before the split kernel read them, so the tile
+    // arithmetic may run while the split grid is still finishing.
     int64_t total = 0, before = 0;
     for (int i = threadIdx.x; i < a.B; i += blockDim.x) {
         const int64_t c = static_cast<int64_t>(a.H_KV) * tiles_of(seq_len_at(a, i));
@@ -41,51 +61,83 @@ __global__ void __launch_bounds__(256) combine_kernel(const KernelArgs a, int gr
     }
     __syncthreads();
     total = before = 0;
-    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) {
+#pragma unroll
+    for (int i = 0; i < kCombineThreads / 32; ++i) {
         total += red_total[i];
         before += red_before[i];
     }
-
     const int n_b = tiles_of(seq_len_at(a, b));
+    const int64_t out_base = (static_cast<int64_t>(b) * a.H_Q + static_cast<int64_t>(kv) * R) * D;
+
     if (n_b == 0) {
-        for (int idx = threadIdx.x; idx < a.H_Q * D; idx += blockDim.x) {
-            const int64_t oi = static_cast<int64_t>(b) * a.H_Q * D + idx;
-            if constexpr (OUT_BF16)
-                static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(0.f);
-            else
-                static_cast<float*>(a.out)[oi] = 0.f;
-        }
+        grid_dependency_wait();  // out may still be in use by the previous call's kernels
+        for (int idx = threadIdx.x; idx < R * D; idx += blockDim.x) store_out<D, OUT_BF16>(a.out, out_base + idx, 0.f);
         return;
     }
     const int g = effective_grid(total, grid);
+    const int64_t s_u = before + static_cast<int64_t>(kv) * n_b;
+    const int64_t ca = owner_of_tile(s_u, total, g);
+    const int64_t cb = owner_of_tile(s_u + n_b - 1, total, g);
+    if (ca == cb) return;  // finished by the split kernel
+    const int n_parts = static_cast<int>(cb - ca + 1);
+    const int64_t slot0 = cta_first_tile(ca, total, g) < s_u ? 2 * ca + 1 : 2 * ca;
+
+    grid_dependency_wait();  // partials of the split grid are complete and visible from here
+
+    constexpr int EPT = 4;  // output elements per thread per pass
     const float NEG_INF = -__int_as_float(0x7f800000);
-    for (int kv = 0; kv < a.H_KV; ++kv) {
-        const int64_t s_u = before + static_cast<int64_t>(kv) * n_b;
-        const int64_t e_u = s_u + n_b;
-        const int64_t ca = owner_of_tile(s_u, total, g);
-        const int64_t cb = owner_of_tile(e_u - 1, total, g);
-        if (ca == cb) continue;  // finished by the split kernel
-        const int n_parts = static_cast<int>(cb - ca + 1);
-        const int64_t slot0 = cta_first_tile(ca, total, g) < s_u ? 2 * ca + 1 : 2 * ca;
-        for (int idx = threadIdx.x; idx < a.R * D; idx += blockDim.x) {
-            const int r = idx / D, d = idx % D;
-            float M = NEG_INF;
-            for (int j = 0; j < n_parts; ++j) {
+    for (int base = 0; base < R * D; base += EPT * kCombineThreads) {
+        float m[EPT], sum[EPT], acc[EPT];
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+            m[e] = NEG_INF;
+            sum[e] = 0.f;
+            acc[e] = 0.f;
+        }
+        for (int j0 = 0; j0 < n_parts; j0 += kCombineChunk) {
+            const int nj = min(kCombineChunk, n_parts - j0);
+            __syncthreads();  // previous chunk's s_lse fully consumed
+            for (int i = threadIdx.x; i < nj * R; i += blockDim.x) {
+                const int jj = i / R, r = i % R;
+                const int j = j0 + jj;
                 const int64_t slot = j == 0 ? slot0 : 2 * (ca + j);
-                M = fmaxf(M, a.ws_lse[slot * a.R + r]);
+                s_lse[jj * R + r] = a.ws_lse[slot * R + r];
             }
-            float wsum = 0.f, acc = 0.f;
-            for (int j = 0; j < n_parts; ++j) {
-                const int64_t slot = j == 0 ? slot0 : 2 * (ca + j);
-                const float e = exp2f(a.ws_lse[slot * a.R + r] - M);
-                wsum += e;
-                acc += e * a.ws_o[(slot * a.R + r) * D + d];
+            __syncthreads();
+#pragma unroll
+            for (int e = 0; e < EPT; ++e) {
+                const int idx = base + e * kCombineThreads + threadIdx.x;
+                if (idx >= R * D) break;
+                const int r = idx / D, d = idx % D;
+                float ov[kCombineChunk];
+#pragma unroll
+                for (int jj = 0; jj < kCombineChunk; ++jj) {
+                    const int j = j0 + jj;
+                    const int64_t slot = j == 0 ? slot0 : 2 * (ca + j);
+                    ov[jj] = jj < nj ? a.ws_o[(slot * R + r) * D + d] : 0.f;
+                }
+                float mx = m[e];
+#pragma unroll
+                for (int jj = 0; jj < kCombineChunk; ++jj)
+                    if (jj < nj) mx = fmaxf(mx, s_lse[jj * R + r]);
+                const float rescale = exp2f(m[e] - mx);  // m = -inf on the first chunk -> 0
+                sum[e] *= rescale;
+                acc[e] *= rescale;
+#pragma unroll
+                for (int jj = 0; jj < kCombineChunk; ++jj) {
+                    if (jj < nj) {
+                        const float wj = exp2f(s_lse[jj * R + r] - mx);
+                        sum[e] += wj;
+                        acc[e] = fmaf(wj, ov[jj], acc[e]);
+                    }
+                }
+                m[e] = mx;
             }
-            const int64_t oi = (static_cast<int64_t>(b) * a.H_Q + kv * a.R + r) * D + d;
-            if constexpr (OUT_BF16)
-                static_cast<__nv_bfloat16*>(a.out)[oi] = __float2bfloat16_rn(acc / wsum);
-            else
-                static_cast<float*>(a.out)[oi] = acc / wsum;
+        }
+#pragma unroll
+        for (int e = 0; e < EPT; ++e) {
+            const int idx = base + e * kCombineThreads + threadIdx.x;
+            if (idx < R * D) store_out<D, OUT_BF16>(a.out, out_base + idx, acc[e] / sum[e]);
         }
     }
 }

@@ -69,6 +69,7 @@ gqa_status validate_params(const gqa_decode_params* p) {
         if (static_cast<int64_t>(p->max_seq_len) > static_cast<int64_t>(p->max_blocks_per_seq) * kTile)
             return GQA_ERR_INVALID;
     }
+    if (p->H_Q / p->H_KV > kMaxR) return GQA_ERR_UNSUPPORTED;
     // 64-bit element offsets are used throughout; keep 32-bit grid / head math safe.
     if (static_cast<int64_t>(p->B) * p->H_Q > (int64_t(1) << 30)) return GQA_ERR_UNSUPPORTED;
     return GQA_OK;
@@ -250,7 +251,9 @@ cudaError_t launch_all(const gqa_decode_params* p, const Buffers& buf, const Ker
                      : launch_split<D, false, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (e != cudaSuccess) return e;
     if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return e;
-    return launch_chained(combine_kernel<D, OUTB>, p->B, 256, 0, stream, args, grid);
+    const size_t smem = sizeof(float) * kCombineChunk * static_cast<size_t>(args.R);
+    return launch_chained(combine_kernel<D, OUTB>, p->B * p->H_KV, kCombineThreads, smem, stream,
+                          args, grid);
 }
 
 gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const void* v,

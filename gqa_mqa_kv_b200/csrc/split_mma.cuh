@@ -248,24 +248,33 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
             if (last_tile && t0 + n0 >= w.L) break;  // no live token in this chunk
             const bool mask = last_tile && (t0 + n0 + 16 > w.L);
 
-            // S = Q K^T for 16 query rows x 16 tokens.
-            float s[2][4];
+            // S = Q K^T for 16 query rows x 16 tokens.  Even and odd k-steps
+            // accumulate separately so four independent mma chains interleave.
+            float s[2][4], s2[2][4];
 #pragma unroll
-            for (int n = 0; n < 2; ++n) s[n][0] = s[n][1] = s[n][2] = s[n][3] = 0.f;
+            for (int n = 0; n < 2; ++n)
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const int p = ks >> 2, c0 = (ks & 3) << 1;
+                for (int i = 0; i < 4; ++i) s[n][i] = s2[n][i] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ks += 2) {
                 const int row = n0 + (lane & 7) + ((lane >> 4) << 3);
-                const int ch = c0 + ((lane >> 3) & 1);
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kb + p * C::PANEL_BYTES + row * 128 + ((ch ^ (lane & 7)) << 4), b0, b1, b2, b3);
-                mma_bf16_16816(s[0], qa[ks], b0, b1);
-                mma_bf16_16816(s[1], qa[ks], b2, b3);
+                uint32_t b[2][4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int p = (ks + h) >> 2, c0 = ((ks + h) & 3) << 1;
+                    const int ch = c0 + ((lane >> 3) & 1);
+                    ldsm_x4(kb + p * C::PANEL_BYTES + row * 128 + ((ch ^ (lane & 7)) << 4), b[h][0], b[h][1],
+                            b[h][2], b[h][3]);
+                }
+                mma_bf16_16816(s[0], qa[ks], b[0][0], b[0][1]);
+                mma_bf16_16816(s[1], qa[ks], b[0][2], b[0][3]);
+                mma_bf16_16816(s2[0], qa[ks + 1], b[1][0], b[1][1]);
+                mma_bf16_16816(s2[1], qa[ks + 1], b[1][2], b[1][3]);
             }
 #pragma unroll
             for (int n = 0; n < 2; ++n)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) s[n][i] *= a.sl2;
+                for (int i = 0; i < 4; ++i) s[n][i] = (s[n][i] + s2[n][i]) * a.sl2;
             uint32_t vmask_a = 0xffffffffu, vmask_b = 0xffffffffu;
             if (mask) {
 #pragma unroll
@@ -318,22 +327,34 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
             split_bf16x2(p[1][0], p[1][1], ph_[2], pl_[2]);
             split_bf16x2(p[1][2], p[1][3], ph_[3], pl_[3]);
 
-            // O += P V  (P as hi + lo bf16 parts).
+            // O += P V  (P as hi + lo bf16 parts).  Two 16-column blocks per
+            // step: the hi products of four accumulators issue before the lo
+            // products that depend on them.
 #pragma unroll
-            for (int j = 0; j < D / 16; ++j) {
-                const int pnl = j >> 2, c0 = (j & 3) << 1;
+            for (int j = 0; j < D / 16; j += 2) {
                 const int row = n0 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                const int ch = c0 + (lane >> 4);
-                uint32_t v0, v1, v2, v3;
-                ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + row * 128 + ((ch ^ (lane & 7)) << 4), v0, v1, v2, v3);
-                v0 &= vmask_a;
-                v1 &= vmask_b;
-                v2 &= vmask_a;
-                v3 &= vmask_b;
-                mma_bf16_16816(o[2 * j], ph_, v0, v1);
-                mma_bf16_16816(o[2 * j], pl_, v0, v1);
-                mma_bf16_16816(o[2 * j + 1], ph_, v2, v3);
-                mma_bf16_16816(o[2 * j + 1], pl_, v2, v3);
+                uint32_t v[2][4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int pnl = (j + h) >> 2, c0 = ((j + h) & 3) << 1;
+                    const int ch = c0 + (lane >> 4);
+                    ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + row * 128 + ((ch ^ (lane & 7)) << 4), v[h][0],
+                                  v[h][1], v[h][2], v[h][3]);
+                    v[h][0] &= vmask_a;
+                    v[h][1] &= vmask_b;
+                    v[h][2] &= vmask_a;
+                    v[h][3] &= vmask_b;
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    mma_bf16_16816(o[2 * (j + h)], ph_, v[h][0], v[h][1]);
+                    mma_bf16_16816(o[2 * (j + h) + 1], ph_, v[h][2], v[h][3]);
+                }
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    mma_bf16_16816(o[2 * (j + h)], pl_, v[h][0], v[h][1]);
+                    mma_bf16_16816(o[2 * (j + h) + 1], pl_, v[h][2], v[h][3]);
+                }
             }
         }
         __syncwarp();
