@@ -22,7 +22,8 @@ import os
 import threading
 
 __all__ = [
-    "GqaError", "Params", "gqa_decode", "gqa_decode_timed", "workspace_bytes", "make_workspace",
+    "GqaError", "Params", "gqa_decode", "gqa_decode_timed", "gqa_decode_static_workspace",
+    "workspace_bytes", "make_workspace",
     "read_status", "kv_cache_bytes", "library", "LIB_PATH", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_BAD_BLOCK", "FLAG_TIMEOUT", "PAGE_SIZE",
 ]
@@ -34,7 +35,7 @@ FLAG_SEQ_LEN_CLAMPED, FLAG_BAD_BLOCK, FLAG_TIMEOUT = 1, 2, 4
 
 EXPORTED = (
     "gqa_decode_workspace_size", "gqa_decode", "gqa_decode_timed", "gqa_read_status",
-    "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version",
+    "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version", "gqa_decode_static_workspace",
 )
 
 
@@ -89,6 +90,9 @@ def library() -> ctypes.CDLL:
             lib.gqa_status_string.restype = ctypes.c_char_p
             lib.gqa_version.argtypes = []
             lib.gqa_version.restype = ctypes.c_int
+            lib.gqa_decode_static_workspace.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_float, vp,
+                                                        vp]
+            lib.gqa_decode_static_workspace.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -244,6 +248,40 @@ def gqa_decode_timed(events, q, k_cache, v_cache, seq_lens, block_table=None, sc
     """gqa_decode with torch.cuda.Event pair ``events`` recorded around the split kernel."""
     return _call(q, k_cache, v_cache, seq_lens, block_table, scale, out, out_dtype, workspace,
                  stream, events, max_seq_len)
+
+
+def gqa_decode_static_workspace(q, k_cache, v_cache, seq_lens, block_table=None, scale=None,
+                                out=None, out_dtype=None, stream=None, max_seq_len=None):
+    """gqa_decode on the library's built-in 8 MiB workspace: this call allocates nothing.
+
+    For callers that cannot call cudaMalloc (a plugin whose host application
+    owns all device memory, a loop that must not take cudaMalloc's implicit
+    device synchronisation).  ``out`` must be given for a call that allocates
+    nothing; without it a fresh output tensor is created here.  Calls whose
+    kernels overlap on the GPU share the one built-in workspace and race; the
+    first call on a device should come before any stream capture.
+    """
+    import torch
+
+    _check_inputs(q, k_cache, v_cache, seq_lens, block_table)
+    params = make_params(q, k_cache, seq_lens, block_table, out_dtype if out is None else out.dtype,
+                         max_seq_len)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or torch.float32, device=q.device)
+    elif out.shape != q.shape or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor shaped like q")
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    bt = ctypes.c_void_p(block_table.data_ptr() if block_table is not None else None)
+    st = library().gqa_decode_static_workspace(
+        ctypes.byref(params), ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k_cache.data_ptr()),
+        ctypes.c_void_p(v_cache.data_ptr()), ctypes.c_void_p(seq_lens.data_ptr()), bt,
+        ctypes.c_float(scale), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise GqaError(st, "gqa_decode_static_workspace")
+    return out
 
 
 def read_status(workspace, stream=None, clear=False) -> int:

@@ -313,6 +313,35 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
     return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
+// ------------------------------------------------------------------ fixed workspace
+//
+// Storage for gqa_decode_static_workspace: a workspace that lives in the
+// library itself, for callers that cannot call cudaMalloc.  Every GPU that
+// loads this library holds these bytes until the process exits.  Host code
+// must never hand this name to a kernel: on the host it is only a stand-in,
+// and the device address comes from cudaGetSymbolAddress below.
+constexpr size_t kStaticWorkspaceBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
+
+// Device address of g_static_workspace on the current device, looked up once
+// per device with that device current; its status word is cleared then.
+gqa_status static_workspace_on_current_device(void** ptr, cudaStream_t stream) {
+    static std::mutex mu;
+    static void* addr[kMaxDevices] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GQA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
+            return GQA_ERR_CUDA;
+        if (cudaMemsetAsync(p, 0, kHeaderBytes, stream) != cudaSuccess) return GQA_ERR_CUDA;
+        addr[dev] = p;
+    }
+    *ptr = addr[dev];
+    return GQA_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -342,6 +371,23 @@ gqa_status gqa_decode_timed(const gqa_decode_params* params, const void* q, cons
                             void* split_end) {
     return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, workspace,
                workspace_bytes, stream, split_begin, split_end);
+}
+
+gqa_status gqa_decode_static_workspace(const gqa_decode_params* params, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* seq_lens, const int32_t* block_table,
+                                       float scale, void* out, void* stream) {
+    gqa_status st = validate_params(params);
+    if (st != GQA_OK) return st;
+    if (params->B == 0) return GQA_OK;
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != GQA_OK) return st;
+    if (workspace_for(params, grid_for(params, dev)) > kStaticWorkspaceBytes) return GQA_ERR_WORKSPACE;
+    void* ws = nullptr;
+    if ((st = static_workspace_on_current_device(&ws, static_cast<cudaStream_t>(stream))) != GQA_OK)
+        return st;
+    return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, ws,
+               kStaticWorkspaceBytes, stream, nullptr, nullptr);
 }
 
 gqa_status gqa_read_status(const void* workspace, void* stream, uint32_t* flags, int clear) {

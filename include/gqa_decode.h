@@ -147,6 +147,36 @@ gqa_status gqa_decode_timed(const gqa_decode_params* params, const void* q, cons
                             void* split_end);
 
 /*
+ * gqa_decode without a caller-supplied workspace, for callers that cannot
+ * call cudaMalloc -- for example a plugin inside a host application that has
+ * already handed all device memory to its own pool, or a latency-critical
+ * loop that must not take cudaMalloc's implicit device-wide synchronisation.
+ * The pages this library follows have no counterpart to this entry point; it
+ * is a deployment convenience.
+ *
+ * The workspace is a fixed 8 MiB array inside the library (GQA_STATIC_WORKSPACE_BYTES),
+ * held on every GPU that loads the library until the process exits.  The
+ * call allocates nothing.  Arguments, layouts and results are those of
+ * gqa_decode; the caller still provides q, the caches, seq_lens,
+ * block_table and out.
+ *
+ *  - Returns GQA_ERR_WORKSPACE, before launching anything, when these
+ *    parameters need more workspace than the array holds (see
+ *    gqa_decode_workspace_size).
+ *  - The first call on each device looks up the array's device address with
+ *    that device current and clears its status word on `stream`; make that
+ *    first call before any stream capture begins.
+ *  - Every call on a device shares the one array, and it keeps the last
+ *    call's contents.  Calls whose kernels overlap on the GPU (different
+ *    streams, or different host threads) race on it: order them.
+ */
+#define GQA_STATIC_WORKSPACE_BYTES (8u << 20)
+gqa_status gqa_decode_static_workspace(const gqa_decode_params* params, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* seq_lens, const int32_t* block_table,
+                                       float scale, void* out, void* stream);
+
+/*
  * Reads the workspace status word (GQA_FLAG_* bits) into *flags after
  * synchronising `stream`; clears it when `clear` is non-zero.
  */
