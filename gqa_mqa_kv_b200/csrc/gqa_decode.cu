@@ -69,7 +69,6 @@ gqa_status validate_params(const gqa_decode_params* p) {
         if (static_cast<int64_t>(p->max_seq_len) > static_cast<int64_t>(p->max_blocks_per_seq) * kTile)
             return GQA_ERR_INVALID;
     }
-    if (p->H_Q / p->H_KV > kMaxR) return GQA_ERR_UNSUPPORTED;
     // 64-bit element offsets are used throughout; keep 32-bit grid / head math safe.
     if (static_cast<int64_t>(p->B) * p->H_Q > (int64_t(1) << 30)) return GQA_ERR_UNSUPPORTED;
     return GQA_OK;
@@ -169,17 +168,17 @@ struct Buffers {
     const void* v;
 };
 
-template <int D, int HG, bool PAGED, bool OUTB>
+template <int D, int NT, int HG, bool PAGED, bool OUTB>
 cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArgs args,
                        const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
-    using C = MmaCfg<D, HG>;
+    using C = MmaCfg<D, NT, HG>;
     const int R = p->H_Q / p->H_KV;
     int stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
     if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     args.n_stages = stages;
-    args.q_rows = R < 16 ? R : 16;
-    args.q_groups = (R + 15) / 16;
+    args.q_rows = R < C::ROWS ? R : C::ROWS;
+    args.q_groups = (R + C::ROWS - 1) / C::ROWS;
 
     CUtensorMap tmQ, tmK, tmV;
     const uint64_t row = static_cast<uint64_t>(D) * 2;
@@ -209,7 +208,7 @@ cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArg
                      encode_bf16(&tmV, buf.v, 4, dims, strides, box4);
     }
     if (!*encode_ok) return cudaErrorInvalidValue;
-    auto kernel = split_mma_kernel<D, HG, PAGED, OUTB>;
+    auto kernel = split_mma_kernel<D, NT, HG, PAGED, OUTB>;
     const int smem = C::smem_bytes(stages);
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
@@ -221,9 +220,10 @@ cudaError_t launch_mma_groups(const gqa_decode_params* p, const Buffers& buf,
                               const KernelArgs& args, const DeviceInfo& dev, int grid,
                               cudaStream_t stream, bool* encode_ok) {
     const int R = p->H_Q / p->H_KV;
-    if (R <= 16) return launch_mma<D, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
-    if (R <= 32) return launch_mma<D, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
-    return launch_mma<D, 4, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (R <= 8) return launch_mma<D, 1, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (R <= 16) return launch_mma<D, 2, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (R <= 32) return launch_mma<D, 4, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    return launch_mma<D, 4, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
 }
 
 template <typename T, int D, bool PAGED, bool OUTB>
@@ -251,9 +251,9 @@ cudaError_t launch_all(const gqa_decode_params* p, const Buffers& buf, const Ker
                      : launch_split<D, false, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (e != cudaSuccess) return e;
     if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return e;
-    const size_t smem = sizeof(float) * kCombineChunk * static_cast<size_t>(args.R);
-    return launch_chained(combine_kernel<D, OUTB>, p->B * p->H_KV, kCombineThreads, smem, stream,
-                          args, grid);
+    const int parts = (args.R * D + kCombineSpan - 1) / kCombineSpan;
+    return launch_chained(combine_kernel<D, OUTB>, p->B * p->H_KV * parts, kCombineThreads, 0,
+                          stream, args, grid);
 }
 
 gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const void* v,

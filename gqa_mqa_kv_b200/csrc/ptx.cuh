@@ -143,6 +143,14 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// Transposes an 8x8 b16 matrix held one fragment per lane (lane i: row i/4,
+// columns 2(i%4), 2(i%4)+1) into the fragment of its transpose.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 hi) {
     return static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
            (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
@@ -157,6 +165,18 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, u
     __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
     hi = pack_bf16x2(h0, h1);
     lo = pack_bf16x2(l0, l1);
+}
+
+// ---------------------------------------------------------------- special functions
+
+// 2^x by the SFU's approximate base-2 exponential (PTX ex2.approx.ftz.f32:
+// a few ulp in the normal range; results below 2^-126 flush to +0, and
+// 2^-inf = +0).  Softmax weights that small are negligible next to the
+// running maximum's weight of 1.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 // ---------------------------------------------------------------- launch chaining

@@ -13,12 +13,14 @@
 //     loads (128-byte swizzle, L2 evict-first for the cache), completing on
 //     mbarriers.  Paged caches only change the tile coordinate: the page id
 //     from the block table replaces (token, sequence).
-//   * NTG x HG consumer warps: head group hg (16 query rows) x token group tg
-//     (64/NTG tokens of each tile).  Per 16-token chunk a warp computes
-//     S = Q K^T with mma.sync m16n8k16 (bf16 in, fp32 out), masks tokens
-//     >= L_b, updates an fp32 online softmax (base-2 exponent, warp shuffles
-//     for the row max), and accumulates O += P V with P split into bf16
-//     hi + lo parts so the weights keep ~16 significant bits.
+//   * NTG x HG consumer warps (four in all): head group hg (ROWS = 8*NT query
+//     heads) x token group tg (64/NTG tokens of each tile).  The contraction is laid out
+//     token-major: per 16-token chunk a warp computes S^T = K Q^T with
+//     mma.sync m16n8k16 (tokens on M, heads on N, so no rows are padding),
+//     masks tokens >= L_b, updates an fp32 online softmax per head (column),
+//     transposes P^T into B fragments with movmatrix, and accumulates
+//     O^T += V^T P^T with P split into bf16 hi + lo parts so the weights keep
+//     ~16 significant bits.
 //   * at a segment end the token groups are merged in shared memory and the
 //     segment writes either the final output or a partial (o / l, m + log2 l).
 //
@@ -31,22 +33,25 @@
 
 namespace gqa {
 
-template <int D, int HG>
+template <int D, int NT, int HG>
 struct MmaCfg {
     static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
-    static_assert(HG == 1 || HG == 2 || HG == 4, "head groups: 1, 2 or 4");
-    static constexpr int NTG = HG >= 4 ? 2 : 4;        // token groups
+    static_assert(NT == 1 || NT == 2 || NT == 4, "8, 16 or 32 query heads per warp");
+    static_assert(HG == 1 || HG == 2, "head groups: 1 or 2");
+    static constexpr int ROWS = 8 * NT;                 // query heads per warp
+    static constexpr bool Q_IN_REGS = NT <= 2;          // else Q fragments are re-read from smem
+    static constexpr int NTG = 4 / HG;                  // token groups
     static constexpr int TPW = kTile / NTG;             // tokens per warp per tile
     static constexpr int NC = NTG * HG;                 // consumer warps
     static constexpr int THREADS = 32 * (NC + 1);
     static constexpr int PANELS = D / 64;               // 128-byte-wide column panels
     static constexpr int PANEL_BYTES = kTile * 128;     // 64 tokens x 64 bf16
     static constexpr int STAGE_BYTES = 2 * PANELS * PANEL_BYTES;
-    static constexpr int QPANEL_BYTES = 16 * 128;       // 16 query rows x 64 bf16
+    static constexpr int QPANEL_BYTES = ROWS * 128;     // ROWS query rows x 64 bf16
     static constexpr int QSLOT_BYTES = HG * PANELS * QPANEL_BYTES;
     static constexpr int OROW = D + 4;                  // padded merge row (floats)
-    static constexpr int MERGE_O_FLOATS = (NTG - 1) * HG * 16 * OROW;
-    static constexpr int MERGE_ML_FLOATS = (NTG - 1) * HG * 16 * 2;
+    static constexpr int MERGE_O_FLOATS = (NTG - 1) * HG * ROWS * OROW;
+    static constexpr int MERGE_ML_FLOATS = (NTG - 1) * HG * ROWS * 2;
     static constexpr int MAX_STAGES = 8;
     static constexpr int CTRL_BYTES = 256;
     static constexpr int FIXED_BYTES =
@@ -55,8 +60,8 @@ struct MmaCfg {
 };
 
 struct __align__(16) MmaControl {
-    uint64_t full[MmaCfg<128, 1>::MAX_STAGES];
-    uint64_t empty[MmaCfg<128, 1>::MAX_STAGES];
+    uint64_t full[MmaCfg<128, 1, 1>::MAX_STAGES];
+    uint64_t empty[MmaCfg<128, 1, 1>::MAX_STAGES];
     uint64_t qfull[2];
     uint64_t qempty[2];
     uint64_t merge_full;
@@ -64,13 +69,14 @@ struct __align__(16) MmaControl {
     Plan plan;
     int abort;
 };
-static_assert(sizeof(MmaControl) <= MmaCfg<128, 1>::CTRL_BYTES, "control block overflows its slot");
+static_assert(sizeof(MmaControl) <= MmaCfg<128, 1, 1>::CTRL_BYTES, "control block overflows its slot");
 
-template <int D, int HG, bool PAGED, bool OUT_BF16>
-__global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
+template <int D, int NT, int HG, bool PAGED, bool OUT_BF16>
+__global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     split_mma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const KernelArgs a) {
-    using C = MmaCfg<D, HG>;
+    using C = MmaCfg<D, NT, HG>;
+    constexpr int KS = D / 16;  // k-steps over the head dimension; also 16-row blocks of d
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
@@ -86,6 +92,11 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
+    if (warp == C::NC && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_addr(&ctrl->full[s]), 1);
@@ -99,7 +110,7 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
         mbar_init(smem_addr(&ctrl->merge_free), HG);
         ctrl->abort = 0;
     }
-    // Query rows a TMA box does not cover (R < 16) must read as zeros.
+    // Query rows a TMA box does not cover (R < ROWS) must read as zeros.
     for (int i = threadIdx.x; i < 2 * C::QSLOT_BYTES / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(base_ptr + NS * C::STAGE_BYTES)[i] = make_uint4(0, 0, 0, 0);
 
@@ -117,11 +128,6 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
 
     if (warp == C::NC) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            prefetch_tensormap(&tmQ);
-            prefetch_tensormap(&tmK);
-            prefetch_tensormap(&tmV);
-        }
         const uint64_t pol_kv = policy_evict_first();
         const uint64_t pol_q = policy_evict_last();
         const uint32_t q_bytes = static_cast<uint32_t>(a.q_groups * C::PANELS * a.q_rows * 128);
@@ -140,7 +146,7 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
                     for (int g = 0; g < a.q_groups; ++g)
                         for (int p = 0; p < C::PANELS; ++p)
                             tma_load_3d(qring + qs * C::QSLOT_BYTES + (g * C::PANELS + p) * C::QPANEL_BYTES,
-                                        &tmQ, bar, 64 * p, w.kv * a.R + 16 * g, w.b, pol_q);
+                                        &tmQ, bar, 64 * p, w.kv * a.R + C::ROWS * g, w.b, pol_q);
                 }
                 ++q_issued;
                 if (++qs == 2) { qs = 0; qph ^= 1u; }
@@ -193,6 +199,9 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
     }
 
     // ---------------------------------------------------------------- consumers
+    // Fragment ownership (g = lane / 4, t = lane % 4):
+    //   S^T, P:  token n0 + g (+8)      x head 8 nt + 2t (+1)
+    //   O^T:     d 16 mm + g (+8)       x head 8 nt + 2t (+1)
     const int hg = warp / C::NTG;
     const int tg = warp % C::NTG;
     const int g = lane >> 2;
@@ -203,9 +212,10 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
     uint32_t ph = 0, qph = 0, mfull_ph = 0, mfree_ph = 0;
     bool first_seg = true;
     int seg_start_tile = 0;
-    uint32_t qa[D / 16][4];
-    float o[D / 8][4];
-    float m0 = NEG_INF, m1 = NEG_INF, l0 = 0.f, l1 = 0.f;
+    uint32_t qb[C::Q_IN_REGS ? KS : 1][NT][2];  // B fragments of Q^T (k-step, 8-head tile)
+    int seg_q = 0;                                  // Q-ring slot of the current segment
+    float o[KS][NT][4];      // O^T accumulators, per 16-row block of d and 8-head tile
+    float m[NT][2], l[NT][2];
 
     auto fail = [&]() {
         *abort_flag = 1;
@@ -219,22 +229,43 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
         if (seg_first) {
             seg_start_tile = w.tile;
             if (!mbar_wait_warp(smem_addr(&ctrl->qfull[qs]), qph, abort_flag)) { fail(); break; }
+            seg_q = qs;
             const uint32_t qbase = qring + qs * C::QSLOT_BYTES + hg * C::PANELS * C::QPANEL_BYTES;
+            if constexpr (!C::Q_IN_REGS) {
+                // read per chunk from the ring slot; released at the segment end
+            } else if constexpr (NT == 2) {
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ++ks) {
-                const int p = ks >> 2, c0 = (ks & 3) << 1;
-                const int row = (lane & 7) + (((lane >> 3) & 1) << 3);
-                const int ch = c0 + (lane >> 4);
-                ldsm_x4(qbase + p * C::QPANEL_BYTES + row * 128 + ((ch ^ (row & 7)) << 4), qa[ks][0],
-                        qa[ks][1], qa[ks][2], qa[ks][3]);
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int p = ks >> 2, c0 = (ks & 3) << 1;
+                    const int row = (lane & 7) + ((lane >> 4) << 3);
+                    const int ch = c0 + ((lane >> 3) & 1);
+                    ldsm_x4(qbase + p * C::QPANEL_BYTES + row * 128 + ((ch ^ (row & 7)) << 4), qb[ks][0][0],
+                            qb[ks][0][1], qb[ks][1][0], qb[ks][1][1]);
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < KS; ks += 2) {
+                    const int kk = ks + (lane >> 4);
+                    const int p = kk >> 2, ch = ((kk & 3) << 1) + ((lane >> 3) & 1);
+                    const int row = lane & 7;
+                    ldsm_x4(qbase + p * C::QPANEL_BYTES + row * 128 + ((ch ^ row) << 4), qb[ks][0][0],
+                            qb[ks][0][1], qb[ks + 1][0][0], qb[ks + 1][0][1]);
+                }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[qs]));
+            if constexpr (C::Q_IN_REGS) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[qs]));
+            }
             if (++qs == 2) { qs = 0; qph ^= 1u; }
-            m0 = m1 = NEG_INF;
-            l0 = l1 = 0.f;
 #pragma unroll
-            for (int n = 0; n < D / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+            for (int nt = 0; nt < NT; ++nt) {
+                m[nt][0] = m[nt][1] = NEG_INF;
+                l[nt][0] = l[nt][1] = 0.f;
+            }
+#pragma unroll
+            for (int mm = 0; mm < KS; ++mm)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) o[mm][nt][0] = o[mm][nt][1] = o[mm][nt][2] = o[mm][nt][3] = 0.f;
         }
 
         if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { fail(); break; }
@@ -248,113 +279,142 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
             if (last_tile && t0 + n0 >= w.L) break;  // no live token in this chunk
             const bool mask = last_tile && (t0 + n0 + 16 > w.L);
 
-            // S = Q K^T for 16 query rows x 16 tokens.  Even and odd k-steps
-            // accumulate separately so four independent mma chains interleave.
-            float s[2][4], s2[2][4];
+            // S^T = K Q^T: 16 tokens x ROWS heads.  k-steps rotate over NSET
+            // accumulator sets so independent mma chains interleave.
+            constexpr int NSET = NT == 1 ? 4 : (NT == 2 ? 2 : 1);
+            float sa[NSET][NT][4];
 #pragma unroll
-            for (int n = 0; n < 2; ++n)
+            for (int q = 0; q < NSET; ++q)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) s[n][i] = s2[n][i] = 0.f;
+                for (int nt = 0; nt < NT; ++nt) sa[q][nt][0] = sa[q][nt][1] = sa[q][nt][2] = sa[q][nt][3] = 0.f;
+            const int krow = n0 + (lane & 7) + (((lane >> 3) & 1) << 3);
 #pragma unroll
-            for (int ks = 0; ks < D / 16; ks += 2) {
-                const int row = n0 + (lane & 7) + ((lane >> 4) << 3);
-                uint32_t b[2][4];
+            for (int ks = 0; ks < KS; ks += 2) {
+                uint32_t ka[2][4];
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int p = (ks + h) >> 2, c0 = ((ks + h) & 3) << 1;
-                    const int ch = c0 + ((lane >> 3) & 1);
-                    ldsm_x4(kb + p * C::PANEL_BYTES + row * 128 + ((ch ^ (lane & 7)) << 4), b[h][0], b[h][1],
-                            b[h][2], b[h][3]);
+                    const int p = (ks + h) >> 2, ch = (((ks + h) & 3) << 1) + (lane >> 4);
+                    ldsm_x4(kb + p * C::PANEL_BYTES + krow * 128 + ((ch ^ (lane & 7)) << 4), ka[h][0], ka[h][1],
+                            ka[h][2], ka[h][3]);
                 }
-                mma_bf16_16816(s[0], qa[ks], b[0][0], b[0][1]);
-                mma_bf16_16816(s[1], qa[ks], b[0][2], b[0][3]);
-                mma_bf16_16816(s2[0], qa[ks + 1], b[1][0], b[1][1]);
-                mma_bf16_16816(s2[1], qa[ks + 1], b[1][2], b[1][3]);
+                if constexpr (C::Q_IN_REGS) {
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_bf16_16816(sa[(ks + h) % NSET][nt], ka[h], qb[ks + h][nt][0], qb[ks + h][nt][1]);
+                } else {
+                    const uint32_t qbase = qring + seg_q * C::QSLOT_BYTES + hg * C::PANELS * C::QPANEL_BYTES;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const int kk = ks + h;
+                        const int p = kk >> 2, ch = ((kk & 3) << 1) + ((lane >> 3) & 1);
+                        uint32_t qf[NT][2];
+#pragma unroll
+                        for (int np = 0; np < NT / 2; ++np) {
+                            const int row = 16 * np + (lane & 7) + ((lane >> 4) << 3);
+                            ldsm_x4(qbase + p * C::QPANEL_BYTES + row * 128 + ((ch ^ (row & 7)) << 4),
+                                    qf[2 * np][0], qf[2 * np][1], qf[2 * np + 1][0], qf[2 * np + 1][1]);
+                        }
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt)
+                            mma_bf16_16816(sa[kk % NSET][nt], ka[h], qf[nt][0], qf[nt][1]);
+                    }
+                }
             }
+            float s[NT][4];
 #pragma unroll
-            for (int n = 0; n < 2; ++n)
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int i = 0; i < 4; ++i) s[n][i] = (s[n][i] + s2[n][i]) * a.sl2;
+                for (int i = 0; i < 4; ++i) {
+                    float x = sa[0][nt][i];
+#pragma unroll
+                    for (int q = 1; q < NSET; ++q) x += sa[q][nt][i];
+                    s[nt][i] = x * a.sl2;
+                }
             uint32_t vmask_a = 0xffffffffu, vmask_b = 0xffffffffu;
             if (mask) {
+                const bool live0 = t0 + n0 + g < w.L, live1 = t0 + n0 + g + 8 < w.L;
 #pragma unroll
-                for (int n = 0; n < 2; ++n)
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const int tok = t0 + n0 + 8 * n + 2 * t + (i & 1);
-                        if (tok >= w.L) s[n][i] = NEG_INF;
-                    }
+                for (int nt = 0; nt < NT; ++nt) {
+                    if (!live0) s[nt][0] = s[nt][1] = NEG_INF;
+                    if (!live1) s[nt][2] = s[nt][3] = NEG_INF;
+                }
                 const int ta = t0 + n0 + 2 * t;
                 vmask_a = (ta < w.L ? 0x0000ffffu : 0u) | (ta + 1 < w.L ? 0xffff0000u : 0u);
                 vmask_b = (ta + 8 < w.L ? 0x0000ffffu : 0u) | (ta + 9 < w.L ? 0xffff0000u : 0u);
             }
 
-            // Online softmax (rows g and g + 8 of the head group).
-            float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-            float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-            mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-            mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-            const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-            const float ref0 = mn0 == NEG_INF ? 0.f : mn0;
-            const float ref1 = mn1 == NEG_INF ? 0.f : mn1;
-            const float al0 = exp2f(m0 - ref0), al1 = exp2f(m1 - ref1);
-            m0 = mn0;
-            m1 = mn1;
-            float p[2][4];
+            // Online softmax per head column: reduce over the 8 lanes that share t.
+            float p[NT][4], alpha[NT][2];
+            bool rescale = false;
 #pragma unroll
-            for (int n = 0; n < 2; ++n) {
-                p[n][0] = exp2f(s[n][0] - ref0);
-                p[n][1] = exp2f(s[n][1] - ref0);
-                p[n][2] = exp2f(s[n][2] - ref1);
-                p[n][3] = exp2f(s[n][3] - ref1);
-            }
-            l0 = l0 * al0 + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-            l1 = l1 * al1 + (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
-            if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+            for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    o[n][0] *= al0;
-                    o[n][1] *= al0;
-                    o[n][2] *= al1;
-                    o[n][3] *= al1;
+                for (int j = 0; j < 2; ++j) {
+                    float mx = fmaxf(s[nt][j], s[nt][j + 2]);
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+                    const float mn = fmaxf(m[nt][j], mx);
+                    const float ref = mn == NEG_INF ? 0.f : mn;
+                    alpha[nt][j] = fast_exp2(m[nt][j] - ref);
+                    m[nt][j] = mn;
+                    p[nt][j] = fast_exp2(s[nt][j] - ref);
+                    p[nt][j + 2] = fast_exp2(s[nt][j + 2] - ref);
+                    l[nt][j] = l[nt][j] * alpha[nt][j] + (p[nt][j] + p[nt][j + 2]);
+                    rescale |= alpha[nt][j] != 1.f;
                 }
+            if (__any_sync(0xffffffffu, rescale)) {
+#pragma unroll
+                for (int mm = 0; mm < KS; ++mm)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        o[mm][nt][0] *= alpha[nt][0];
+                        o[mm][nt][1] *= alpha[nt][1];
+                        o[mm][nt][2] *= alpha[nt][0];
+                        o[mm][nt][3] *= alpha[nt][1];
+                    }
             }
-            uint32_t ph_[4], pl_[4];
-            split_bf16x2(p[0][0], p[0][1], ph_[0], pl_[0]);
-            split_bf16x2(p[0][2], p[0][3], ph_[1], pl_[1]);
-            split_bf16x2(p[1][0], p[1][1], ph_[2], pl_[2]);
-            split_bf16x2(p[1][2], p[1][3], ph_[3], pl_[3]);
+            // P^T as B fragments (tokens x heads), hi and lo bf16 parts.
+            uint32_t pbh[NT][2], pbl[NT][2];
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+                uint32_t h0, l0, h1, l1;
+                split_bf16x2(p[nt][0], p[nt][1], h0, l0);  // token g:     heads 2t, 2t+1
+                split_bf16x2(p[nt][2], p[nt][3], h1, l1);  // token g + 8: heads 2t, 2t+1
+                pbh[nt][0] = movmatrix_trans(h0);
+                pbh[nt][1] = movmatrix_trans(h1);
+                pbl[nt][0] = movmatrix_trans(l0);
+                pbl[nt][1] = movmatrix_trans(l1);
+            }
 
-            // O += P V  (P as hi + lo bf16 parts).  Two 16-column blocks per
-            // step: the hi products of four accumulators issue before the lo
-            // products that depend on them.
+            // O^T += V^T P^T.  Hi products of a group of accumulators issue
+            // before the lo products that depend on them.
+            constexpr int MG = 4 / NT;  // 16-row blocks of d per group
+            const int vrow = n0 + (lane & 7) + ((lane >> 4) << 3);
 #pragma unroll
-            for (int j = 0; j < D / 16; j += 2) {
-                const int row = n0 + (lane & 7) + (((lane >> 3) & 1) << 3);
-                uint32_t v[2][4];
+            for (int m0 = 0; m0 < KS; m0 += MG) {
+                uint32_t va[MG][4];
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int pnl = (j + h) >> 2, c0 = ((j + h) & 3) << 1;
-                    const int ch = c0 + (lane >> 4);
-                    ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + row * 128 + ((ch ^ (lane & 7)) << 4), v[h][0],
-                                  v[h][1], v[h][2], v[h][3]);
-                    v[h][0] &= vmask_a;
-                    v[h][1] &= vmask_b;
-                    v[h][2] &= vmask_a;
-                    v[h][3] &= vmask_b;
+                for (int h = 0; h < MG; ++h) {
+                    const int mm = m0 + h;
+                    const int pnl = mm >> 2, ch = ((mm & 3) << 1) + ((lane >> 3) & 1);
+                    ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + vrow * 128 + ((ch ^ (lane & 7)) << 4), va[h][0],
+                                  va[h][1], va[h][2], va[h][3]);
+                    va[h][0] &= vmask_a;
+                    va[h][1] &= vmask_a;
+                    va[h][2] &= vmask_b;
+                    va[h][3] &= vmask_b;
                 }
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    mma_bf16_16816(o[2 * (j + h)], ph_, v[h][0], v[h][1]);
-                    mma_bf16_16816(o[2 * (j + h) + 1], ph_, v[h][2], v[h][3]);
-                }
+                for (int h = 0; h < MG; ++h)
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    mma_bf16_16816(o[2 * (j + h)], pl_, v[h][0], v[h][1]);
-                    mma_bf16_16816(o[2 * (j + h) + 1], pl_, v[h][2], v[h][3]);
-                }
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[m0 + h][nt], va[h], pbh[nt][0], pbh[nt][1]);
+#pragma unroll
+                for (int h = 0; h < MG; ++h)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[m0 + h][nt], va[h], pbl[nt][0], pbl[nt][1]);
             }
         }
         __syncwarp();
@@ -363,108 +423,111 @@ __global__ void __launch_bounds__(MmaCfg<D, HG>::THREADS, 1)
 
         if (seg_last) {
             // ---------------------------------------------------- segment end
-            l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-            l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-            l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+            if constexpr (!C::Q_IN_REGS) {
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[seg_q]));
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    l[nt][j] += __shfl_xor_sync(0xffffffffu, l[nt][j], 4);
+                    l[nt][j] += __shfl_xor_sync(0xffffffffu, l[nt][j], 8);
+                    l[nt][j] += __shfl_xor_sync(0xffffffffu, l[nt][j], 16);
+                }
             const bool whole = (seg_start_tile == 0) && last_tile;
             if (tg > 0) {
                 if (!mbar_wait_warp(smem_addr(&ctrl->merge_free), mfree_ph ^ 1u, abort_flag)) { fail(); break; }
                 mfree_ph ^= 1u;
-                float* mo = merge_o + ((tg - 1) * HG + hg) * 16 * C::OROW;
-                float* ml = merge_ml + ((tg - 1) * HG + hg) * 32;
-                if (t == 0) {
-                    ml[g * 2] = m0;
-                    ml[g * 2 + 1] = l0;
-                    ml[(g + 8) * 2] = m1;
-                    ml[(g + 8) * 2 + 1] = l1;
+                float* mo = merge_o + ((tg - 1) * HG + hg) * C::ROWS * C::OROW;
+                float* ml = merge_ml + ((tg - 1) * HG + hg) * C::ROWS * 2;
+                if (g == 0) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) {
+                            ml[(8 * nt + 2 * t + j) * 2] = m[nt][j];
+                            ml[(8 * nt + 2 * t + j) * 2 + 1] = l[nt][j];
+                        }
                 }
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    *reinterpret_cast<float2*>(&mo[g * C::OROW + 8 * n + 2 * t]) = make_float2(o[n][0], o[n][1]);
-                    *reinterpret_cast<float2*>(&mo[(g + 8) * C::OROW + 8 * n + 2 * t]) = make_float2(o[n][2], o[n][3]);
-                }
+                for (int mm = 0; mm < KS; ++mm)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            mo[(8 * nt + 2 * t + (e & 1)) * C::OROW + 16 * mm + g + 8 * (e >> 1)] = o[mm][nt][e];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->merge_full));
             } else {
                 if (!mbar_wait_warp(smem_addr(&ctrl->merge_full), mfull_ph, abort_flag)) { fail(); break; }
                 mfull_ph ^= 1u;
-                float M0 = m0, M1 = m1;
+                float M[NT][2], Lsum[NT][2];
 #pragma unroll
-                for (int k = 1; k < C::NTG; ++k) {
-                    const float* ml = merge_ml + ((k - 1) * HG + hg) * 32;
-                    M0 = fmaxf(M0, ml[g * 2]);
-                    M1 = fmaxf(M1, ml[(g + 8) * 2]);
-                }
-                const float R0 = M0 == NEG_INF ? 0.f : M0;
-                const float R1 = M1 == NEG_INF ? 0.f : M1;
-                const float f0 = exp2f(m0 - R0), f1 = exp2f(m1 - R1);
-                float L0 = l0 * f0, L1 = l1 * f1;
+                for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                for (int n = 0; n < D / 8; ++n) {
-                    o[n][0] *= f0;
-                    o[n][1] *= f0;
-                    o[n][2] *= f1;
-                    o[n][3] *= f1;
-                }
+                    for (int j = 0; j < 2; ++j) {
+                        const int hl = 8 * nt + 2 * t + j;
+                        float mx = m[nt][j];
 #pragma unroll
-                for (int k = 1; k < C::NTG; ++k) {
-                    const float* ml = merge_ml + ((k - 1) * HG + hg) * 32;
-                    const float* mo = merge_o + ((k - 1) * HG + hg) * 16 * C::OROW;
-                    const float e0 = exp2f(ml[g * 2] - R0), e1 = exp2f(ml[(g + 8) * 2] - R1);
-                    L0 += ml[g * 2 + 1] * e0;
-                    L1 += ml[(g + 8) * 2 + 1] * e1;
+                        for (int k = 1; k < C::NTG; ++k)
+                            mx = fmaxf(mx, merge_ml[(((k - 1) * HG + hg) * C::ROWS + hl) * 2]);
+                        M[nt][j] = mx;
+                        const float ref = mx == NEG_INF ? 0.f : mx;
+                        const float f = fast_exp2(m[nt][j] - ref);
+                        float L = l[nt][j] * f;
 #pragma unroll
-                    for (int n = 0; n < D / 8; ++n) {
-                        const float2 x = *reinterpret_cast<const float2*>(&mo[g * C::OROW + 8 * n + 2 * t]);
-                        const float2 y = *reinterpret_cast<const float2*>(&mo[(g + 8) * C::OROW + 8 * n + 2 * t]);
-                        o[n][0] += x.x * e0;
-                        o[n][1] += x.y * e0;
-                        o[n][2] += y.x * e1;
-                        o[n][3] += y.y * e1;
+                        for (int mm = 0; mm < KS; ++mm) {
+                            o[mm][nt][j] *= f;
+                            o[mm][nt][j + 2] *= f;
+                        }
+#pragma unroll
+                        for (int k = 1; k < C::NTG; ++k) {
+                            const float* ml = merge_ml + (((k - 1) * HG + hg) * C::ROWS + hl) * 2;
+                            const float* mo = merge_o + (((k - 1) * HG + hg) * C::ROWS + hl) * C::OROW;
+                            const float e = fast_exp2(ml[0] - ref);
+                            L += ml[1] * e;
+#pragma unroll
+                            for (int mm = 0; mm < KS; ++mm) {
+                                o[mm][nt][j] += mo[16 * mm + g] * e;
+                                o[mm][nt][j + 2] += mo[16 * mm + g + 8] * e;
+                            }
+                        }
+                        Lsum[nt][j] = L;
                     }
-                }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->merge_free));
-                const float inv0 = 1.f / L0, inv1 = 1.f / L1;
-                const int r0 = hg * 16 + g, r1 = r0 + 8;
-                if (whole) {
-                    const int64_t row0 = static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + r0;
-                    const int64_t row1 = row0 + 8;
+                const int64_t slot = first_seg ? 2 * static_cast<int64_t>(blockIdx.x) : 2 * static_cast<int64_t>(blockIdx.x) + 1;
 #pragma unroll
-                    for (int n = 0; n < D / 8; ++n) {
-                        const int d = 8 * n + 2 * t;
-                        if constexpr (OUT_BF16) {
-                            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(a.out);
-                            if (r0 < a.R)
-                                *reinterpret_cast<__nv_bfloat162*>(out + row0 * D + d) =
-                                    __floats2bfloat162_rn(o[n][0] * inv0, o[n][1] * inv0);
-                            if (r1 < a.R)
-                                *reinterpret_cast<__nv_bfloat162*>(out + row1 * D + d) =
-                                    __floats2bfloat162_rn(o[n][2] * inv1, o[n][3] * inv1);
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int r = hg * C::ROWS + 8 * nt + 2 * t + j;
+                        if (r >= a.R) continue;
+                        const float inv = 1.f / Lsum[nt][j];
+                        if (whole) {
+                            const int64_t row = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + r) * D;
+#pragma unroll
+                            for (int mm = 0; mm < KS; ++mm)
+#pragma unroll
+                                for (int hh = 0; hh < 2; ++hh) {
+                                    const float x = o[mm][nt][j + 2 * hh] * inv;
+                                    const int64_t i = row + 16 * mm + g + 8 * hh;
+                                    if constexpr (OUT_BF16)
+                                        static_cast<__nv_bfloat16*>(a.out)[i] = __float2bfloat16_rn(x);
+                                    else
+                                        static_cast<float*>(a.out)[i] = x;
+                                }
                         } else {
-                            float* out = static_cast<float*>(a.out);
-                            if (r0 < a.R)
-                                *reinterpret_cast<float2*>(out + row0 * D + d) = make_float2(o[n][0] * inv0, o[n][1] * inv0);
-                            if (r1 < a.R)
-                                *reinterpret_cast<float2*>(out + row1 * D + d) = make_float2(o[n][2] * inv1, o[n][3] * inv1);
+                            float* dst = a.ws_o + (slot * a.R + r) * D;
+#pragma unroll
+                            for (int mm = 0; mm < KS; ++mm) {
+                                dst[16 * mm + g] = o[mm][nt][j] * inv;
+                                dst[16 * mm + g + 8] = o[mm][nt][j + 2] * inv;
+                            }
+                            if (g == 0) a.ws_lse[slot * a.R + r] = M[nt][j] + log2f(Lsum[nt][j]);
                         }
                     }
-                } else {
-                    const int64_t slot = first_seg ? 2 * static_cast<int64_t>(blockIdx.x) : 2 * static_cast<int64_t>(blockIdx.x) + 1;
-#pragma unroll
-                    for (int n = 0; n < D / 8; ++n) {
-                        const int d = 8 * n + 2 * t;
-                        if (r0 < a.R)
-                            *reinterpret_cast<float2*>(a.ws_o + (slot * a.R + r0) * D + d) = make_float2(o[n][0] * inv0, o[n][1] * inv0);
-                        if (r1 < a.R)
-                            *reinterpret_cast<float2*>(a.ws_o + (slot * a.R + r1) * D + d) = make_float2(o[n][2] * inv1, o[n][3] * inv1);
-                    }
-                    if (t == 0) {
-                        if (r0 < a.R) a.ws_lse[slot * a.R + r0] = M0 + log2f(L0);
-                        if (r1 < a.R) a.ws_lse[slot * a.R + r1] = M1 + log2f(L1);
-                    }
-                }
             }
             first_seg = false;
         }

@@ -98,8 +98,8 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
                     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
                     s *= a.sl2;
                     const float mn = fmaxf(m[j], s);
-                    const float al = exp2f(m[j] - mn);
-                    const float p = exp2f(s - mn);
+                    const float al = fast_exp2(m[j] - mn);
+                    const float p = fast_exp2(s - mn);
                     l[j] = l[j] * al + p;
 #pragma unroll
                     for (int i = 0; i < DPL; ++i) o[j][i] = fmaf(p, vr[i], o[j][i] * al);
@@ -125,7 +125,7 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
                 float L = 0.f, O = 0.f;
 #pragma unroll
                 for (int ww = 0; ww < kSimtWarps; ++ww) {
-                    const float e = exp2f(sm_m[ww][j] - ref);
+                    const float e = fast_exp2(sm_m[ww][j] - ref);
                     L += sm_l[ww][j] * e;
                     O += sm_o[ww][j][d] * e;
                 }
