@@ -1,0 +1,38 @@
+"""Host-side partitioning of one decode step across ranks.
+
+Two ways to split the step, neither of which needs an exchange on the data
+path:
+
+* batch sharding: each rank owns a contiguous block of sequences;
+* tensor-parallel head sharding ("Grouped-Query Attention (GQA) and
+  Multi-Query Attention (MQA): Mathematical Foundations, ...", section 4,
+  "Tensor Parallelism (TP) Head Partitioning"): rank j of N holds KV heads
+  [j H_KV/N, (j+1) H_KV/N) and the query heads that read them,
+  [j H_Q/N, (j+1) H_Q/N); this requires H_KV mod N = 0.  Because the group map
+  is contiguous, every query head of a rank's slice reads a KV head of the
+  same slice, so each rank runs an ordinary GQA decode on its slice.
+"""
+
+from __future__ import annotations
+
+
+def batch_shard(B: int, world: int, rank: int) -> slice:
+    """Contiguous block of sequences for `rank` (sizes differ by at most one)."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError("bad world/rank")
+    lo = rank * B // world
+    hi = (rank + 1) * B // world
+    return slice(lo, hi)
+
+
+def tp_head_shard(H_Q: int, H_KV: int, world: int, rank: int) -> tuple[slice, slice]:
+    """(query-head slice, KV-head slice) of `rank` under tensor parallelism."""
+    if world <= 0 or not 0 <= rank < world:
+        raise ValueError("bad world/rank")
+    if H_Q % H_KV != 0:
+        raise ValueError("H_Q must be a multiple of H_KV")
+    if H_KV % world != 0:
+        raise ValueError("tensor parallelism without duplication needs H_KV % world == 0")
+    kv_per = H_KV // world
+    q_per = H_Q // world
+    return slice(rank * q_per, (rank + 1) * q_per), slice(rank * kv_per, (rank + 1) * kv_per)

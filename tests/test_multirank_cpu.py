@@ -1,0 +1,145 @@
+"""Multi-rank host logic on CPU with world_size 2 gloo process groups.
+
+Covers the benchmark's distributed plumbing (rank environment, max-over-ranks
+timing, rank-0-only reference arm) and the partitioning helpers: batch shards
+and tensor-parallel head shards, each checked by running the fp64 oracle on
+every rank's shard and comparing the gathered result with the unsharded one.
+"""
+
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, fn_name, out_q):
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    try:
+        import bench  # noqa: F401  (imports must work on a CPU-only host)
+
+        g = globals()[fn_name]
+        res = g(rank, world)
+        out_q.put((rank, "ok", res))
+    except Exception as e:  # report to the parent instead of hanging it
+        out_q.put((rank, "error", repr(e)))
+    finally:
+        if dist.is_initialized():
+            dist.destroy_process_group()
+
+
+def run_ranks(fn_name, world=2):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = free_port()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, fn_name, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = {}
+    for _ in range(world):
+        rank, status, res = q.get(timeout=180)
+        assert status == "ok", res
+        results[rank] = res
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return results
+
+
+def rank_timing(rank, world):
+    import bench
+
+    w, r, local = bench.dist_env()
+    assert (w, r, local) == (world, rank, rank)
+    d = bench.init_dist(w, "gloo")
+    t = bench.max_over_ranks(1.5 + rank, d, torch.device("cpu"))
+    d.barrier()
+    return t
+
+
+def rank_batch_shards(rank, world):
+    import oracle
+    from gqa_mqa_kv_b200.sharding import batch_shard
+    from gqa_mqa_kv_b200.workloads import WORKLOADS, make_inputs
+    import dataclasses
+
+    dist.init_process_group("gloo")
+    w = dataclasses.replace(WORKLOADS["llama2_70b_ragged"], B=5, seq_len=300)
+    inp = make_inputs(w)
+    sl = batch_shard(w.B, world, rank)
+    mine = oracle.gqa_decode(inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["seq_lens"][sl], w.softmax_scale)
+    parts = [None] * world
+    dist.all_gather_object(parts, (sl.start, mine))
+    full = oracle.gqa_decode(inp["q"], inp["k"], inp["v"], inp["seq_lens"], w.softmax_scale)
+    import numpy as np
+
+    got = np.concatenate([p[1] for p in sorted(parts, key=lambda x: x[0])])
+    return bool(np.array_equal(got, full))
+
+
+def rank_tp_shards(rank, world):
+    import numpy as np
+
+    import oracle
+    from gqa_mqa_kv_b200.sharding import tp_head_shard
+    from gqa_mqa_kv_b200.workloads import WORKLOADS, make_inputs
+    import dataclasses
+
+    dist.init_process_group("gloo")
+    w = dataclasses.replace(WORKLOADS["llama2_70b_ragged"], B=3, seq_len=200)
+    inp = make_inputs(w)
+    qs, ks = tp_head_shard(w.H_Q, w.H_KV, world, rank)
+    mine = oracle.gqa_decode(inp["q"][:, qs].contiguous(), inp["k"][:, :, ks].contiguous(),
+                             inp["v"][:, :, ks].contiguous(), inp["seq_lens"], w.softmax_scale)
+    parts = [None] * world
+    dist.all_gather_object(parts, (qs.start, mine))
+    got = np.concatenate([p[1] for p in sorted(parts, key=lambda x: x[0])], axis=1)
+    full = oracle.gqa_decode(inp["q"], inp["k"], inp["v"], inp["seq_lens"], w.softmax_scale)
+    return bool(np.array_equal(got, full))
+
+
+def rank_reference_arm(rank, world):
+    import bench
+
+    if rank != 0:
+        return bench.run_reference(bench.parse_args(["--impl", "reference", "--gpus", str(world)]))
+    return 0  # rank 0 would run the oracle; only the non-zero ranks' early exit is checked here
+
+
+def test_max_over_ranks_with_gloo():
+    res = run_ranks("rank_timing")
+    assert res == {0: 2.5, 1: 2.5}
+
+
+def test_batch_shards_reassemble_the_full_step():
+    assert run_ranks("rank_batch_shards") == {0: True, 1: True}
+
+
+def test_tensor_parallel_head_shards_reassemble_the_full_step():
+    assert run_ranks("rank_tp_shards") == {0: True, 1: True}
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    assert run_ranks("rank_reference_arm") == {0: 0, 1: 0}
+
+
+def test_shard_helpers():
+    from gqa_mqa_kv_b200.sharding import batch_shard, tp_head_shard
+
+    assert [batch_shard(7, 3, r) for r in range(3)] == [slice(0, 2), slice(2, 4), slice(4, 7)]
+    assert tp_head_shard(64, 8, 8, 3) == (slice(24, 32), slice(3, 4))
+    with pytest.raises(ValueError):
+        tp_head_shard(32, 4, 8, 0)  # TP > H_KV needs duplication
