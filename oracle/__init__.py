@@ -63,6 +63,8 @@ def _load():
             lib.oracle_lse_combine.restype = i32
             lib.oracle_kv_cache_bytes.argtypes = [i64, i64, i64, i64, i64]
             lib.oracle_kv_cache_bytes.restype = dbl
+            lib.oracle_rope.argtypes = [vp, i32, i32, i32, i32, vp, dbl, i32, vp]
+            lib.oracle_rope.restype = i32
             lib.oracle_hardware_threads.argtypes = []
             lib.oracle_hardware_threads.restype = i32
             _lib = lib
@@ -191,6 +193,22 @@ def kv_cache_bytes(layers, tokens, h_kv, d, elem_bytes=2):
     """2 x layers x tokens x KV heads x head dim x bytes per element."""
     return _load().oracle_kv_cache_bytes(int(layers), int(tokens), int(h_kv), int(d),
                                          int(elem_bytes))
+
+
+def rope(x, positions, base=10000.0, pairing="adjacent"):
+    """fp64 rotary embedding of x [B, H, D] at positions [B] -> float64 [B, H, D].
+
+    pairing "adjacent" rotates (2i, 2i+1); "halves" rotates (i, i + D/2).
+    """
+    xa, xt = _as_array(x)
+    pa = _lens(positions)
+    B, H, D = xa.shape
+    out = np.zeros((B, H, D), dtype=np.float64)
+    code = {"adjacent": 0, "halves": 1}[pairing]
+    rc = _load().oracle_rope(_ptr(xa), xt, B, H, D, _ptr(pa), float(base), code, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_rope rejected its arguments")
+    return out
 
 
 def hardware_threads() -> int:

@@ -266,6 +266,36 @@ double oracle_kv_cache_bytes(int64_t layers, int64_t tokens, int64_t H_KV, int64
            static_cast<double>(H_KV) * static_cast<double>(d) * static_cast<double>(elem_bytes);
 }
 
+// Rotary position embedding of every row of x [B, H, D] at position pos[b]
+// ([LLMS] section 4, "Rotary Position Embeddings (RoPE) Interaction":
+// R_{Theta,m} = diag(R_{theta_1,m}, ..., R_{theta_{d/2},m}), one 2x2 rotation
+// by angle m * theta_i per coordinate pair).  Readings: theta_i =
+// base^(-2(i-1)/d) for i = 1..d/2 (the RoFormer frequencies the page cites);
+// pairing 0 rotates adjacent coordinates (2i, 2i+1), the block-diagonal form
+// as written; pairing 1 rotates (i, i + d/2).  out is [B, H, D] double.
+int oracle_rope(const void* x, int dtype, int B, int H, int D, const int32_t* pos, double base,
+                int pairing, double* out) {
+    if (!x || !pos || !out || B < 0 || H <= 0 || D <= 0 || D % 2 != 0 || !(base > 0.0)) return 1;
+    if (dtype < IN_BF16 || dtype > IN_F64 || (pairing != 0 && pairing != 1)) return 1;
+    const int half = D / 2;
+    for (int b = 0; b < B; ++b) {
+        const double m = static_cast<double>(pos[b]);
+        for (int h = 0; h < H; ++h) {
+            const int64_t row = (static_cast<int64_t>(b) * H + h) * D;
+            for (int i = 0; i < half; ++i) {
+                const double theta = std::pow(base, -2.0 * i / D);
+                const double c = std::cos(m * theta), sn = std::sin(m * theta);
+                const int i0 = pairing == 0 ? 2 * i : i;
+                const int i1 = pairing == 0 ? 2 * i + 1 : i + half;
+                const double x0 = load_elem(x, dtype, row + i0), x1 = load_elem(x, dtype, row + i1);
+                out[row + i0] = x0 * c - x1 * sn;
+                out[row + i1] = x0 * sn + x1 * c;
+            }
+        }
+    }
+    return 0;
+}
+
 int oracle_hardware_threads(void) {
     return static_cast<int>(std::thread::hardware_concurrency());
 }
