@@ -222,7 +222,7 @@ cudaError_t launch_mma_groups(const gqa_decode_params* p, const Buffers& buf,
     const int R = p->H_Q / p->H_KV;
     if (R <= 8) return launch_mma<D, 1, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (R <= 16) return launch_mma<D, 2, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
-    if (R <= 32) return launch_mma<D, 4, 1, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
+    if (R <= 32) return launch_mma<D, 2, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     return launch_mma<D, 4, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
 }
 

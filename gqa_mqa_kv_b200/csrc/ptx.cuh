@@ -157,14 +157,14 @@ __device__ __forceinline__ uint32_t pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 
 }
 
 // Splits two fp32 values into bf16 hi parts and bf16 residual parts so that
-// hi + lo carries about 16 significant bits of each value.
+// hi + lo carries about 16 significant bits of each value.  x0 lands in the
+// low half of each packed word.
 __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    __nv_bfloat16 h0 = __float2bfloat16_rn(x0);
-    __nv_bfloat16 h1 = __float2bfloat16_rn(x1);
-    __nv_bfloat16 l0 = __float2bfloat16_rn(x0 - __bfloat162float(h0));
-    __nv_bfloat16 l1 = __float2bfloat16_rn(x1 - __bfloat162float(h1));
-    hi = pack_bf16x2(h0, h1);
-    lo = pack_bf16x2(l0, l1);
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // ---------------------------------------------------------------- special functions

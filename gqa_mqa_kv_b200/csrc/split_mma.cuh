@@ -13,8 +13,10 @@
 //     loads (128-byte swizzle, L2 evict-first for the cache), completing on
 //     mbarriers.  Paged caches only change the tile coordinate: the page id
 //     from the block table replaces (token, sequence).
-//   * NTG x HG consumer warps (four in all): head group hg (ROWS = 8*NT query
-//     heads) x token group tg (64/NTG tokens of each tile).  The contraction is laid out
+//   * consumer warps: head group hg (ROWS = 8*NT query heads) x token group tg
+//     (64/NTG tokens of each tile) x tile set (with 8 heads per warp, two
+//     sets of four warps take alternate tiles so two dependency chains share
+//     each SM sub-partition).  The contraction is laid out
 //     token-major: per 16-token chunk a warp computes S^T = K Q^T with
 //     mma.sync m16n8k16 (tokens on M, heads on N, so no rows are padding),
 //     masks tokens >= L_b, updates an fp32 online softmax per head (column),
@@ -33,16 +35,22 @@
 
 namespace gqa {
 
+// Largest base-2 growth of the running maximum absorbed without rescaling.
+constexpr float kLazyRescale = 8.f;
+
 template <int D, int NT, int HG>
 struct MmaCfg {
     static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
     static_assert(NT == 1 || NT == 2 || NT == 4, "8, 16 or 32 query heads per warp");
     static_assert(HG == 1 || HG == 2, "head groups: 1 or 2");
     static constexpr int ROWS = 8 * NT;                 // query heads per warp
-    static constexpr bool Q_IN_REGS = NT <= 2;          // else Q fragments are re-read from smem
-    static constexpr int NTG = 4 / HG;                  // token groups
+    static constexpr int NTG = (NT == 4 && HG == 2) ? 2 : 4;  // token groups
+    static constexpr bool Q_IN_REGS = NT <= 2 && NTG * HG == 4;  // else Q is re-read from smem
+    static constexpr int TS = NT == 1 ? 2 : 1;          // tile sets taking alternate tiles
     static constexpr int TPW = kTile / NTG;             // tokens per warp per tile
-    static constexpr int NC = NTG * HG;                 // consumer warps
+    static constexpr int MGN = NTG * TS;                // partial softmax states per head group
+    static constexpr int NC = NTG * HG * TS;            // consumer warps
+    static constexpr int TILE_WARPS = NTG * HG;         // consumer warps reading one tile
     static constexpr int THREADS = 32 * (NC + 1);
     static constexpr int PANELS = D / 64;               // 128-byte-wide column panels
     static constexpr int PANEL_BYTES = kTile * 128;     // 64 tokens x 64 bf16
@@ -50,8 +58,8 @@ struct MmaCfg {
     static constexpr int QPANEL_BYTES = ROWS * 128;     // ROWS query rows x 64 bf16
     static constexpr int QSLOT_BYTES = HG * PANELS * QPANEL_BYTES;
     static constexpr int OROW = D + 4;                  // padded merge row (floats)
-    static constexpr int MERGE_O_FLOATS = (NTG - 1) * HG * ROWS * OROW;
-    static constexpr int MERGE_ML_FLOATS = (NTG - 1) * HG * ROWS * 2;
+    static constexpr int MERGE_O_FLOATS = (MGN - 1) * HG * ROWS * OROW;
+    static constexpr int MERGE_ML_FLOATS = (MGN - 1) * HG * ROWS * 2;
     static constexpr int MAX_STAGES = 8;
     static constexpr int CTRL_BYTES = 256;
     static constexpr int FIXED_BYTES =
@@ -100,13 +108,13 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_addr(&ctrl->full[s]), 1);
-            mbar_init(smem_addr(&ctrl->empty[s]), C::NC);
+            mbar_init(smem_addr(&ctrl->empty[s]), C::TILE_WARPS);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->qfull[s]), 1);
             mbar_init(smem_addr(&ctrl->qempty[s]), C::NC);
         }
-        mbar_init(smem_addr(&ctrl->merge_full), (C::NTG - 1) * HG);
+        mbar_init(smem_addr(&ctrl->merge_full), (C::MGN - 1) * HG);
         mbar_init(smem_addr(&ctrl->merge_free), HG);
         ctrl->abort = 0;
     }
@@ -202,8 +210,10 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     // Fragment ownership (g = lane / 4, t = lane % 4):
     //   S^T, P:  token n0 + g (+8)      x head 8 nt + 2t (+1)
     //   O^T:     d 16 mm + g (+8)       x head 8 nt + 2t (+1)
-    const int hg = warp / C::NTG;
+    const int tset = warp / (C::NTG * HG);          // which alternate tiles this warp takes
+    const int hg = (warp / C::NTG) % HG;
     const int tg = warp % C::NTG;
+    const int mg = tset * C::NTG + tg;              // partial-state index; 0 merges
     const int g = lane >> 2;
     const int t = lane & 3;
     const float NEG_INF = -__int_as_float(0x7f800000);
@@ -268,6 +278,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                 for (int nt = 0; nt < NT; ++nt) o[mm][nt][0] = o[mm][nt][1] = o[mm][nt][2] = o[mm][nt][3] = 0.f;
         }
 
+        const bool mine = C::TS == 1 || ((gi - lo) % C::TS) == tset;  // tiles alternate between tile sets
+        if (mine) {
         if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { fail(); break; }
         const uint32_t kb = stages + st * C::STAGE_BYTES;
         const uint32_t vb = kb + C::PANELS * C::PANEL_BYTES;
@@ -345,7 +357,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                 vmask_b = (ta + 8 < w.L ? 0x0000ffffu : 0u) | (ta + 9 < w.L ? 0xffff0000u : 0u);
             }
 
-            // Online softmax per head column: reduce over the 8 lanes that share t.
+            // Online softmax per head column: reduce over the 8 lanes that share
+            // t.  The reference m moves only when the chunk maximum exceeds it
+            // by more than kLazyRescale (base 2), so weights stay <= 2^8 and
+            // the accumulator is rarely rescaled; o / l is unchanged by the
+            // choice of reference.
             float p[NT][4], alpha[NT][2];
             bool rescale = false;
 #pragma unroll
@@ -356,14 +372,16 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
                     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
-                    const float mn = fmaxf(m[nt][j], mx);
-                    const float ref = mn == NEG_INF ? 0.f : mn;
-                    alpha[nt][j] = fast_exp2(m[nt][j] - ref);
-                    m[nt][j] = mn;
+                    alpha[nt][j] = 1.f;
+                    if (mx > m[nt][j] + kLazyRescale) {  // also the first live chunk (m = -inf)
+                        alpha[nt][j] = fast_exp2(m[nt][j] - mx);
+                        m[nt][j] = mx;
+                        rescale = true;
+                    }
+                    const float ref = m[nt][j] == NEG_INF ? 0.f : m[nt][j];
                     p[nt][j] = fast_exp2(s[nt][j] - ref);
                     p[nt][j + 2] = fast_exp2(s[nt][j + 2] - ref);
                     l[nt][j] = l[nt][j] * alpha[nt][j] + (p[nt][j] + p[nt][j + 2]);
-                    rescale |= alpha[nt][j] != 1.f;
                 }
             if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
@@ -402,10 +420,12 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                     const int pnl = mm >> 2, ch = ((mm & 3) << 1) + ((lane >> 3) & 1);
                     ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + vrow * 128 + ((ch ^ (lane & 7)) << 4), va[h][0],
                                   va[h][1], va[h][2], va[h][3]);
-                    va[h][0] &= vmask_a;
-                    va[h][1] &= vmask_a;
-                    va[h][2] &= vmask_b;
-                    va[h][3] &= vmask_b;
+                    if (mask) {  // rows past L_b may hold anything; 0 * NaN would poison O
+                        va[h][0] &= vmask_a;
+                        va[h][1] &= vmask_a;
+                        va[h][2] &= vmask_b;
+                        va[h][3] &= vmask_b;
+                    }
                 }
 #pragma unroll
                 for (int h = 0; h < MG; ++h)
@@ -419,6 +439,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_addr(&ctrl->empty[st]));
+        }  // mine
         if (++st == NS) { st = 0; ph ^= 1u; }
 
         if (seg_last) {
@@ -436,11 +457,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                     l[nt][j] += __shfl_xor_sync(0xffffffffu, l[nt][j], 16);
                 }
             const bool whole = (seg_start_tile == 0) && last_tile;
-            if (tg > 0) {
+            if (mg > 0) {
                 if (!mbar_wait_warp(smem_addr(&ctrl->merge_free), mfree_ph ^ 1u, abort_flag)) { fail(); break; }
                 mfree_ph ^= 1u;
-                float* mo = merge_o + ((tg - 1) * HG + hg) * C::ROWS * C::OROW;
-                float* ml = merge_ml + ((tg - 1) * HG + hg) * C::ROWS * 2;
+                float* mo = merge_o + ((mg - 1) * HG + hg) * C::ROWS * C::OROW;
+                float* ml = merge_ml + ((mg - 1) * HG + hg) * C::ROWS * 2;
                 if (g == 0) {
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt)
@@ -470,7 +491,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                         const int hl = 8 * nt + 2 * t + j;
                         float mx = m[nt][j];
 #pragma unroll
-                        for (int k = 1; k < C::NTG; ++k)
+                        for (int k = 1; k < C::MGN; ++k)
                             mx = fmaxf(mx, merge_ml[(((k - 1) * HG + hg) * C::ROWS + hl) * 2]);
                         M[nt][j] = mx;
                         const float ref = mx == NEG_INF ? 0.f : mx;
@@ -482,7 +503,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                             o[mm][nt][j + 2] *= f;
                         }
 #pragma unroll
-                        for (int k = 1; k < C::NTG; ++k) {
+                        for (int k = 1; k < C::MGN; ++k) {
                             const float* ml = merge_ml + (((k - 1) * HG + hg) * C::ROWS + hl) * 2;
                             const float* mo = merge_o + (((k - 1) * HG + hg) * C::ROWS + hl) * C::OROW;
                             const float e = fast_exp2(ml[0] - ref);
