@@ -23,6 +23,7 @@ import threading
 
 __all__ = [
     "GqaError", "Params", "gqa_decode", "gqa_decode_timed", "gqa_decode_static_workspace",
+    "gqa_rope_append", "FLAG_BAD_POSITION",
     "workspace_bytes", "make_workspace",
     "read_status", "kv_cache_bytes", "library", "LIB_PATH", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_BAD_BLOCK", "FLAG_TIMEOUT", "PAGE_SIZE",
@@ -31,11 +32,13 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa_decode.so")
 PAGE_SIZE = 64
 GQA_BF16, GQA_F32 = 0, 1
-FLAG_SEQ_LEN_CLAMPED, FLAG_BAD_BLOCK, FLAG_TIMEOUT = 1, 2, 4
+FLAG_SEQ_LEN_CLAMPED, FLAG_BAD_BLOCK, FLAG_TIMEOUT, FLAG_BAD_POSITION = 1, 2, 4, 8
+ROPE_PAIRING = {"adjacent": 0, "halves": 1}
 
 EXPORTED = (
     "gqa_decode_workspace_size", "gqa_decode", "gqa_decode_timed", "gqa_read_status",
     "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version", "gqa_decode_static_workspace",
+    "gqa_rope_append",
 )
 
 
@@ -93,6 +96,9 @@ def library() -> ctypes.CDLL:
             lib.gqa_decode_static_workspace.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_float, vp,
                                                         vp]
             lib.gqa_decode_static_workspace.restype = ctypes.c_int
+            lib.gqa_rope_append.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_int, vp,
+                                            vp, vp, vp, vp, vp]
+            lib.gqa_rope_append.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -282,6 +288,44 @@ def gqa_decode_static_workspace(q, k_cache, v_cache, seq_lens, block_table=None,
     if st != 0:
         raise GqaError(st, "gqa_decode_static_workspace")
     return out
+
+
+def gqa_rope_append(q, k_new, v_new, positions, k_cache, v_cache, block_table=None,
+                    rope_base=10000.0, pairing="adjacent", q_out=None, seq_lens_out=None,
+                    workspace=None, stream=None, max_seq_len=None):
+    """RoPE on the new token's query heads (returned) and key heads, appended with
+    its value rows to the cache at positions[b]; optionally seq_lens_out[b] = positions[b] + 1.
+
+    q [B, H_Q, D]; k_new, v_new [B, H_KV, D]; positions int32 [B]; caches as in
+    gqa_decode.  q_out may be q itself.  Enqueued on the current stream.
+    """
+    import torch
+
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("positions", positions),
+                    ("k_cache", k_cache), ("v_cache", v_cache)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    B, H_Q, D = q.shape
+    H_KV = k_cache.shape[2]
+    if k_new.shape != (B, H_KV, D) or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must be [B, H_KV, D]")
+    if positions.dtype != torch.int32 or positions.shape != (B,):
+        raise ValueError("positions must be int32 [B]")
+    if not (q.dtype == k_new.dtype == v_new.dtype == k_cache.dtype == v_cache.dtype):
+        raise ValueError("q, k_new, v_new and the caches must share a dtype")
+    params = make_params(q, k_cache, positions, block_table, None, max_seq_len)
+    if q_out is None:
+        q_out = torch.empty_like(q)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opt = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else None)  # noqa: E731
+    st = library().gqa_rope_append(
+        ctypes.byref(params), opt(q), opt(k_new), opt(v_new), opt(positions), opt(block_table),
+        ctypes.c_double(rope_base), ROPE_PAIRING[pairing], opt(q_out), opt(k_cache), opt(v_cache),
+        opt(seq_lens_out), opt(workspace), ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise GqaError(st, "gqa_rope_append")
+    return q_out
 
 
 def read_status(workspace, stream=None, clear=False) -> int:

@@ -9,6 +9,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <set>
@@ -18,6 +19,7 @@
 #include "combine.cuh"
 #include "split_mma.cuh"
 #include "split_simt.cuh"
+#include "rope_append.cuh"
 
 namespace {
 
@@ -342,6 +344,23 @@ gqa_status static_workspace_on_current_device(void** ptr, cudaStream_t stream) {
     return GQA_OK;
 }
 
+// ------------------------------------------------------------------ RoPE + append
+
+bool ranges_overlap(const void* a, size_t na, const void* b, size_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + nb && y < x + na;
+}
+
+template <typename T>
+cudaError_t launch_rope(const void* q, const void* k_new, const void* v_new, void* q_out, void* k_cache,
+                        void* v_cache, const RopeArgs& ra, cudaStream_t stream) {
+    const int64_t rows = static_cast<int64_t>(ra.B) * (ra.H_Q + ra.H_KV);
+    const int blocks = static_cast<int>((rows + 3) / 4);
+    return launch_chained(rope_append_kernel<T>, blocks, 128, 0, stream, static_cast<const T*>(q),
+                          static_cast<const T*>(k_new), static_cast<const T*>(v_new), static_cast<T*>(q_out),
+                          static_cast<T*>(k_cache), static_cast<T*>(v_cache), ra);
+}
+
 }  // namespace
 
 extern "C" {
@@ -388,6 +407,51 @@ gqa_status gqa_decode_static_workspace(const gqa_decode_params* params, const vo
         return st;
     return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, ws,
                kStaticWorkspaceBytes, stream, nullptr, nullptr);
+}
+
+gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const void* k_new,
+                           const void* v_new, const int32_t* positions, const int32_t* block_table,
+                           double rope_base, int pairing, void* q_out, void* k_cache, void* v_cache,
+                           int32_t* seq_lens_out, void* workspace, void* stream) {
+    gqa_status st = validate_params(params);
+    if (st != GQA_OK) return st;
+    if (params->B == 0) return GQA_OK;
+    if (!q || !k_new || !v_new || !positions || !q_out || !k_cache || !v_cache) return GQA_ERR_INVALID;
+    if ((params->page_size != 0) != (block_table != nullptr)) return GQA_ERR_INVALID;
+    if (!(rope_base > 0.0) || rope_base > 1e300 || (pairing != GQA_ROPE_ADJACENT && pairing != GQA_ROPE_HALVES))
+        return GQA_ERR_INVALID;
+    const void* bufs[] = {q, k_new, v_new, q_out, k_cache, v_cache};
+    for (const void* p : bufs)
+        if (!aligned(p, 16)) return GQA_ERR_INVALID;
+    if (!aligned(positions, 4) || (seq_lens_out && !aligned(seq_lens_out, 4)) ||
+        (block_table && !aligned(block_table, 4)))
+        return GQA_ERR_INVALID;
+    const size_t lens_bytes = sizeof(int32_t) * static_cast<size_t>(params->B);
+    if (seq_lens_out && ranges_overlap(seq_lens_out, lens_bytes, positions, lens_bytes)) return GQA_ERR_INVALID;
+    if (workspace && !aligned(workspace, 256)) return GQA_ERR_WORKSPACE;
+
+    RopeArgs ra;
+    std::memset(&ra, 0, sizeof ra);
+    ra.B = params->B;
+    ra.H_Q = params->H_Q;
+    ra.H_KV = params->H_KV;
+    ra.D = params->head_dim;
+    ra.max_len = params->page_size ? params->max_blocks_per_seq * kTile : params->max_seq_len;
+    if (params->page_size && params->max_seq_len < ra.max_len) ra.max_len = params->max_seq_len;
+    ra.S_max = params->page_size ? 0 : params->max_seq_len;
+    ra.max_blocks = params->max_blocks_per_seq;
+    ra.num_blocks = params->num_blocks;
+    ra.positions = positions;
+    ra.block_table = block_table;
+    ra.seq_lens_out = seq_lens_out;
+    ra.status = static_cast<uint32_t*>(workspace);
+    ra.log2_base = std::log2(rope_base);
+    ra.halves = pairing == GQA_ROPE_HALVES;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const cudaError_t e = params->qkv_dtype == GQA_F32
+                              ? launch_rope<float>(q, k_new, v_new, q_out, k_cache, v_cache, ra, s)
+                              : launch_rope<__nv_bfloat16>(q, k_new, v_new, q_out, k_cache, v_cache, ra, s);
+    return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 gqa_status gqa_read_status(const void* workspace, void* stream, uint32_t* flags, int clear) {

@@ -63,10 +63,17 @@ typedef enum gqa_dtype {
     GQA_F32 = 1
 } gqa_dtype;
 
+/* Coordinate pairs a rotary embedding turns together. */
+typedef enum gqa_rope_pairing {
+    GQA_ROPE_ADJACENT = 0,  /* (2i, 2i+1): the block-diagonal R_{Theta,m} as written */
+    GQA_ROPE_HALVES = 1     /* (i, i + head_dim/2) */
+} gqa_rope_pairing;
+
 /* Device status flags, accumulated (bitwise OR) in the workspace. */
 #define GQA_FLAG_SEQ_LEN_CLAMPED 1u   /* a seq_lens entry was < 0 or > max_seq_len */
 #define GQA_FLAG_BAD_BLOCK 2u         /* a live block_table entry was outside [0, num_blocks) */
 #define GQA_FLAG_TIMEOUT 4u           /* an internal pipeline wait gave up; outputs invalid */
+#define GQA_FLAG_BAD_POSITION 8u      /* a rope/append position was outside [0, max_seq_len) */
 
 /*
  * Problem description.  All counts are element counts.
@@ -175,6 +182,42 @@ gqa_status gqa_decode_static_workspace(const gqa_decode_params* params, const vo
                                        const void* k_cache, const void* v_cache,
                                        const int32_t* seq_lens, const int32_t* block_table,
                                        float scale, void* out, void* stream);
+
+/*
+ * The step before gqa_decode for a new token: rotary position embedding of
+ * its query heads, and the append of its key and value rows to the cache.
+ * [LLMS] section 4, "Rotary Position Embeddings (RoPE) Interaction": RoPE is
+ * applied to each of the H_Q query heads and once to each of the H_KV key
+ * heads, R_{Theta,m} = diag(R_{theta_1,m}, ..., R_{theta_{d/2},m}) with the
+ * token's position m; theta_i = rope_base^(-2i/head_dim), i = 0..head_dim/2-1
+ * (the RoFormer frequencies the page cites; e.g. rope_base 10000).
+ *
+ * For every b, with m = positions[b] (the number of tokens already cached):
+ *   q_out[b,h,:]              = RoPE_m(q[b,h,:])            h < H_Q
+ *   cache row (b, m, g) of k  = RoPE_m(k_new[b,g,:])        g < H_KV
+ *   cache row (b, m, g) of v  = v_new[b,g,:]
+ *   seq_lens_out[b]           = m + 1                        (if not NULL)
+ * The cache row is k_cache[b][m][g] (contiguous) or
+ * k_cache[block_table[b][m/64]][m%64][g] (paged), as in gqa_decode.
+ *
+ *   params      as for gqa_decode (cache geometry, qkv_dtype; out_dtype unused)
+ *   q, q_out    [B, H_Q, head_dim]; q_out may equal q (in place)
+ *   k_new,v_new [B, H_KV, head_dim]
+ *   positions   int32 [B], device
+ *   pairing     gqa_rope_pairing
+ *   seq_lens_out int32 [B] device or NULL; must not overlap positions
+ *   workspace   a gqa_decode workspace (status word) or NULL
+ * Angles and rotations are evaluated in double and rounded once to the
+ * storage type.  A position outside [0, max_seq_len) (or a page outside
+ * [0, num_blocks)) skips that sequence's cache write and raises
+ * GQA_FLAG_BAD_POSITION (GQA_FLAG_BAD_BLOCK) in the workspace status word.
+ * Enqueued on `stream`, chained so that a following gqa_decode may launch
+ * early; argument errors return before anything is enqueued.
+ */
+gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const void* k_new,
+                           const void* v_new, const int32_t* positions, const int32_t* block_table,
+                           double rope_base, int pairing, void* q_out, void* k_cache, void* v_cache,
+                           int32_t* seq_lens_out, void* workspace, void* stream);
 
 /*
  * Reads the workspace status word (GQA_FLAG_* bits) into *flags after

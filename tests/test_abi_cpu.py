@@ -153,3 +153,27 @@ def test_package_does_not_import_the_oracle():
                 text = open(os.path.join(dirpath, f)).read()
                 assert "import oracle" not in text and "from oracle" not in text, f
                 assert "gqa_oracle" not in text, f
+
+
+def call_rope(lib, p, q=16, kn=16, vn=16, pos=16, table=None, base=10000.0, pairing=0, qo=16, kc=16,
+              vc=16, lens_out=None, ws=None):
+    vp = ctypes.c_void_p
+    return lib.gqa_rope_append(ctypes.byref(p), vp(q), vp(kn), vp(vn), vp(pos), vp(table),
+                               ctypes.c_double(base), pairing, vp(qo), vp(kc), vp(vc), vp(lens_out), vp(ws),
+                               vp(None))
+
+
+def test_rope_append_rejects_bad_arguments_on_host(lib):
+    p = params()
+    assert call_rope(lib, params(H_Q=6, H_KV=4)) == GQA_ERR_INVALID
+    assert call_rope(lib, p, base=0.0) == GQA_ERR_INVALID
+    assert call_rope(lib, p, base=float("nan")) == GQA_ERR_INVALID
+    assert call_rope(lib, p, pairing=2) == GQA_ERR_INVALID
+    assert call_rope(lib, p, kn=None) == GQA_ERR_INVALID
+    assert call_rope(lib, p, pos=None) == GQA_ERR_INVALID
+    assert call_rope(lib, p, kc=24) == GQA_ERR_INVALID
+    assert call_rope(lib, p, table=16) == GQA_ERR_INVALID           # table on a contiguous cache
+    assert call_rope(lib, p, pos=4096, lens_out=4100) == GQA_ERR_INVALID  # overlapping int32 [B]
+    assert call_rope(lib, p, ws=128) == GQA_ERR_WORKSPACE
+    assert call_rope(lib, params(B=0), q=None, kn=None, vn=None, pos=None, qo=None, kc=None,
+                     vc=None) == GQA_OK
