@@ -59,6 +59,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--path", default="decode", choices=["decode", "append_decode"],
+                    help="decode: gqa_decode per step; append_decode: gqa_rope_append of the "
+                         "newest token (re-appended at L_b - 1) followed by gqa_decode")
     return ap.parse_args(argv)
 
 
@@ -294,10 +297,31 @@ def run_ours(args):
     stream = torch.cuda.current_stream(dev)
     big = w.seq_len * w.B * w.H_KV * w.D * 4 > 2 * 126e6
     flush = None if big else torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    appending = args.path == "append_decode"
+    if appending:
+        # The newest token of every sequence is (re-)appended at position L_b - 1, so
+        # each step rotates q and k and writes one cache row without growing the cache.
+        gnew = torch.Generator().manual_seed(w.seed + 100)
+        k_new = torch.randn(w.B, w.H_KV, w.D, generator=gnew).to(q.dtype).to(dev)
+        v_new = torch.randn(w.B, w.H_KV, w.D, generator=gnew).to(q.dtype).to(dev)
+        positions = (lens - 1).clamp(min=0)
+        q_in = q.clone()
+        step_bytes += w.B * w.D * q.element_size() * (2 * w.H_Q + 4 * w.H_KV)
+    launches_per_step = 3 if appending else 2
+
+    def append_call(events=None):
+        if events is not None:
+            events[0].record(stream)
+        gq.gqa_rope_append(q_in, k_new, v_new, positions, k, v, table, q_out=q, workspace=ws,
+                           stream=stream)
+        if events is not None:
+            events[1].record(stream)
 
     def step():
         if flush is not None:
             flush.zero_()
+        if appending:
+            append_call()
         gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws, stream=stream)
 
     for _ in range(max(args.warmup, 3)):
@@ -323,6 +347,8 @@ def run_ours(args):
             if flush is not None:
                 flush.zero_()
                 step_ev[i][0].record(stream)
+            if appending:
+                append_call()
             gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws,
                           stream=stream)
             if flush is not None:
@@ -337,9 +363,13 @@ def run_ours(args):
         # pass is not the headline).
         split_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     for _ in range(args.steps)]
+        append_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                     for _ in range(args.steps)] if appending else None
         for i in range(args.steps):
             if flush is not None:
                 flush.zero_()
+            if appending:
+                append_call(append_ev[i])
             gq.gqa_decode_timed(split_ev[i], q, k, v, lens, table, scale=w.softmax_scale, out=out,
                                 workspace=ws, stream=stream)
         torch.cuda.synchronize(dev)
@@ -385,7 +415,7 @@ def run_ours(args):
     peak, peak_kind = hbm_peak()
     ms_per_step = elapsed_ms / args.steps
     value = world * step_bytes / (ms_per_step * 1e-3) / 1e9
-    achieved = step_bytes / (split_ms_max * 1e-3) / 1e9
+    achieved = algorithmic_bytes(w, lens_host) / (split_ms_max * 1e-3) / 1e9
     traffic = recorded_traffic(w.name)
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -400,7 +430,7 @@ def run_ours(args):
                 "d2h_bytes_per_step": world * d2h,
                 "path": "pinned q and seq_lens copied in, gqa_decode, out copied back, every step; "
                         "KV cache resident in HBM"},
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
                      "kernel": "split-KV decode kernel (combine excluded)",
@@ -408,6 +438,10 @@ def run_ours(args):
                      "peak_note": f"{peak_kind} HBM copy bandwidth"},
         "device_status_flags": status,
     }
+    if appending:
+        append_us = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in append_ev), dist, dev) * 1e3
+        line["config"]["path"] = "rope_append + decode"
+        line["append_kernel_us"] = append_us
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_oracle_sample(w, inp, args.cpu_sample_seconds)
     if rank == 0:
