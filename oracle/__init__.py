@@ -48,7 +48,9 @@ def _load():
     global _lib
     with _lock:
         if _lib is None:
-            lib = ctypes.CDLL(build())
+            # ORACLE_LIB points the wrapper at another build of gqa_oracle.cpp
+            # (the mutation tests use it to run the pins against planted mistakes).
+            lib = ctypes.CDLL(os.environ.get("ORACLE_LIB") or build())
             vp, i32, i64, dbl = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_double
             lib.oracle_gqa_decode.argtypes = [vp, i32, vp, vp, i32, vp, i32, i32, i32, i32, i64,
                                               dbl, vp, i64, vp, i32]
