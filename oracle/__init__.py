@@ -29,7 +29,7 @@ _LIB = os.path.join(_HERE, "libgqa_oracle.so")
 _lock = threading.Lock()
 _lib = None
 
-IN_BF16, IN_F32, IN_F64 = 0, 1, 2
+IN_BF16, IN_F32, IN_F64, IN_E4M3 = 0, 1, 2, 3
 
 
 def build(force: bool = False) -> str:
@@ -66,6 +66,11 @@ def _load():
             lib.oracle_kv_cache_bytes.argtypes = [i64, i64, i64, i64, i64]
             lib.oracle_kv_cache_bytes.restype = dbl
             lib.oracle_rope.argtypes = [vp, i32, i32, i32, i32, vp, dbl, i32, vp]
+            lib.oracle_gqa_decode_scaled.argtypes = [vp, i32, vp, vp, i32, vp, vp, vp, i32, i32, i32,
+                                                     i32, i64, dbl, vp, i64, vp, i32]
+            lib.oracle_gqa_decode_scaled.restype = i32
+            lib.oracle_e4m3_table.argtypes = [vp]
+            lib.oracle_e4m3_table.restype = None
             lib.oracle_rope.restype = i32
             lib.oracle_hardware_threads.argtypes = []
             lib.oracle_hardware_threads.restype = i32
@@ -91,6 +96,8 @@ def _as_array(x):
             return x.numpy(), IN_F32
         if x.dtype == torch.float64:
             return x.numpy(), IN_F64
+        if x.dtype == torch.float8_e4m3fn:
+            return x.view(torch.uint8).numpy(), IN_E4M3
         raise TypeError(f"oracle: unsupported dtype {x.dtype}")
     x = np.ascontiguousarray(x)
     if x.dtype == np.uint16:
@@ -143,6 +150,43 @@ def gqa_decode(q, k, v, seq_lens, scale, pairs=None, n_threads=0):
                                    D, S_max, float(scale), pp, n, _ptr(out), int(n_threads))
     if rc != 0:
         raise ValueError("oracle_gqa_decode rejected its arguments")
+    return out
+
+
+def gqa_decode_scaled(q, k, v, seq_lens, scale, k_scale, v_scale, pairs=None, n_threads=0):
+    """fp64 decode over a cache whose stored K/V are multiplied by per-KV-head
+    factors (k_scale, v_scale [H_KV]); k, v may be torch.float8_e4m3fn."""
+    qa, qt = _as_array(q)
+    ka, kt = _as_array(k)
+    va, vt = _as_array(v)
+    if kt != vt:
+        raise TypeError("oracle: k and v must share a dtype")
+    ks = np.ascontiguousarray(np.asarray(k_scale, dtype=np.float64))
+    vs = np.ascontiguousarray(np.asarray(v_scale, dtype=np.float64))
+    lens = _lens(seq_lens)
+    B, H_Q, D = qa.shape
+    Bk, S_max, H_KV, Dk = ka.shape
+    if Bk != B or Dk != D or va.shape != ka.shape or ks.shape != (H_KV,) or vs.shape != (H_KV,):
+        raise ValueError("oracle: inconsistent shapes")
+    if pairs is None:
+        out = np.zeros((B, H_Q, D), dtype=np.float64)
+        pp, n = None, 0
+    else:
+        pa = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32).reshape(-1, 2))
+        out = np.zeros((pa.shape[0], D), dtype=np.float64)
+        pp, n = _ptr(pa), pa.shape[0]
+    rc = _load().oracle_gqa_decode_scaled(_ptr(qa), qt, _ptr(ka), _ptr(va), kt, _ptr(ks), _ptr(vs),
+                                          _ptr(lens), B, H_Q, H_KV, D, S_max, float(scale), pp, n,
+                                          _ptr(out), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_gqa_decode_scaled rejected its arguments")
+    return out
+
+
+def e4m3_table():
+    """float64 [256]: the oracle's decoded value of every E4M3 byte."""
+    out = np.zeros(256, dtype=np.float64)
+    _load().oracle_e4m3_table(_ptr(out))
     return out
 
 

@@ -55,7 +55,21 @@
 
 namespace {
 
-enum InputType { IN_BF16 = 0, IN_F32 = 1, IN_F64 = 2 };
+enum InputType { IN_BF16 = 0, IN_F32 = 1, IN_F64 = 2, IN_E4M3 = 3 };
+
+// OCP 8-bit floating point, E4M3 encoding: sign bit 7, exponent bits 6..3 with
+// bias 7, mantissa bits 2..0; exponent 0 is subnormal (m * 2^-9); S.1111.111 is
+// NaN and there is no infinity, so the largest finite value is 448.
+double decode_e4m3(uint8_t byte) {
+    const int sign = byte >> 7, e = (byte >> 3) & 15, m = byte & 7;
+    double mag;
+    if (e == 15 && m == 7) return std::numeric_limits<double>::quiet_NaN();
+    if (e == 0)
+        mag = std::ldexp(static_cast<double>(m), -9);
+    else
+        mag = std::ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
 
 // Exact widening of one stored element to double.
 double load_elem(const void* base, int dtype, int64_t index) {
@@ -67,6 +81,7 @@ double load_elem(const void* base, int dtype, int64_t index) {
         return static_cast<double>(f);
     }
     if (dtype == IN_F32) return static_cast<double>(static_cast<const float*>(base)[index]);
+    if (dtype == IN_E4M3) return decode_e4m3(static_cast<const uint8_t*>(base)[index]);
     return static_cast<const double*>(base)[index];
 }
 
@@ -80,6 +95,8 @@ struct Problem {
     int B, H_Q, H_KV, D;
     int64_t S_max;
     double scale;
+    const double* k_scale = nullptr;  // [H_KV]: stored keys are multiplied by it (quantised caches)
+    const double* v_scale = nullptr;  // [H_KV]: stored values likewise
 };
 
 int64_t q_index(const Problem& p, int b, int h, int i) {
@@ -105,7 +122,8 @@ double score(const Problem& p, int b, int h, int64_t t) {
     for (int i = 0; i < p.D; ++i)
         acc += load_elem(p.q, p.q_dtype, q_index(p, b, h, i)) *
                load_elem(p.k, p.kv_dtype, kv_index(p, b, t, g, i));
-    return p.scale * acc;
+    const double ks = p.k_scale ? p.k_scale[g] : 1.0;
+    return p.scale * ks * acc;
 }
 
 // Softmax weights over tokens [0, L_b), two passes: max, then exp and sum.
@@ -131,10 +149,11 @@ std::vector<double> softmax_weights(const Problem& p, int b, int h) {
 void attend_one(const Problem& p, int b, int h, double* out) {
     std::vector<double> w = softmax_weights(p, b, h);
     int g = group_of(p, h);
+    const double vs = p.v_scale ? p.v_scale[g] : 1.0;
     for (int i = 0; i < p.D; ++i) out[i] = 0.0;
     for (int64_t t = 0; t < static_cast<int64_t>(w.size()); ++t)
         for (int i = 0; i < p.D; ++i)
-            out[i] += w[t] * load_elem(p.v, p.kv_dtype, kv_index(p, b, t, g, i));
+            out[i] += w[t] * vs * load_elem(p.v, p.kv_dtype, kv_index(p, b, t, g, i));
 }
 
 int check_problem(const Problem& p) {
@@ -142,7 +161,7 @@ int check_problem(const Problem& p) {
     if (p.B < 0 || p.H_Q <= 0 || p.H_KV <= 0 || p.D <= 0 || p.S_max < 0) return 1;
     if (p.H_Q % p.H_KV != 0) return 1;  // [LLMS] section 2: R = H_Q / G is a whole number
     if (p.q_dtype < IN_BF16 || p.q_dtype > IN_F64) return 1;
-    if (p.kv_dtype < IN_BF16 || p.kv_dtype > IN_F64) return 1;
+    if (p.kv_dtype < IN_BF16 || p.kv_dtype > IN_E4M3) return 1;
     for (int b = 0; b < p.B; ++b)
         if (p.seq_lens[b] < 0 || p.seq_lens[b] > p.S_max) return 1;
     return 0;
@@ -191,6 +210,45 @@ int oracle_gqa_decode(const void* q, int q_dtype, const void* k, const void* v, 
     }
     for (auto& t : pool) t.join();
     return 0;
+}
+
+// oracle_gqa_decode for a cache whose stored keys and values are multiplied by
+// per-KV-head factors k_scale[g], v_scale[g] (e.g. an 8-bit cache with
+// kv_dtype 3 = E4M3): K = stored_k * k_scale[g], V = stored_v * v_scale[g].
+int oracle_gqa_decode_scaled(const void* q, int q_dtype, const void* k, const void* v, int kv_dtype,
+                             const double* k_scale, const double* v_scale, const int32_t* seq_lens,
+                             int B, int H_Q, int H_KV, int D, int64_t S_max, double scale,
+                             const int32_t* pairs, int64_t n_pairs, double* out, int n_threads) {
+    Problem p{q, k, v, q_dtype, kv_dtype, seq_lens, B, H_Q, H_KV, D, S_max, scale};
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    if (check_problem(p) || !out || !k_scale || !v_scale) return 1;
+    int64_t n = pairs ? n_pairs : static_cast<int64_t>(B) * H_Q;
+    if (n < 0) return 1;
+    if (pairs) {
+        for (int64_t j = 0; j < n; ++j)
+            if (pairs[2 * j] < 0 || pairs[2 * j] >= B || pairs[2 * j + 1] < 0 ||
+                pairs[2 * j + 1] >= H_Q)
+                return 1;
+    }
+    int nt = thread_count(n_threads, n);
+    std::vector<std::thread> pool;
+    for (int w = 0; w < nt; ++w) {
+        pool.emplace_back([&, w]() {
+            for (int64_t j = w; j < n; j += nt) {
+                int b = pairs ? pairs[2 * j] : static_cast<int>(j / H_Q);
+                int h = pairs ? pairs[2 * j + 1] : static_cast<int>(j % H_Q);
+                attend_one(p, b, h, out + j * D);
+            }
+        });
+    }
+    for (auto& t : pool) t.join();
+    return 0;
+}
+
+// Decoded value of every E4M3 byte 0..255 (out[256]), for pinning the decoder.
+void oracle_e4m3_table(double* out) {
+    for (int i = 0; i < 256; ++i) out[i] = decode_e4m3(static_cast<uint8_t>(i));
 }
 
 // The normalised softmax weights w_t, t in [0, L_b), of one (b, h) pair.

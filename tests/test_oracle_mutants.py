@@ -17,12 +17,12 @@ SRC = os.path.join(ROOT, "oracle", "gqa_oracle.cpp")
 
 MUTANTS = {
     "strided_group_map": ("    return h / R;", "    return h % p.H_KV;"),
-    "dropped_scale": ("    return p.scale * acc;", "    return acc;"),
+    "dropped_scale": ("    return p.scale * ks * acc;", "    return ks * acc;"),
     "exponent_sign": ("        s[t] = std::exp(s[t] - m);", "        s[t] = std::exp(m - s[t]);"),
     "drops_last_token": ("    int64_t L = p.seq_lens[b];\n    std::vector<double> s(",
                          "    int64_t L = p.seq_lens[b] > 1 ? p.seq_lens[b] - 1 : p.seq_lens[b];\n    std::vector<double> s("),
-    "values_from_keys": ("            out[i] += w[t] * load_elem(p.v, p.kv_dtype, kv_index(p, b, t, g, i));",
-                         "            out[i] += w[t] * load_elem(p.k, p.kv_dtype, kv_index(p, b, t, g, i));"),
+    "values_from_keys": ("            out[i] += w[t] * vs * load_elem(p.v, p.kv_dtype, kv_index(p, b, t, g, i));",
+                         "            out[i] += w[t] * vs * load_elem(p.k, p.kv_dtype, kv_index(p, b, t, g, i));"),
     "batch_stride": ("    return ((static_cast<int64_t>(b) * p.S_max + t) * p.H_KV + g) * p.D + i;",
                      "    return ((static_cast<int64_t>(b) * (p.S_max > 1 ? p.S_max - 1 : 1) + t) * p.H_KV + g) * p.D + i;"),
     "query_stride": ("    return (static_cast<int64_t>(b) * p.H_Q + h) * p.D + i;",
@@ -36,11 +36,14 @@ MUTANTS = {
     "rope_frequency": ("                const double theta = std::pow(base, -2.0 * i / D);",
                        "                const double theta = std::pow(base, -1.0 * i / D);"),
     "rope_rotation_sign": ("                out[row + i1] = x0 * sn + x1 * c;", "                out[row + i1] = -x0 * sn + x1 * c;"),
+    "e4m3_bias": ("        mag = std::ldexp(1.0 + m / 8.0, e - 7);", "        mag = std::ldexp(1.0 + m / 8.0, e - 8);"),
+    "e4m3_subnormal": ("        mag = std::ldexp(static_cast<double>(m), -9);", "        mag = std::ldexp(static_cast<double>(m), -10);"),
+    "value_scale_dropped": ("    const double vs = p.v_scale ? p.v_scale[g] : 1.0;", "    const double vs = 1.0;"),
     "rope_pairing": ("                const int i1 = pairing == 0 ? 2 * i + 1 : i + half;",
                      "                const int i1 = pairing == 0 ? 2 * i + 1 : i + half - 1;"),
 }
 
-PIN_SUITES = ["tests/test_oracle_pins.py", "tests/test_oracle_rope_pins.py"]
+PIN_SUITES = ["tests/test_oracle_pins.py", "tests/test_oracle_rope_pins.py", "tests/test_oracle_fp8_pins.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
