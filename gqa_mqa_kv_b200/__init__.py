@@ -23,7 +23,7 @@ import threading
 
 __all__ = [
     "GqaError", "Params", "gqa_decode", "gqa_decode_timed", "gqa_decode_static_workspace",
-    "gqa_rope_append", "FLAG_BAD_POSITION",
+    "gqa_rope_append", "gqa_decode_fp8kv", "FLAG_BAD_POSITION",
     "workspace_bytes", "make_workspace",
     "read_status", "kv_cache_bytes", "library", "LIB_PATH", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_BAD_BLOCK", "FLAG_TIMEOUT", "PAGE_SIZE",
@@ -38,7 +38,7 @@ ROPE_PAIRING = {"adjacent": 0, "halves": 1}
 EXPORTED = (
     "gqa_decode_workspace_size", "gqa_decode", "gqa_decode_timed", "gqa_read_status",
     "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version", "gqa_decode_static_workspace",
-    "gqa_rope_append",
+    "gqa_rope_append", "gqa_decode_fp8kv",
 )
 
 
@@ -99,6 +99,9 @@ def library() -> ctypes.CDLL:
             lib.gqa_rope_append.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_int, vp,
                                             vp, vp, vp, vp, vp]
             lib.gqa_rope_append.restype = ctypes.c_int
+            lib.gqa_decode_fp8kv.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz,
+                                             vp]
+            lib.gqa_decode_fp8kv.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -326,6 +329,51 @@ def gqa_rope_append(q, k_new, v_new, positions, k_cache, v_cache, block_table=No
     if st != 0:
         raise GqaError(st, "gqa_rope_append")
     return q_out
+
+
+def gqa_decode_fp8kv(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_table=None,
+                     scale=None, out=None, out_dtype=None, workspace=None, stream=None,
+                     max_seq_len=None):
+    """gqa_decode over an 8-bit cache: k_cache, v_cache hold E4M3 values
+    (torch.float8_e4m3fn or their uint8 bytes) multiplied by per-KV-head
+    k_scale, v_scale (float32 [H_KV]).  q is bf16."""
+    import torch
+
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("seq_lens", seq_lens),
+                    ("k_scale", k_scale), ("v_scale", v_scale)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if q.dtype != torch.bfloat16:
+        raise ValueError("q must be bf16 for an 8-bit cache")
+    if k_cache.dtype not in (torch.float8_e4m3fn, torch.uint8) or v_cache.dtype != k_cache.dtype:
+        raise ValueError("k_cache and v_cache must be float8_e4m3fn (or uint8 bytes)")
+    if k_cache.shape != v_cache.shape:
+        raise ValueError("k_cache and v_cache must match in shape")
+    H_KV = k_cache.shape[2]
+    for name, t in (("k_scale", k_scale), ("v_scale", v_scale)):
+        if t.dtype != torch.float32 or t.shape != (H_KV,):
+            raise ValueError(f"{name} must be float32 [H_KV]")
+    if seq_lens.dtype != torch.int32 or seq_lens.shape != (q.shape[0],):
+        raise ValueError("seq_lens must be int32 [B]")
+    params = make_params(q, k_cache, seq_lens, block_table, out_dtype if out is None else out.dtype,
+                         max_seq_len)
+    params.qkv_dtype = GQA_BF16
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or torch.float32, device=q.device)
+    if workspace is None:
+        workspace = make_workspace(params, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opt = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else None)  # noqa: E731
+    st = library().gqa_decode_fp8kv(
+        ctypes.byref(params), opt(q), opt(k_cache), opt(v_cache), opt(k_scale), opt(v_scale),
+        opt(seq_lens), opt(block_table), ctypes.c_float(scale), opt(out), opt(workspace),
+        ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise GqaError(st, "gqa_decode_fp8kv")
+    return out
 
 
 def read_status(workspace, stream=None, clear=False) -> int:

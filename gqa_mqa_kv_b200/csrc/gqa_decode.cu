@@ -112,9 +112,9 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// bf16 tensor map, 128-byte swizzle, out-of-bounds elements read as zero.
-bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                 const uint64_t* strides_bytes, const uint32_t* box) {
+// Tiled tensor map with a 128-byte swizzle; out-of-bounds elements read as zero.
+bool encode_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank,
+                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t d[5], s[4];
@@ -125,7 +125,7 @@ bool encode_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* d
         es[i] = 1;
         if (i + 1 < rank) s[i] = strides_bytes[i];
     }
-    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+    return fn(map, type, static_cast<cuuint32_t>(rank),
               const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -168,17 +168,27 @@ struct Buffers {
     const void* q;
     const void* k;
     const void* v;
+    bool kv8;  // k and v hold E4M3 bytes (scales in KernelArgs)
 };
 
-template <int D, int NT, int HG, bool PAGED, bool OUTB>
+template <int D, int NT, int HG, bool PAGED, bool OUTB, bool KV8 = false>
 cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArgs args,
                        const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
-    using C = MmaCfg<D, NT, HG>;
+    using C = MmaCfg<D, NT, HG, KV8>;
     const int R = p->H_Q / p->H_KV;
-    int stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
-    if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
+    int stages, stages8 = 0;
+    if constexpr (KV8) {  // 4 decoded stages; the rest of shared memory stages 8-bit tiles
+        stages = 4;
+        stages8 = (dev.smem_optin - C::FIXED_BYTES - 1024 - stages * C::STAGE_BYTES) / C::STAGE8_BYTES;
+        if (stages8 > C::MAX_STAGES) stages8 = C::MAX_STAGES;
+        if (stages8 < 2) return cudaErrorInvalidConfiguration;
+    } else {
+        stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
+        if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
+    }
     if (stages < 2) return cudaErrorInvalidConfiguration;
     args.n_stages = stages;
+    args.n_stages8 = stages8;
     args.q_rows = R < C::ROWS ? R : C::ROWS;
     args.q_groups = (R + C::ROWS - 1) / C::ROWS;
 
@@ -189,15 +199,17 @@ cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArg
                                   static_cast<uint64_t>(p->B)};
         const uint64_t strides[2] = {row, row * p->H_Q};
         const uint32_t box[3] = {64, static_cast<uint32_t>(args.q_rows), 1};
-        *encode_ok = encode_bf16(&tmQ, buf.q, 3, dims, strides, box);
+        *encode_ok = encode_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, buf.q, 3, dims, strides, box);
     }
-    const uint32_t box4[4] = {64, 1, static_cast<uint32_t>(kTile), 1};
+    // K/V boxes: 64 tokens x 64 bf16 (128 bytes), or 64 tokens x 128 E4M3 bytes.
+    const uint32_t box4[4] = {KV8 ? static_cast<uint32_t>(D) : 64u, 1, static_cast<uint32_t>(kTile), 1};
+    const uint64_t kv_row = KV8 ? static_cast<uint64_t>(D) : row;
     if (*encode_ok) {
         uint64_t dims[4], strides[3];
         dims[0] = D;
         dims[1] = p->H_KV;
-        strides[0] = row;
-        strides[1] = row * p->H_KV;
+        strides[0] = kv_row;
+        strides[1] = kv_row * p->H_KV;
         if (PAGED) {
             dims[2] = kTile;
             dims[3] = p->num_blocks;
@@ -206,12 +218,13 @@ cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArg
             dims[3] = p->B;
         }
         strides[2] = strides[1] * dims[2];
-        *encode_ok = encode_bf16(&tmK, buf.k, 4, dims, strides, box4) &&
-                     encode_bf16(&tmV, buf.v, 4, dims, strides, box4);
+        const CUtensorMapDataType kv_type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        *encode_ok = encode_map(&tmK, kv_type, buf.k, 4, dims, strides, box4) &&
+                     encode_map(&tmV, kv_type, buf.v, 4, dims, strides, box4);
     }
     if (!*encode_ok) return cudaErrorInvalidValue;
-    auto kernel = split_mma_kernel<D, NT, HG, PAGED, OUTB>;
-    const int smem = C::smem_bytes(stages);
+    auto kernel = split_mma_kernel<D, NT, HG, PAGED, OUTB, KV8>;
+    const int smem = C::smem_bytes(stages, stages8);
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
     return launch_chained(kernel, grid, C::THREADS, smem, stream, tmQ, tmK, tmV, args);
@@ -228,19 +241,26 @@ cudaError_t launch_mma_groups(const gqa_decode_params* p, const Buffers& buf,
     return launch_mma<D, 4, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
 }
 
-template <typename T, int D, bool PAGED, bool OUTB>
+template <typename TQ, typename TKV, int D, bool PAGED, bool OUTB>
 cudaError_t launch_simt(const Buffers& buf, const KernelArgs& args, int grid, cudaStream_t stream) {
-    return launch_chained(split_simt_kernel<T, D, PAGED, OUTB>, grid, 32 * kSimtWarps, 0, stream,
-                          static_cast<const T*>(buf.q), static_cast<const T*>(buf.k),
-                          static_cast<const T*>(buf.v), args);
+    return launch_chained(split_simt_kernel<TQ, TKV, D, PAGED, OUTB>, grid, 32 * kSimtWarps, 0, stream,
+                          static_cast<const TQ*>(buf.q), static_cast<const TKV*>(buf.k),
+                          static_cast<const TKV*>(buf.v), args);
 }
 
 template <int D, bool PAGED, bool OUTB>
 cudaError_t launch_split(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
                          const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
+    if (buf.kv8) {
+        if constexpr (D == 128) {
+            if (p->H_Q / p->H_KV <= 8)
+                return launch_mma<128, 1, 1, PAGED, OUTB, true>(p, buf, args, dev, grid, stream, encode_ok);
+        }
+        return launch_simt<__nv_bfloat16, __nv_fp8_e4m3, D, PAGED, OUTB>(buf, args, grid, stream);
+    }
     if (use_tensor_cores(p)) return launch_mma_groups<D, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
-    if (p->qkv_dtype == GQA_F32) return launch_simt<float, D, PAGED, OUTB>(buf, args, grid, stream);
-    return launch_simt<__nv_bfloat16, D, PAGED, OUTB>(buf, args, grid, stream);
+    if (p->qkv_dtype == GQA_F32) return launch_simt<float, float, D, PAGED, OUTB>(buf, args, grid, stream);
+    return launch_simt<__nv_bfloat16, __nv_bfloat16, D, PAGED, OUTB>(buf, args, grid, stream);
 }
 
 template <int D, bool OUTB>
@@ -260,7 +280,9 @@ cudaError_t launch_all(const gqa_decode_params* p, const Buffers& buf, const Ker
 
 gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const void* v,
                const int32_t* seq_lens, const int32_t* block_table, float scale, void* out,
-               void* workspace, size_t workspace_bytes, void* stream_ptr, void* ev0, void* ev1) {
+               void* workspace, size_t workspace_bytes, void* stream_ptr, void* ev0, void* ev1,
+               const float* k_scale = nullptr, const float* v_scale = nullptr) {
+    const bool kv8 = k_scale != nullptr;
     gqa_status st = validate_params(p);
     if (st != GQA_OK) return st;
     if (p->B == 0) return GQA_OK;
@@ -273,7 +295,9 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
 
     DeviceInfo dev;
     if ((st = device_info(&dev)) != GQA_OK) return st;
-    const int grid = grid_for(p, dev);
+    // 8-bit caches always use one CTA per SM, so gqa_decode_workspace_size's
+    // answer for the same parameters is always enough.
+    const int grid = kv8 ? dev.sms : grid_for(p, dev);
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < workspace_for(p, grid))
         return GQA_ERR_WORKSPACE;
 
@@ -298,8 +322,10 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
     args.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes);
     args.ws_lse = reinterpret_cast<float*>(
         ws + kHeaderBytes + round_up(slots * R * p->head_dim * sizeof(float), 256));
+    args.k_scale = k_scale;
+    args.v_scale = v_scale;
 
-    const Buffers buf{q, k, v};
+    const Buffers buf{q, k, v, kv8};
     cudaStream_t stream = static_cast<cudaStream_t>(stream_ptr);
     cudaEvent_t e0 = static_cast<cudaEvent_t>(ev0), e1 = static_cast<cudaEvent_t>(ev1);
     bool encode_ok = true;
@@ -381,6 +407,19 @@ gqa_status gqa_decode(const gqa_decode_params* params, const void* q, const void
                       void* stream) {
     return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, workspace,
                workspace_bytes, stream, nullptr, nullptr);
+}
+
+gqa_status gqa_decode_fp8kv(const gqa_decode_params* params, const void* q, const void* k_cache,
+                            const void* v_cache, const float* k_scale, const float* v_scale,
+                            const int32_t* seq_lens, const int32_t* block_table, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+    gqa_status st = validate_params(params);
+    if (st != GQA_OK) return st;
+    if (params->B == 0) return GQA_OK;
+    if (params->qkv_dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;  // q is bf16 on this path
+    if (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)) return GQA_ERR_INVALID;
+    return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, workspace,
+               workspace_bytes, stream, nullptr, nullptr, k_scale, v_scale);
 }
 
 gqa_status gqa_decode_timed(const gqa_decode_params* params, const void* q, const void* k_cache,

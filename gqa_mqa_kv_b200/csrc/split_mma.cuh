@@ -38,20 +38,24 @@ namespace gqa {
 // Largest base-2 growth of the running maximum absorbed without rescaling.
 constexpr float kLazyRescale = 8.f;
 
-template <int D, int NT, int HG>
+template <int D, int NT, int HG, bool KV8 = false>
 struct MmaCfg {
     static_assert(D == 64 || D == 128, "head_dim must be 64 or 128");
+    static_assert(!KV8 || (D == 128 && NT == 1 && HG == 1), "8-bit caches: head_dim 128, <= 8 heads");
     static_assert(NT == 1 || NT == 2 || NT == 4, "8, 16 or 32 query heads per warp");
     static_assert(HG == 1 || HG == 2, "head groups: 1 or 2");
     static constexpr int ROWS = 8 * NT;                 // query heads per warp
     static constexpr int NTG = (NT == 4 && HG == 2) ? 2 : 4;  // token groups
     static constexpr bool Q_IN_REGS = NT <= 2 && NTG * HG == 4;  // else Q is re-read from smem
-    static constexpr int TS = NT == 1 ? 2 : 1;          // tile sets taking alternate tiles
+    static constexpr int TS = (NT == 1 && !KV8) ? 2 : 1;  // tile sets taking alternate tiles
     static constexpr int TPW = kTile / NTG;             // tokens per warp per tile
     static constexpr int MGN = NTG * TS;                // partial softmax states per head group
     static constexpr int NC = NTG * HG * TS;            // consumer warps
     static constexpr int TILE_WARPS = NTG * HG;         // consumer warps reading one tile
-    static constexpr int THREADS = 32 * (NC + 1);
+    static constexpr int NV = KV8 ? 4 : 0;              // warps decoding 8-bit tiles to f16
+    static constexpr int PRODUCER = NC + NV;            // index of the TMA warp
+    static constexpr int THREADS = 32 * (NC + NV + 1);
+    static constexpr int STAGE8_BYTES = KV8 ? 2 * kTile * D : 0;  // one 8-bit K tile + V tile
     static constexpr int PANELS = D / 64;               // 128-byte-wide column panels
     static constexpr int PANEL_BYTES = kTile * 128;     // 64 tokens x 64 bf16
     static constexpr int STAGE_BYTES = 2 * PANELS * PANEL_BYTES;
@@ -61,15 +65,19 @@ struct MmaCfg {
     static constexpr int MERGE_O_FLOATS = (MGN - 1) * HG * ROWS * OROW;
     static constexpr int MERGE_ML_FLOATS = (MGN - 1) * HG * ROWS * 2;
     static constexpr int MAX_STAGES = 8;
-    static constexpr int CTRL_BYTES = 256;
+    static constexpr int CTRL_BYTES = 512;
     static constexpr int FIXED_BYTES =
         2 * QSLOT_BYTES + 4 * (MERGE_O_FLOATS + MERGE_ML_FLOATS) + CTRL_BYTES;
-    static constexpr int smem_bytes(int stages) { return 1024 + stages * STAGE_BYTES + FIXED_BYTES; }
+    static constexpr int smem_bytes(int stages, int stages8) {
+        return 1024 + stages * STAGE_BYTES + stages8 * STAGE8_BYTES + FIXED_BYTES;
+    }
 };
 
 struct __align__(16) MmaControl {
     uint64_t full[MmaCfg<128, 1, 1>::MAX_STAGES];
     uint64_t empty[MmaCfg<128, 1, 1>::MAX_STAGES];
+    uint64_t full8[MmaCfg<128, 1, 1>::MAX_STAGES];   // 8-bit staging ring (KV8 only)
+    uint64_t empty8[MmaCfg<128, 1, 1>::MAX_STAGES];
     uint64_t qfull[2];
     uint64_t qempty[2];
     uint64_t merge_full;
@@ -77,22 +85,29 @@ struct __align__(16) MmaControl {
     Plan plan;
     int abort;
 };
-static_assert(sizeof(MmaControl) <= MmaCfg<128, 1, 1>::CTRL_BYTES, "control block overflows its slot");
+static_assert(sizeof(MmaControl) <= MmaCfg<128, 1, 1, false>::CTRL_BYTES, "control block overflows its slot");
 
-template <int D, int NT, int HG, bool PAGED, bool OUT_BF16>
-__global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
+// KV8: the cache holds OCP E4M3 bytes with per-KV-head scales; converter warps
+// decode each staged 8-bit tile to f16 (exactly) and the consumers run the
+// same contraction on f16 mma.sync, with k_scale folded into the score scale
+// and v_scale into the output.
+template <int D, int NT, int HG, bool PAGED, bool OUT_BF16, bool KV8 = false>
+__global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     split_mma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const KernelArgs a) {
-    using C = MmaCfg<D, NT, HG>;
+    using C = MmaCfg<D, NT, HG, KV8>;
     constexpr int KS = D / 16;  // k-steps over the head dimension; also 16-row blocks of d
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = smem_raw + (base - raw);
     const int NS = a.n_stages;
+    const int NS8 = KV8 ? a.n_stages8 : 0;
     const uint32_t stages = base;
-    const uint32_t qring = base + NS * C::STAGE_BYTES;
-    float* merge_o = reinterpret_cast<float*>(base_ptr + NS * C::STAGE_BYTES + 2 * C::QSLOT_BYTES);
+    const uint32_t stages8 = base + NS * C::STAGE_BYTES;
+    const int ring_bytes = NS * C::STAGE_BYTES + NS8 * C::STAGE8_BYTES;
+    const uint32_t qring = base + ring_bytes;
+    float* merge_o = reinterpret_cast<float*>(base_ptr + ring_bytes + 2 * C::QSLOT_BYTES);
     float* merge_ml = merge_o + C::MERGE_O_FLOATS;
     MmaControl* ctrl = reinterpret_cast<MmaControl*>(merge_ml + C::MERGE_ML_FLOATS);
     volatile int* abort_flag = &ctrl->abort;
@@ -100,15 +115,19 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    if (warp == C::NC && lane == 0) {
+    if (warp == C::PRODUCER && lane == 0) {
         prefetch_tensormap(&tmQ);
         prefetch_tensormap(&tmK);
         prefetch_tensormap(&tmV);
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(smem_addr(&ctrl->full[s]), 1);
+            mbar_init(smem_addr(&ctrl->full[s]), KV8 ? C::NV : 1);
             mbar_init(smem_addr(&ctrl->empty[s]), C::TILE_WARPS);
+        }
+        for (int s = 0; s < NS8; ++s) {
+            mbar_init(smem_addr(&ctrl->full8[s]), 1);
+            mbar_init(smem_addr(&ctrl->empty8[s]), C::NV);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->qfull[s]), 1);
@@ -120,7 +139,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     }
     // Query rows a TMA box does not cover (R < ROWS) must read as zeros.
     for (int i = threadIdx.x; i < 2 * C::QSLOT_BYTES / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(base_ptr + NS * C::STAGE_BYTES)[i] = make_uint4(0, 0, 0, 0);
+        reinterpret_cast<uint4*>(base_ptr + ring_bytes)[i] = make_uint4(0, 0, 0, 0);
 
     grid_dependency_wait();
     grid_launch_dependents();
@@ -134,7 +153,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     if (lo >= hi) return;
     Walk w{ctrl->plan.b, ctrl->plan.kv, ctrl->plan.tile, ctrl->plan.n_b, ctrl->plan.L};
 
-    if (warp == C::NC) {
+    if (warp == C::PRODUCER) {
         // ------------------------------------------------------------ producer
         const uint64_t pol_kv = policy_evict_first();
         const uint64_t pol_q = policy_evict_last();
@@ -144,6 +163,10 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
         int64_t issued = 0, q_issued = 0;
         int page_word = 0, page_base = -1;
         bool ok = true;
+        // Tiles go to the f16/bf16 stage ring, or for 8-bit caches to the staging ring.
+        const int RN = KV8 ? NS8 : NS;
+        uint64_t* rfull = KV8 ? ctrl->full8 : ctrl->full;
+        uint64_t* rempty = KV8 ? ctrl->empty8 : ctrl->empty;
         for (int64_t gi = lo; gi < hi; ++gi) {
             const bool seg_first = (gi == lo) || (w.tile == 0);
             if (seg_first) {
@@ -177,33 +200,88 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                 c2 = w.tile * kTile;
                 c3 = w.b;
             }
-            if (!mbar_wait_warp(smem_addr(&ctrl->empty[st]), ph ^ 1u, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(smem_addr(&rempty[st]), ph ^ 1u, abort_flag)) { ok = false; break; }
             if (lane == 0) {
-                const uint32_t bar = smem_addr(&ctrl->full[st]);
-                const uint32_t kb = stages + st * C::STAGE_BYTES;
-                const uint32_t vb = kb + C::PANELS * C::PANEL_BYTES;
-                mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-                for (int p = 0; p < C::PANELS; ++p) {
-                    tma_load_4d(kb + p * C::PANEL_BYTES, &tmK, bar, 64 * p, w.kv, c2, c3, pol_kv);
-                    tma_load_4d(vb + p * C::PANEL_BYTES, &tmV, bar, 64 * p, w.kv, c2, c3, pol_kv);
+                const uint32_t bar = smem_addr(&rfull[st]);
+                if constexpr (KV8) {
+                    const uint32_t kb = stages8 + st * C::STAGE8_BYTES;  // 64 rows x D bytes each
+                    mbar_arrive_expect_tx(bar, C::STAGE8_BYTES);
+                    tma_load_4d(kb, &tmK, bar, 0, w.kv, c2, c3, pol_kv);
+                    tma_load_4d(kb + kTile * D, &tmV, bar, 0, w.kv, c2, c3, pol_kv);
+                } else {
+                    const uint32_t kb = stages + st * C::STAGE_BYTES;
+                    const uint32_t vb = kb + C::PANELS * C::PANEL_BYTES;
+                    mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+                    for (int p = 0; p < C::PANELS; ++p) {
+                        tma_load_4d(kb + p * C::PANEL_BYTES, &tmK, bar, 64 * p, w.kv, c2, c3, pol_kv);
+                        tma_load_4d(vb + p * C::PANEL_BYTES, &tmV, bar, 64 * p, w.kv, c2, c3, pol_kv);
+                    }
                 }
             }
             ++issued;
-            if (++st == NS) { st = 0; ph ^= 1u; }
+            if (++st == RN) { st = 0; ph ^= 1u; }
             if (gi + 1 < hi) w.advance(a);
         }
         if (!ok) {
             *abort_flag = 1;
             if (lane == 0) atomicOr(a.status, kFlagTimeout);
             // Let copies already in flight land before the CTA's shared memory goes away.
-            const int64_t first = issued > NS ? issued - NS : 0;
+            const int64_t first = issued > RN ? issued - RN : 0;
             for (int64_t i = first; i < issued; ++i)
-                mbar_wait(smem_addr(&ctrl->full[i % NS]), static_cast<uint32_t>((i / NS) & 1), nullptr);
+                mbar_wait(smem_addr(&rfull[i % RN]), static_cast<uint32_t>((i / RN) & 1), nullptr);
             const int64_t qfirst = q_issued > 2 ? q_issued - 2 : 0;
             for (int64_t i = qfirst; i < q_issued; ++i)
                 mbar_wait(smem_addr(&ctrl->qfull[i % 2]), static_cast<uint32_t>((i / 2) & 1), nullptr);
         }
         return;
+    }
+
+    if constexpr (KV8) {
+        if (warp >= C::NC) {
+            // -------------------------------------------------------- converters
+            // Decode each staged 8-bit K and V tile (64 rows x 128 bytes, 128-byte
+            // swizzle) into the f16 stage layout the consumers read (two 64-column
+            // panels per operand, same swizzle).  E4M3 -> f16 is exact.
+            const int vt = threadIdx.x - 32 * C::NC;
+            constexpr int CHUNKS = 2 * kTile * (D / 16);  // 16-byte 8-bit chunks per stage
+            int st = 0, st8 = 0;
+            uint32_t ph = 0, ph8 = 0;
+            for (int64_t gi = lo; gi < hi; ++gi) {
+                const bool ok = mbar_wait_warp(smem_addr(&ctrl->full8[st8]), ph8, abort_flag) &&
+                                mbar_wait_warp(smem_addr(&ctrl->empty[st]), ph ^ 1u, abort_flag);
+                if (!ok) {
+                    *abort_flag = 1;
+                    if (lane == 0) atomicOr(a.status, kFlagTimeout);
+                    break;
+                }
+                const uint32_t src = stages8 + st8 * C::STAGE8_BYTES;
+                const uint32_t dst = stages + st * C::STAGE_BYTES;
+#pragma unroll 2
+                for (int i = 0; i < CHUNKS / (32 * C::NV); ++i) {
+                    const int j = vt + 32 * C::NV * i;
+                    const int op = j / (kTile * (D / 16));  // 0: K, 1: V
+                    const int row = (j / (D / 16)) % kTile;
+                    const int c = j % (D / 16);  // values d = 16c .. 16c+15
+                    const uint4 raw = ld_shared_v4(src + op * kTile * D + row * 128 + ((c ^ (row & 7)) << 4));
+                    const int ch0 = (c & 3) << 1;
+                    const uint32_t pb = dst + op * C::PANELS * C::PANEL_BYTES + (c >> 2) * C::PANEL_BYTES + row * 128;
+                    st_shared_v4(pb + ((ch0 ^ (row & 7)) << 4), e4m3x2_to_f16x2(raw.x & 0xffffu),
+                                 e4m3x2_to_f16x2(raw.x >> 16), e4m3x2_to_f16x2(raw.y & 0xffffu),
+                                 e4m3x2_to_f16x2(raw.y >> 16));
+                    st_shared_v4(pb + (((ch0 + 1) ^ (row & 7)) << 4), e4m3x2_to_f16x2(raw.z & 0xffffu),
+                                 e4m3x2_to_f16x2(raw.z >> 16), e4m3x2_to_f16x2(raw.w & 0xffffu),
+                                 e4m3x2_to_f16x2(raw.w >> 16));
+                }
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive(smem_addr(&ctrl->empty8[st8]));
+                    mbar_arrive(smem_addr(&ctrl->full[st]));
+                }
+                if (++st8 == NS8) { st8 = 0; ph8 ^= 1u; }
+                if (++st == NS) { st = 0; ph ^= 1u; }
+            }
+            return;
+        }
     }
 
     // ---------------------------------------------------------------- consumers
@@ -226,6 +304,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
     int seg_q = 0;                                  // Q-ring slot of the current segment
     float o[KS][NT][4];      // O^T accumulators, per 16-row block of d and 8-head tile
     float m[NT][2], l[NT][2];
+    float seg_sl2 = a.sl2, seg_vs = 1.f;  // score scale (x k_scale) and value scale of the segment's KV head
 
     auto fail = [&]() {
         *abort_flag = 1;
@@ -265,6 +344,19 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
             if constexpr (C::Q_IN_REGS) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[qs]));
+                if constexpr (KV8) {  // the 8-bit path multiplies in f16
+#pragma unroll
+                    for (int ks = 0; ks < KS; ++ks)
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            qb[ks][nt][0] = bf16x2_to_f16x2(qb[ks][nt][0]);
+                            qb[ks][nt][1] = bf16x2_to_f16x2(qb[ks][nt][1]);
+                        }
+                }
+            }
+            if constexpr (KV8) {
+                seg_sl2 = a.sl2 * __ldg(a.k_scale + w.kv);
+                seg_vs = __ldg(a.v_scale + w.kv);
             }
             if (++qs == 2) { qs = 0; qph ^= 1u; }
 #pragma unroll
@@ -314,7 +406,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                     for (int h = 0; h < 2; ++h)
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
-                            mma_bf16_16816(sa[(ks + h) % NSET][nt], ka[h], qb[ks + h][nt][0], qb[ks + h][nt][1]);
+                            mma_16816<KV8>(sa[(ks + h) % NSET][nt], ka[h], qb[ks + h][nt][0], qb[ks + h][nt][1]);
                 } else {
                     const uint32_t qbase = qring + seg_q * C::QSLOT_BYTES + hg * C::PANELS * C::QPANEL_BYTES;
 #pragma unroll
@@ -330,7 +422,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                         }
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt)
-                            mma_bf16_16816(sa[kk % NSET][nt], ka[h], qf[nt][0], qf[nt][1]);
+                            mma_16816<KV8>(sa[kk % NSET][nt], ka[h], qf[nt][0], qf[nt][1]);
                     }
                 }
             }
@@ -342,7 +434,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                     float x = sa[0][nt][i];
 #pragma unroll
                     for (int q = 1; q < NSET; ++q) x += sa[q][nt][i];
-                    s[nt][i] = x * a.sl2;
+                    s[nt][i] = x * seg_sl2;
                 }
             uint32_t vmask_a = 0xffffffffu, vmask_b = 0xffffffffu;
             if (mask) {
@@ -399,8 +491,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
                 uint32_t h0, l0, h1, l1;
-                split_bf16x2(p[nt][0], p[nt][1], h0, l0);  // token g:     heads 2t, 2t+1
-                split_bf16x2(p[nt][2], p[nt][3], h1, l1);  // token g + 8: heads 2t, 2t+1
+                split_x2<KV8>(p[nt][0], p[nt][1], h0, l0);  // token g:     heads 2t, 2t+1
+                split_x2<KV8>(p[nt][2], p[nt][3], h1, l1);  // token g + 8: heads 2t, 2t+1
                 pbh[nt][0] = movmatrix_trans(h0);
                 pbh[nt][1] = movmatrix_trans(h1);
                 pbl[nt][0] = movmatrix_trans(l0);
@@ -430,11 +522,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
 #pragma unroll
                 for (int h = 0; h < MG; ++h)
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[m0 + h][nt], va[h], pbh[nt][0], pbh[nt][1]);
+                    for (int nt = 0; nt < NT; ++nt) mma_16816<KV8>(o[m0 + h][nt], va[h], pbh[nt][0], pbh[nt][1]);
 #pragma unroll
                 for (int h = 0; h < MG; ++h)
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16_16816(o[m0 + h][nt], va[h], pbl[nt][0], pbl[nt][1]);
+                    for (int nt = 0; nt < NT; ++nt) mma_16816<KV8>(o[m0 + h][nt], va[h], pbl[nt][0], pbl[nt][1]);
             }
         }
         __syncwarp();
@@ -525,7 +617,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG>::THREADS, 1)
                     for (int j = 0; j < 2; ++j) {
                         const int r = hg * C::ROWS + 8 * nt + 2 * t + j;
                         if (r >= a.R) continue;
-                        const float inv = 1.f / Lsum[nt][j];
+                        const float inv = seg_vs / Lsum[nt][j];
                         if (whole) {
                             const int64_t row = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + r) * D;
 #pragma unroll

@@ -10,6 +10,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include "ptx.cuh"
 #include "schedule.cuh"
@@ -22,13 +23,17 @@ template <>
 __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <>
+__device__ __forceinline__ float to_f32<__nv_fp8_e4m3>(__nv_fp8_e4m3 x) { return static_cast<float>(x); }
 
 constexpr int kSimtWarps = 4;
 constexpr int kSimtHeads = 8;
 
-template <typename T, int D, bool PAGED, bool OUT_BF16>
+// TQ: element type of q; TKV: element type of the cache (fp32, bf16 or E4M3
+// bytes, the latter multiplied by per-KV-head k_scale / v_scale).
+template <typename TQ, typename TKV, int D, bool PAGED, bool OUT_BF16>
 __global__ void __launch_bounds__(32 * kSimtWarps)
-    split_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+    split_simt_kernel(const TQ* __restrict__ q, const TKV* __restrict__ k, const TKV* __restrict__ v,
                       const KernelArgs a) {
     constexpr int DPL = D / 32;
     constexpr int HC = kSimtHeads;
@@ -57,6 +62,8 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
         const int64_t slot = first ? 2 * static_cast<int64_t>(blockIdx.x) : 2 * static_cast<int64_t>(blockIdx.x) + 1;
         const int t_begin = w.tile * kTile;
         const int t_end = min((w.tile + seg_tiles) * kTile, w.L);
+        const float sl2 = a.sl2 * (a.k_scale ? __ldg(a.k_scale + w.kv) : 1.f);
+        const float vsc = a.v_scale ? __ldg(a.v_scale + w.kv) : 1.f;
 
         for (int hc = 0; hc < a.R; hc += HC) {
             const int nh = min(HC, a.R - hc);
@@ -96,7 +103,7 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
                     for (int i = 0; i < DPL; ++i) s = fmaf(qr[j][i], kr[i], s);
 #pragma unroll
                     for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-                    s *= a.sl2;
+                    s *= sl2;
                     const float mn = fmaxf(m[j], s);
                     const float al = fast_exp2(m[j] - mn);
                     const float p = fast_exp2(s - mn);
@@ -130,6 +137,7 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
                     O += sm_o[ww][j][d] * e;
                 }
                 const int r = hc + j;
+                O *= vsc;
                 if (whole) {
                     const int64_t oi = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + r) * D + d;
                     if constexpr (OUT_BF16)

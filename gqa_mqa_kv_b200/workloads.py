@@ -53,6 +53,7 @@ class Workload:
     page_size: int = 0
     seed: int = 0
     scale: float | None = None  # None -> 1/sqrt(D)
+    kv8: bool = False  # cache stored as OCP E4M3 bytes with per-KV-head scales
 
     @property
     def R(self) -> int:
@@ -86,6 +87,8 @@ WORKLOADS: dict[str, Workload] = {
         _wl("sweep_hkv1", 32, 32, 1, 128, 8192, 3),
         _wl("llama2_70b_ragged", 32, 64, 8, 128, 32768, 4, ragged=True),
         _wl("paged_long", 8, 64, 8, 128, 131072, 5, page_size=PAGE_SIZE),
+        _wl("llama2_70b_ragged_fp8", 32, 64, 8, 128, 32768, 4, ragged=True, kv8=True),
+        _wl("paged_long_fp8", 8, 64, 8, 128, 131072, 5, page_size=PAGE_SIZE, kv8=True),
     ]
 }
 
@@ -133,6 +136,18 @@ def block_table_for(w: Workload) -> torch.Tensor:
     return torch.from_numpy(perm).view(w.B, w.max_blocks_per_seq)
 
 
+def kv_scales(w: Workload) -> tuple[torch.Tensor, torch.Tensor]:
+    """Per-KV-head float32 factors of an 8-bit cache (distinct per head)."""
+    g = torch.arange(w.H_KV, dtype=torch.float32)
+    return (5.0 + 0.5 * g) / 448.0, (5.5 + 0.25 * g) / 448.0
+
+
+def _quantize_e4m3(x: torch.Tensor, scale: torch.Tensor) -> torch.Tensor:
+    """E4M3 bytes of x / scale[head] (heads on dim -2), saturated at +-448."""
+    y = (x.float() / scale[:, None]).clamp(-448.0, 448.0)
+    return y.to(torch.float8_e4m3fn)
+
+
 def make_inputs(w: Workload, pad_value: float = 0.0, seq_lens: torch.Tensor | None = None):
     """Generate one decode step's inputs on the host.
 
@@ -157,6 +172,21 @@ def make_inputs(w: Workload, pad_value: float = 0.0, seq_lens: torch.Tensor | No
             _fill_normal(k[b, :L], (w.seed, _S_K, b))
             _fill_normal(v[b, :L], (w.seed, _S_V, b))
     out = {"q": q, "k": k, "v": v, "seq_lens": lens}
+    if w.kv8:
+        # The draws above are in bf16; quantise them per KV head to E4M3 bytes.
+        ks, vs = kv_scales(w)
+        k8 = torch.zeros(k.shape, dtype=torch.uint8)
+        v8 = torch.zeros(v.shape, dtype=torch.uint8)
+        if pad_value != 0.0:
+            k8.fill_(0x7F)  # E4M3 NaN
+            v8.fill_(0x7F)
+        for b in range(w.B):
+            L = int(lens[b])
+            if L > 0:
+                k8[b, :L] = _quantize_e4m3(k[b, :L], ks).view(torch.uint8)
+                v8[b, :L] = _quantize_e4m3(v[b, :L], vs).view(torch.uint8)
+        out.update(k=k8.view(torch.float8_e4m3fn), v=v8.view(torch.float8_e4m3fn), k_scale=ks, v_scale=vs)
+        k, v = out["k"], out["v"]
     if w.page_size:
         table = block_table_for(w)
         out["block_table"] = table
@@ -175,13 +205,16 @@ def to_pages(x: torch.Tensor, table: torch.Tensor, page_size: int) -> torch.Tens
     nb = S // page_size
     assert nb * page_size == S and table.shape == (B, nb)
     num_blocks = int(table.max()) + 1 if table.numel() else 0
-    pages = torch.zeros(num_blocks, page_size, H, D, dtype=x.dtype)
-    pages[table.reshape(-1).long()] = x.reshape(B * nb, page_size, H, D)
-    return pages
+    byte_view = x.dtype == torch.float8_e4m3fn
+    src = x.view(torch.uint8) if byte_view else x
+    pages = torch.zeros(num_blocks, page_size, H, D, dtype=src.dtype)
+    pages[table.reshape(-1).long()] = src.reshape(B * nb, page_size, H, D)
+    return pages.view(torch.float8_e4m3fn) if byte_view else pages
 
 
 def algorithmic_bytes(w: Workload, seq_lens: torch.Tensor, out_bytes: int = 4) -> int:
     """Bytes the step must move at minimum: K and V rows actually cached, plus Q and O."""
     e = 2 if w.dtype == "bf16" else 4
-    kv = int(seq_lens.to(torch.int64).sum()) * w.H_KV * w.D * e * 2
+    e_kv = 1 if w.kv8 else e
+    kv = int(seq_lens.to(torch.int64).sum()) * w.H_KV * w.D * e_kv * 2
     return kv + w.B * w.H_Q * w.D * e + w.B * w.H_Q * w.D * out_bytes

@@ -143,6 +143,25 @@ gqa_status gqa_decode(const gqa_decode_params* params, const void* q, const void
                       void* stream);
 
 /*
+ * gqa_decode over an 8-bit cache: k_cache and v_cache hold OCP E4M3 bytes
+ * (sign, 4 exponent bits with bias 7, 3 mantissa bits; 0x7F/0xFF are NaN; max
+ * 448) and the cached keys and values are
+ *     K[b,t,g,:] = e4m3(k_cache[b,t,g,:]) * k_scale[g]
+ *     V[b,t,g,:] = e4m3(v_cache[b,t,g,:]) * v_scale[g]
+ * with per-KV-head fp32 factors k_scale[H_KV], v_scale[H_KV] (device).  This is
+ * the bytes-per-element term of [AIT]'s cache estimate: the same attention
+ * over a cache that moves half the bytes of bf16.  q stays bf16
+ * (params->qkv_dtype must be GQA_BF16, |q| below 65504); layouts, seq_lens,
+ * block_table, scale, out and the workspace (gqa_decode_workspace_size with
+ * the same params suffices) are as for gqa_decode.  head_dim 128 with up to 8
+ * query heads per KV head runs on tensor cores; other shapes on CUDA cores.
+ */
+gqa_status gqa_decode_fp8kv(const gqa_decode_params* params, const void* q, const void* k_cache,
+                            const void* v_cache, const float* k_scale, const float* v_scale,
+                            const int32_t* seq_lens, const int32_t* block_table, float scale, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * gqa_decode that also records `split_begin` just before and `split_end`
  * just after the split-KV kernel (both cudaEvent_t, either may be NULL).
  * For measuring the dominant kernel alone; the result equals gqa_decode's.

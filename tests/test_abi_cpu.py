@@ -177,3 +177,17 @@ def test_rope_append_rejects_bad_arguments_on_host(lib):
     assert call_rope(lib, p, ws=128) == GQA_ERR_WORKSPACE
     assert call_rope(lib, params(B=0), q=None, kn=None, vn=None, pos=None, qo=None, kc=None,
                      vc=None) == GQA_OK
+
+
+def test_fp8kv_rejects_bad_arguments_on_host(lib):
+    vp = ctypes.c_void_p
+
+    def call(p, ks=64, vs=64, q=16):
+        return lib.gqa_decode_fp8kv(ctypes.byref(p), vp(q), vp(16), vp(16), vp(ks), vp(vs), vp(16), vp(None),
+                                    ctypes.c_float(0.1), vp(16), vp(256), ctypes.c_size_t(1 << 20), vp(None))
+
+    assert call(params(), ks=None) == GQA_ERR_INVALID
+    assert call(params(), vs=None) == GQA_ERR_INVALID
+    assert call(params(), ks=66) == GQA_ERR_INVALID          # misaligned float array
+    assert call(params(qkv_dtype=1)) == GQA_ERR_UNSUPPORTED  # q must be bf16
+    assert call(params(H_Q=6, H_KV=4)) == GQA_ERR_INVALID
