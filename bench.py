@@ -199,8 +199,12 @@ def cpu_oracle_sample(w, inp, seconds: float):
     # calibrate on all heads of the first non-empty sequence
     b0 = int(torch.nonzero(lens > 0)[0])
     t0 = time.perf_counter()
-    oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale,
-                      pairs=[(b0, h) for h in range(H_Q)], n_threads=0)
+    run = ((lambda pairs: oracle.gqa_decode_scaled(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale,
+                                                    inp["k_scale"], inp["v_scale"], pairs=pairs))
+           if w.kv8 else
+           (lambda pairs: oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=pairs,
+                                            n_threads=0)))
+    run([(b0, h) for h in range(H_Q)])
     per_token = max((time.perf_counter() - t0) / max(int(lens[b0]), 1), 1e-12)  # all heads, all threads
     est_full = per_token * int(lens.sum())
     if est_full <= seconds:
@@ -215,11 +219,12 @@ def cpu_oracle_sample(w, inp, seconds: float):
     times = []
     for _ in range(reps):
         t0 = time.perf_counter()
-        oracle.gqa_decode(inp["q"], inp["k"], inp["v"], lens, w.softmax_scale, pairs=pairs, n_threads=0)
+        run(pairs)
         times.append(time.perf_counter() - t0)
     dt = statistics.median(times)
     e = 2 if w.dtype == "bf16" else 4
-    sample_bytes = (int(lens[:nb].to(torch.int64).sum()) * w.H_KV * w.D * e * 2
+    e_kv = 1 if w.kv8 else e
+    sample_bytes = (int(lens[:nb].to(torch.int64).sum()) * w.H_KV * w.D * e_kv * 2
                     + nb * H_Q * w.D * e + nb * H_Q * w.D * 4)
     what = "the whole step" if nb == w.B else f"sequences 0..{nb - 1} of {w.B}"
     return {
@@ -261,11 +266,17 @@ def run_reference(args):
 
 # ---------------------------------------------------------------- GPU arm
 
+def cache_capacity_bytes(w):
+    """K plus V bytes at the workload's maximum length (the L2 comparison)."""
+    e_kv = 1 if w.kv8 else (2 if w.dtype == "bf16" else 4)
+    return w.seq_len * w.B * w.H_KV * w.D * e_kv * 2
+
+
 def workload_config(w, n):
     return {"workload": w.name, "B": w.B, "H_Q": w.H_Q, "H_KV": w.H_KV, "head_dim": w.D,
             "seq_len": w.seq_len, "ragged": w.ragged, "page_size": w.page_size,
-            "kv_dtype": w.dtype, "global_batch": w.B * n,
-            "l2": "inputs larger than L2 (no flush)" if w.seq_len * w.B * w.H_KV * w.D * 4 > 2 * 126e6
+            "kv_dtype": "e4m3 (per-KV-head scales)" if w.kv8 else w.dtype, "global_batch": w.B * n,
+            "l2": "inputs larger than L2 (no flush)" if cache_capacity_bytes(w) > 2 * 126e6
                   else "L2 flushed before every step",
             "parallelism": f"dp{n} (independent batch per GPU, no collective)"}
 
@@ -292,10 +303,14 @@ def run_ours(args):
     lens = lens_host.to(dev)
     table = inp["block_table"].to(dev) if paged else None
     out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    ks = inp["k_scale"].to(dev) if w.kv8 else None
+    vs = inp["v_scale"].to(dev) if w.kv8 else None
     params = gq.make_params(q, k, lens, table)
+    if w.kv8:
+        params.qkv_dtype = gq.GQA_BF16
     ws = torch.zeros(gq.workspace_bytes(params), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    big = w.seq_len * w.B * w.H_KV * w.D * 4 > 2 * 126e6
+    big = cache_capacity_bytes(w) > 2 * 126e6
     flush = None if big else torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
     appending = args.path == "append_decode"
     if appending:
@@ -317,12 +332,27 @@ def run_ours(args):
         if events is not None:
             events[1].record(stream)
 
+    def decode_call(events=None):
+        if w.kv8:  # 8-bit cache: events bracket the whole call (split + combine)
+            if events is not None:
+                events[0].record(stream)
+            gq.gqa_decode_fp8kv(q, k, v, ks, vs, lens, table, scale=w.softmax_scale, out=out,
+                                workspace=ws, stream=stream)
+            if events is not None:
+                events[1].record(stream)
+        elif events is not None:
+            gq.gqa_decode_timed(events, q, k, v, lens, table, scale=w.softmax_scale, out=out,
+                                workspace=ws, stream=stream)
+        else:
+            gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws,
+                          stream=stream)
+
     def step():
         if flush is not None:
             flush.zero_()
         if appending:
             append_call()
-        gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws, stream=stream)
+        decode_call()
 
     for _ in range(max(args.warmup, 3)):
         step()
@@ -349,8 +379,7 @@ def run_ours(args):
                 step_ev[i][0].record(stream)
             if appending:
                 append_call()
-            gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws,
-                          stream=stream)
+            decode_call()
             if flush is not None:
                 step_ev[i][1].record(stream)
         ev_end.record(stream)
@@ -370,8 +399,7 @@ def run_ours(args):
                 flush.zero_()
             if appending:
                 append_call(append_ev[i])
-            gq.gqa_decode_timed(split_ev[i], q, k, v, lens, table, scale=w.softmax_scale, out=out,
-                                workspace=ws, stream=stream)
+            decode_call(split_ev[i])
         torch.cuda.synchronize(dev)
         if dist is not None:
             dist.barrier()
@@ -395,7 +423,7 @@ def run_ours(args):
     def e2e_step():
         q.copy_(q_host, non_blocking=True)
         lens.copy_(lens_pin, non_blocking=True)
-        gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws, stream=stream)
+        decode_call()
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(3):
@@ -421,7 +449,8 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "us_per_step": ms_per_step * 1e3,
         "pct_of_hbm_peak": 100.0 * (value / world) / peak, "peak_kind": peak_kind,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16 q, e4m3 KV" if w.kv8 else "bf16",
         "data": "synthetic", "config": workload_config(w, world),
         "algorithmic_bytes_per_step_per_gpu": step_bytes,
         "clocks": clocks.summary(),
@@ -433,7 +462,8 @@ def run_ours(args):
         "gpu_launches": launches_per_step * args.steps,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": traffic,
-                     "kernel": "split-KV decode kernel (combine excluded)",
+                     "kernel": ("split-KV decode call (split + combine)" if w.kv8
+                                else "split-KV decode kernel (combine excluded)"),
                      "split_kernel_us": split_ms_max * 1e3,
                      "peak_note": f"{peak_kind} HBM copy bandwidth"},
         "device_status_flags": status,

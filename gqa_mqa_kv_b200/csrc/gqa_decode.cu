@@ -176,19 +176,10 @@ cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArg
                        const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
     using C = MmaCfg<D, NT, HG, KV8>;
     const int R = p->H_Q / p->H_KV;
-    int stages, stages8 = 0;
-    if constexpr (KV8) {  // 4 decoded stages; the rest of shared memory stages 8-bit tiles
-        stages = 4;
-        stages8 = (dev.smem_optin - C::FIXED_BYTES - 1024 - stages * C::STAGE_BYTES) / C::STAGE8_BYTES;
-        if (stages8 > C::MAX_STAGES) stages8 = C::MAX_STAGES;
-        if (stages8 < 2) return cudaErrorInvalidConfiguration;
-    } else {
-        stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
-        if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
-    }
+    int stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
+    if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
     if (stages < 2) return cudaErrorInvalidConfiguration;
     args.n_stages = stages;
-    args.n_stages8 = stages8;
     args.q_rows = R < C::ROWS ? R : C::ROWS;
     args.q_groups = (R + C::ROWS - 1) / C::ROWS;
 
@@ -224,7 +215,7 @@ cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArg
     }
     if (!*encode_ok) return cudaErrorInvalidValue;
     auto kernel = split_mma_kernel<D, NT, HG, PAGED, OUTB, KV8>;
-    const int smem = C::smem_bytes(stages, stages8);
+    const int smem = C::smem_bytes(stages);
     cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), smem);
     if (e != cudaSuccess) return e;
     return launch_chained(kernel, grid, C::THREADS, smem, stream, tmQ, tmK, tmV, args);

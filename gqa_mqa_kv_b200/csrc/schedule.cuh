@@ -44,7 +44,6 @@ struct KernelArgs {
     int n_stages;    // tensor-core path: pipeline depth
     int q_rows;      // tensor-core path: query rows per TMA box, min(R, 16)
     int q_groups;    // tensor-core path: 16-row head groups holding real rows
-    int n_stages8;   // 8-bit caches: depth of the staging ring
     const float* k_scale;  // [H_KV] or null: stored keys are multiplied by k_scale[g]
     const float* v_scale;  // [H_KV] or null: stored values likewise
 };

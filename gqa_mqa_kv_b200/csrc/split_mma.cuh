@@ -47,37 +47,33 @@ struct MmaCfg {
     static constexpr int ROWS = 8 * NT;                 // query heads per warp
     static constexpr int NTG = (NT == 4 && HG == 2) ? 2 : 4;  // token groups
     static constexpr bool Q_IN_REGS = NT <= 2 && NTG * HG == 4;  // else Q is re-read from smem
-    static constexpr int TS = (NT == 1 && !KV8) ? 2 : 1;  // tile sets taking alternate tiles
+    static constexpr int TS = NT == 1 ? 2 : 1;          // tile sets taking alternate tiles
     static constexpr int TPW = kTile / NTG;             // tokens per warp per tile
     static constexpr int MGN = NTG * TS;                // partial softmax states per head group
     static constexpr int NC = NTG * HG * TS;            // consumer warps
     static constexpr int TILE_WARPS = NTG * HG;         // consumer warps reading one tile
-    static constexpr int NV = KV8 ? 4 : 0;              // warps decoding 8-bit tiles to f16
-    static constexpr int PRODUCER = NC + NV;            // index of the TMA warp
-    static constexpr int THREADS = 32 * (NC + NV + 1);
-    static constexpr int STAGE8_BYTES = KV8 ? 2 * kTile * D : 0;  // one 8-bit K tile + V tile
+    static constexpr int PRODUCER = NC;                 // index of the TMA warp
+    static constexpr int THREADS = 32 * (NC + 1);
     static constexpr int PANELS = D / 64;               // 128-byte-wide column panels
     static constexpr int PANEL_BYTES = kTile * 128;     // 64 tokens x 64 bf16
-    static constexpr int STAGE_BYTES = 2 * PANELS * PANEL_BYTES;
+    // One stage: K and V tiles of 64 tokens, bf16 in 128-byte panels, or 8-bit
+    // rows of D bytes (KV8).
+    static constexpr int STAGE_BYTES = KV8 ? 2 * kTile * D : 2 * PANELS * PANEL_BYTES;
     static constexpr int QPANEL_BYTES = ROWS * 128;     // ROWS query rows x 64 bf16
     static constexpr int QSLOT_BYTES = HG * PANELS * QPANEL_BYTES;
     static constexpr int OROW = D + 4;                  // padded merge row (floats)
     static constexpr int MERGE_O_FLOATS = (MGN - 1) * HG * ROWS * OROW;
     static constexpr int MERGE_ML_FLOATS = (MGN - 1) * HG * ROWS * 2;
-    static constexpr int MAX_STAGES = 8;
+    static constexpr int MAX_STAGES = KV8 ? 12 : 8;
     static constexpr int CTRL_BYTES = 512;
     static constexpr int FIXED_BYTES =
         2 * QSLOT_BYTES + 4 * (MERGE_O_FLOATS + MERGE_ML_FLOATS) + CTRL_BYTES;
-    static constexpr int smem_bytes(int stages, int stages8) {
-        return 1024 + stages * STAGE_BYTES + stages8 * STAGE8_BYTES + FIXED_BYTES;
-    }
+    static constexpr int smem_bytes(int stages) { return 1024 + stages * STAGE_BYTES + FIXED_BYTES; }
 };
 
 struct __align__(16) MmaControl {
-    uint64_t full[MmaCfg<128, 1, 1>::MAX_STAGES];
-    uint64_t empty[MmaCfg<128, 1, 1>::MAX_STAGES];
-    uint64_t full8[MmaCfg<128, 1, 1>::MAX_STAGES];   // 8-bit staging ring (KV8 only)
-    uint64_t empty8[MmaCfg<128, 1, 1>::MAX_STAGES];
+    uint64_t full[MmaCfg<128, 1, 1, true>::MAX_STAGES];
+    uint64_t empty[MmaCfg<128, 1, 1, true>::MAX_STAGES];
     uint64_t qfull[2];
     uint64_t qempty[2];
     uint64_t merge_full;
@@ -87,10 +83,14 @@ struct __align__(16) MmaControl {
 };
 static_assert(sizeof(MmaControl) <= MmaCfg<128, 1, 1, false>::CTRL_BYTES, "control block overflows its slot");
 
-// KV8: the cache holds OCP E4M3 bytes with per-KV-head scales; converter warps
-// decode each staged 8-bit tile to f16 (exactly) and the consumers run the
-// same contraction on f16 mma.sync, with k_scale folded into the score scale
-// and v_scale into the output.
+// KV8: the cache holds OCP E4M3 bytes with per-KV-head scales.  TMA stages
+// the 8-bit tiles as they are; consumers load them with ldmatrix (viewing
+// byte pairs as b16), decode to f16 in registers (exact) and run the same
+// contraction on f16 mma.sync, with k_scale folded into the score scale and
+// v_scale into the output.  The byte order ldmatrix delivers permutes the
+// head dimension inside each 16-value chunk (K side: Q is loaded with the
+// same permutation, so dot products are unchanged; V side: the accumulator
+// rows map to d = 16 m + 2 g + h, undone when the output is written).
 template <int D, int NT, int HG, bool PAGED, bool OUT_BF16, bool KV8 = false>
 __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     split_mma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -102,10 +102,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = smem_raw + (base - raw);
     const int NS = a.n_stages;
-    const int NS8 = KV8 ? a.n_stages8 : 0;
     const uint32_t stages = base;
-    const uint32_t stages8 = base + NS * C::STAGE_BYTES;
-    const int ring_bytes = NS * C::STAGE_BYTES + NS8 * C::STAGE8_BYTES;
+    const int ring_bytes = NS * C::STAGE_BYTES;
     const uint32_t qring = base + ring_bytes;
     float* merge_o = reinterpret_cast<float*>(base_ptr + ring_bytes + 2 * C::QSLOT_BYTES);
     float* merge_ml = merge_o + C::MERGE_O_FLOATS;
@@ -122,12 +120,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
-            mbar_init(smem_addr(&ctrl->full[s]), KV8 ? C::NV : 1);
+            mbar_init(smem_addr(&ctrl->full[s]), 1);
             mbar_init(smem_addr(&ctrl->empty[s]), C::TILE_WARPS);
-        }
-        for (int s = 0; s < NS8; ++s) {
-            mbar_init(smem_addr(&ctrl->full8[s]), 1);
-            mbar_init(smem_addr(&ctrl->empty8[s]), C::NV);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->qfull[s]), 1);
@@ -163,10 +157,9 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
         int64_t issued = 0, q_issued = 0;
         int page_word = 0, page_base = -1;
         bool ok = true;
-        // Tiles go to the f16/bf16 stage ring, or for 8-bit caches to the staging ring.
-        const int RN = KV8 ? NS8 : NS;
-        uint64_t* rfull = KV8 ? ctrl->full8 : ctrl->full;
-        uint64_t* rempty = KV8 ? ctrl->empty8 : ctrl->empty;
+        const int RN = NS;
+        uint64_t* rfull = ctrl->full;
+        uint64_t* rempty = ctrl->empty;
         for (int64_t gi = lo; gi < hi; ++gi) {
             const bool seg_first = (gi == lo) || (w.tile == 0);
             if (seg_first) {
@@ -204,8 +197,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
             if (lane == 0) {
                 const uint32_t bar = smem_addr(&rfull[st]);
                 if constexpr (KV8) {
-                    const uint32_t kb = stages8 + st * C::STAGE8_BYTES;  // 64 rows x D bytes each
-                    mbar_arrive_expect_tx(bar, C::STAGE8_BYTES);
+                    const uint32_t kb = stages + st * C::STAGE_BYTES;  // K then V: 64 rows x D bytes each
+                    mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
                     tma_load_4d(kb, &tmK, bar, 0, w.kv, c2, c3, pol_kv);
                     tma_load_4d(kb + kTile * D, &tmV, bar, 0, w.kv, c2, c3, pol_kv);
                 } else {
@@ -234,54 +227,6 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
                 mbar_wait(smem_addr(&ctrl->qfull[i % 2]), static_cast<uint32_t>((i / 2) & 1), nullptr);
         }
         return;
-    }
-
-    if constexpr (KV8) {
-        if (warp >= C::NC) {
-            // -------------------------------------------------------- converters
-            // Decode each staged 8-bit K and V tile (64 rows x 128 bytes, 128-byte
-            // swizzle) into the f16 stage layout the consumers read (two 64-column
-            // panels per operand, same swizzle).  E4M3 -> f16 is exact.
-            const int vt = threadIdx.x - 32 * C::NC;
-            constexpr int CHUNKS = 2 * kTile * (D / 16);  // 16-byte 8-bit chunks per stage
-            int st = 0, st8 = 0;
-            uint32_t ph = 0, ph8 = 0;
-            for (int64_t gi = lo; gi < hi; ++gi) {
-                const bool ok = mbar_wait_warp(smem_addr(&ctrl->full8[st8]), ph8, abort_flag) &&
-                                mbar_wait_warp(smem_addr(&ctrl->empty[st]), ph ^ 1u, abort_flag);
-                if (!ok) {
-                    *abort_flag = 1;
-                    if (lane == 0) atomicOr(a.status, kFlagTimeout);
-                    break;
-                }
-                const uint32_t src = stages8 + st8 * C::STAGE8_BYTES;
-                const uint32_t dst = stages + st * C::STAGE_BYTES;
-#pragma unroll 2
-                for (int i = 0; i < CHUNKS / (32 * C::NV); ++i) {
-                    const int j = vt + 32 * C::NV * i;
-                    const int op = j / (kTile * (D / 16));  // 0: K, 1: V
-                    const int row = (j / (D / 16)) % kTile;
-                    const int c = j % (D / 16);  // values d = 16c .. 16c+15
-                    const uint4 raw = ld_shared_v4(src + op * kTile * D + row * 128 + ((c ^ (row & 7)) << 4));
-                    const int ch0 = (c & 3) << 1;
-                    const uint32_t pb = dst + op * C::PANELS * C::PANEL_BYTES + (c >> 2) * C::PANEL_BYTES + row * 128;
-                    st_shared_v4(pb + ((ch0 ^ (row & 7)) << 4), e4m3x2_to_f16x2(raw.x & 0xffffu),
-                                 e4m3x2_to_f16x2(raw.x >> 16), e4m3x2_to_f16x2(raw.y & 0xffffu),
-                                 e4m3x2_to_f16x2(raw.y >> 16));
-                    st_shared_v4(pb + (((ch0 + 1) ^ (row & 7)) << 4), e4m3x2_to_f16x2(raw.z & 0xffffu),
-                                 e4m3x2_to_f16x2(raw.z >> 16), e4m3x2_to_f16x2(raw.w & 0xffffu),
-                                 e4m3x2_to_f16x2(raw.w >> 16));
-                }
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_addr(&ctrl->empty8[st8]));
-                    mbar_arrive(smem_addr(&ctrl->full[st]));
-                }
-                if (++st8 == NS8) { st8 = 0; ph8 ^= 1u; }
-                if (++st == NS) { st = 0; ph ^= 1u; }
-            }
-            return;
-        }
     }
 
     // ---------------------------------------------------------------- consumers
@@ -322,6 +267,16 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
             const uint32_t qbase = qring + qs * C::QSLOT_BYTES + hg * C::PANELS * C::QPANEL_BYTES;
             if constexpr (!C::Q_IN_REGS) {
                 // read per chunk from the ring slot; released at the segment end
+            } else if constexpr (KV8) {
+                // Head g, d = 16 ks + 4t .. 4t+3 -> k-slots (2t, 2t+1), (2t+8, 2t+9), as f16.
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int p = ks >> 2, ch = ((ks & 3) << 1) + (t >> 1);
+                    const uint2 w2 = ld_shared_v2(qbase + p * C::QPANEL_BYTES + g * 128 + ((ch ^ (g & 7)) << 4) +
+                                                  ((t & 1) << 3));
+                    qb[ks][0][0] = bf16x2_to_f16x2(w2.x);
+                    qb[ks][0][1] = bf16x2_to_f16x2(w2.y);
+                }
             } else if constexpr (NT == 2) {
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
@@ -344,15 +299,6 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
             if constexpr (C::Q_IN_REGS) {
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[qs]));
-                if constexpr (KV8) {  // the 8-bit path multiplies in f16
-#pragma unroll
-                    for (int ks = 0; ks < KS; ++ks)
-#pragma unroll
-                        for (int nt = 0; nt < NT; ++nt) {
-                            qb[ks][nt][0] = bf16x2_to_f16x2(qb[ks][nt][0]);
-                            qb[ks][nt][1] = bf16x2_to_f16x2(qb[ks][nt][1]);
-                        }
-                }
             }
             if constexpr (KV8) {
                 seg_sl2 = a.sl2 * __ldg(a.k_scale + w.kv);
@@ -374,7 +320,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
         if (mine) {
         if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { fail(); break; }
         const uint32_t kb = stages + st * C::STAGE_BYTES;
-        const uint32_t vb = kb + C::PANELS * C::PANEL_BYTES;
+        const uint32_t vb = kb + (KV8 ? kTile * D : C::PANELS * C::PANEL_BYTES);
         const int t0 = w.tile * kTile;
 
 #pragma unroll
@@ -395,11 +341,26 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
 #pragma unroll
             for (int ks = 0; ks < KS; ks += 2) {
                 uint32_t ka[2][4];
+                if constexpr (KV8) {
+                    // 8-bit K rows: byte pairs as b16; chunks ks and ks+1 for 16 tokens.
+                    uint32_t r0, r1, r2, r3;
+                    const int ch = ks + (lane >> 4);
+                    ldsm_x4(kb + krow * D + ((ch ^ (lane & 7)) << 4), r0, r1, r2, r3);
+                    ka[0][0] = e4m3x2_to_f16x2(r0 & 0xffffu);
+                    ka[0][2] = e4m3x2_to_f16x2(r0 >> 16);
+                    ka[0][1] = e4m3x2_to_f16x2(r1 & 0xffffu);
+                    ka[0][3] = e4m3x2_to_f16x2(r1 >> 16);
+                    ka[1][0] = e4m3x2_to_f16x2(r2 & 0xffffu);
+                    ka[1][2] = e4m3x2_to_f16x2(r2 >> 16);
+                    ka[1][1] = e4m3x2_to_f16x2(r3 & 0xffffu);
+                    ka[1][3] = e4m3x2_to_f16x2(r3 >> 16);
+                } else {
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                    const int p = (ks + h) >> 2, ch = (((ks + h) & 3) << 1) + (lane >> 4);
-                    ldsm_x4(kb + p * C::PANEL_BYTES + krow * 128 + ((ch ^ (lane & 7)) << 4), ka[h][0], ka[h][1],
-                            ka[h][2], ka[h][3]);
+                    for (int h = 0; h < 2; ++h) {
+                        const int p = (ks + h) >> 2, ch = (((ks + h) & 3) << 1) + (lane >> 4);
+                        ldsm_x4(kb + p * C::PANEL_BYTES + krow * 128 + ((ch ^ (lane & 7)) << 4), ka[h][0],
+                                ka[h][1], ka[h][2], ka[h][3]);
+                    }
                 }
                 if constexpr (C::Q_IN_REGS) {
 #pragma unroll
@@ -509,9 +470,31 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
 #pragma unroll
                 for (int h = 0; h < MG; ++h) {
                     const int mm = m0 + h;
-                    const int pnl = mm >> 2, ch = ((mm & 3) << 1) + ((lane >> 3) & 1);
-                    ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + vrow * 128 + ((ch ^ (lane & 7)) << 4), va[h][0],
-                                  va[h][1], va[h][2], va[h][3]);
+                    if constexpr (KV8) {
+                        // 8-bit V rows: one transposing load gives tokens (2t, 2t+1) of d = 16 mm + 2g
+                        // (bytes 0, 2) and of d = 16 mm + 2g + 1 (bytes 1, 3), for token halves 0-7 and
+                        // 8-15 of chunks mm and mm + 1; block mm's accumulator rows are d = 16 mm + 2g + {0,1}.
+                        if ((h & 1) == 0) {
+                            uint32_t r0, r1, r2, r3;
+                            ldsm_x4_trans(vb + krow * D + (((mm + (lane >> 4)) ^ (lane & 7)) << 4), r0, r1, r2,
+                                          r3);
+                            va[h][0] = e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0020));
+                            va[h][1] = e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0031));
+                            va[h][2] = e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0020));
+                            va[h][3] = e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0031));
+                            va[h + 1][0] = e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0020));
+                            va[h + 1][1] = e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0031));
+                            va[h + 1][2] = e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0020));
+                            va[h + 1][3] = e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0031));
+                        }
+                    } else {
+                        const int pnl = mm >> 2, ch = ((mm & 3) << 1) + ((lane >> 3) & 1);
+                        ldsm_x4_trans(vb + pnl * C::PANEL_BYTES + vrow * 128 + ((ch ^ (lane & 7)) << 4),
+                                      va[h][0], va[h][1], va[h][2], va[h][3]);
+                    }
+                }
+#pragma unroll
+                for (int h = 0; h < MG; ++h) {
                     if (mask) {  // rows past L_b may hold anything; 0 * NaN would poison O
                         va[h][0] &= vmask_a;
                         va[h][1] &= vmask_a;
@@ -625,7 +608,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
 #pragma unroll
                                 for (int hh = 0; hh < 2; ++hh) {
                                     const float x = o[mm][nt][j + 2 * hh] * inv;
-                                    const int64_t i = row + 16 * mm + g + 8 * hh;
+                                    const int64_t i = row + (KV8 ? 16 * mm + 2 * g + hh : 16 * mm + g + 8 * hh);
                                     if constexpr (OUT_BF16)
                                         static_cast<__nv_bfloat16*>(a.out)[i] = __float2bfloat16_rn(x);
                                     else
@@ -635,8 +618,13 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
                             float* dst = a.ws_o + (slot * a.R + r) * D;
 #pragma unroll
                             for (int mm = 0; mm < KS; ++mm) {
-                                dst[16 * mm + g] = o[mm][nt][j] * inv;
-                                dst[16 * mm + g + 8] = o[mm][nt][j + 2] * inv;
+                                if constexpr (KV8) {
+                                    *reinterpret_cast<float2*>(dst + 16 * mm + 2 * g) =
+                                        make_float2(o[mm][nt][j] * inv, o[mm][nt][j + 2] * inv);
+                                } else {
+                                    dst[16 * mm + g] = o[mm][nt][j] * inv;
+                                    dst[16 * mm + g + 8] = o[mm][nt][j + 2] * inv;
+                                }
                             }
                             if (g == 0) a.ws_lse[slot * a.R + r] = M[nt][j] + log2f(Lsum[nt][j]);
                         }

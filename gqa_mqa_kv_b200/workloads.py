@@ -87,6 +87,7 @@ WORKLOADS: dict[str, Workload] = {
         _wl("sweep_hkv1", 32, 32, 1, 128, 8192, 3),
         _wl("llama2_70b_ragged", 32, 64, 8, 128, 32768, 4, ragged=True),
         _wl("paged_long", 8, 64, 8, 128, 131072, 5, page_size=PAGE_SIZE),
+        _wl("llama3_8b_fp8", 16, 32, 8, 128, 4096, 2, kv8=True),
         _wl("llama2_70b_ragged_fp8", 32, 64, 8, 128, 32768, 4, ragged=True, kv8=True),
         _wl("paged_long_fp8", 8, 64, 8, 128, 131072, 5, page_size=PAGE_SIZE, kv8=True),
     ]
