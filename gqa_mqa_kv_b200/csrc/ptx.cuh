@@ -6,7 +6,6 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
-#include <cuda_fp8.h>
 #include <stdint.h>
 
 namespace gqa {
@@ -179,10 +178,27 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t x) {
     return *reinterpret_cast<const uint32_t*>(&h);
 }
 
-// Two packed OCP E4M3 values (low byte first) to two packed f16 values; exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+// (a & c) | (b & ~c), one lop3.
+__device__ __forceinline__ uint32_t bit_select(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xE4;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Four packed OCP E4M3 bytes r = [b3 b2 b1 b0] to two f16x2 words holding
+// each value times 2^-8, exactly: even = (b0, b2), odd = (b1, b3), low half
+// first.  An E4M3 byte is sign | 4 exponent bits (bias 7) | 3 mantissa bits;
+// its 7 magnitude bits placed at f16 bits 13..7 form an f16 (bias 15) with
+// the same exponent and mantissa fields, i.e. the value times 2^-8 --
+// subnormals included, since both formats take 2^(1-bias) there.  The sign
+// goes to bit 15.  The NaN encodings S.1111.111 decode as +-480 * 2^-8.
+// Cost: three logic ops and three integer multiplies (the shifts) for four
+// values, against a conversion instruction per pair plus byte extraction.
+__device__ __forceinline__ void e4m3x4_to_f16x2_scaled(uint32_t r, uint32_t& even, uint32_t& odd) {
+    constexpr uint32_t kMag = 0x3F803F80u;  // f16 bits 13..7 of both halves
+    const uint32_t sgn = r & 0x80808080u;   // sign bits of the four bytes, in place
+    odd = bit_select(__umulhi(r, 0x80000000u), sgn, kMag);  // magnitudes of b1, b3 from r >> 1
+    even = bit_select(r << 7, sgn << 8, kMag);              // magnitudes of b0, b2 from r << 7
 }
 
 // m16n8k16 on f16 operands (F16) or bf16 operands.

@@ -85,12 +85,13 @@ static_assert(sizeof(MmaControl) <= MmaCfg<128, 1, 1, false>::CTRL_BYTES, "contr
 
 // KV8: the cache holds OCP E4M3 bytes with per-KV-head scales.  TMA stages
 // the 8-bit tiles as they are; consumers load them with ldmatrix (viewing
-// byte pairs as b16), decode to f16 in registers (exact) and run the same
-// contraction on f16 mma.sync, with k_scale folded into the score scale and
-// v_scale into the output.  The byte order ldmatrix delivers permutes the
-// head dimension inside each 16-value chunk (K side: Q is loaded with the
-// same permutation, so dot products are unchanged; V side: the accumulator
-// rows map to d = 16 m + 2 g + h, undone when the output is written).
+// byte pairs as b16), decode them in registers by bit placement to f16
+// holding value * 2^-8 (exact) and run the same contraction on f16
+// mma.sync, with 2^8 * k_scale folded into the score scale and 2^8 * v_scale
+// into the output.  The byte order ldmatrix delivers permutes the head
+// dimension inside each 16-value chunk (K side: Q is loaded with the same
+// permutation, so dot products are unchanged; V side: the accumulator rows
+// map to d = 16 m + 2 g + h, undone when the output is written).
 template <int D, int NT, int HG, bool PAGED, bool OUT_BF16, bool KV8 = false>
 __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     split_mma_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -268,14 +269,15 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
             if constexpr (!C::Q_IN_REGS) {
                 // read per chunk from the ring slot; released at the segment end
             } else if constexpr (KV8) {
-                // Head g, d = 16 ks + 4t .. 4t+3 -> k-slots (2t, 2t+1), (2t+8, 2t+9), as f16.
+                // Head g, d = 16 ks + 4t + {0, 2} -> k-slots (2t, 2t+1) and d = 16 ks + 4t + {1, 3}
+                // -> k-slots (2t+8, 2t+9), as f16: the order the K decode below produces.
 #pragma unroll
                 for (int ks = 0; ks < KS; ++ks) {
                     const int p = ks >> 2, ch = ((ks & 3) << 1) + (t >> 1);
                     const uint2 w2 = ld_shared_v2(qbase + p * C::QPANEL_BYTES + g * 128 + ((ch ^ (g & 7)) << 4) +
                                                   ((t & 1) << 3));
-                    qb[ks][0][0] = bf16x2_to_f16x2(w2.x);
-                    qb[ks][0][1] = bf16x2_to_f16x2(w2.y);
+                    qb[ks][0][0] = bf16x2_to_f16x2(__byte_perm(w2.x, w2.y, 0x5410));
+                    qb[ks][0][1] = bf16x2_to_f16x2(__byte_perm(w2.x, w2.y, 0x7632));
                 }
             } else if constexpr (NT == 2) {
 #pragma unroll
@@ -300,9 +302,9 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[qs]));
             }
-            if constexpr (KV8) {
-                seg_sl2 = a.sl2 * __ldg(a.k_scale + w.kv);
-                seg_vs = __ldg(a.v_scale + w.kv);
+            if constexpr (KV8) {  // the decode yields e4m3 * 2^-8: fold 2^8 back in
+                seg_sl2 = a.sl2 * (256.f * __ldg(a.k_scale + w.kv));
+                seg_vs = 256.f * __ldg(a.v_scale + w.kv);
             }
             if (++qs == 2) { qs = 0; qph ^= 1u; }
 #pragma unroll
@@ -342,18 +344,16 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
             for (int ks = 0; ks < KS; ks += 2) {
                 uint32_t ka[2][4];
                 if constexpr (KV8) {
-                    // 8-bit K rows: byte pairs as b16; chunks ks and ks+1 for 16 tokens.
+                    // 8-bit K rows: byte pairs as b16; chunks ks and ks+1 for 16 tokens.  Each
+                    // word holds d = 4t .. 4t+3 of one token; the decode pairs (4t, 4t+2) and
+                    // (4t+1, 4t+3).
                     uint32_t r0, r1, r2, r3;
                     const int ch = ks + (lane >> 4);
                     ldsm_x4(kb + krow * D + ((ch ^ (lane & 7)) << 4), r0, r1, r2, r3);
-                    ka[0][0] = e4m3x2_to_f16x2(r0 & 0xffffu);
-                    ka[0][2] = e4m3x2_to_f16x2(r0 >> 16);
-                    ka[0][1] = e4m3x2_to_f16x2(r1 & 0xffffu);
-                    ka[0][3] = e4m3x2_to_f16x2(r1 >> 16);
-                    ka[1][0] = e4m3x2_to_f16x2(r2 & 0xffffu);
-                    ka[1][2] = e4m3x2_to_f16x2(r2 >> 16);
-                    ka[1][1] = e4m3x2_to_f16x2(r3 & 0xffffu);
-                    ka[1][3] = e4m3x2_to_f16x2(r3 >> 16);
+                    e4m3x4_to_f16x2_scaled(r0, ka[0][0], ka[0][2]);
+                    e4m3x4_to_f16x2_scaled(r1, ka[0][1], ka[0][3]);
+                    e4m3x4_to_f16x2_scaled(r2, ka[1][0], ka[1][2]);
+                    e4m3x4_to_f16x2_scaled(r3, ka[1][1], ka[1][3]);
                 } else {
 #pragma unroll
                     for (int h = 0; h < 2; ++h) {
@@ -478,14 +478,10 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
                             uint32_t r0, r1, r2, r3;
                             ldsm_x4_trans(vb + krow * D + (((mm + (lane >> 4)) ^ (lane & 7)) << 4), r0, r1, r2,
                                           r3);
-                            va[h][0] = e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0020));
-                            va[h][1] = e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0031));
-                            va[h][2] = e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0020));
-                            va[h][3] = e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0031));
-                            va[h + 1][0] = e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0020));
-                            va[h + 1][1] = e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0031));
-                            va[h + 1][2] = e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0020));
-                            va[h + 1][3] = e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0031));
+                            e4m3x4_to_f16x2_scaled(r0, va[h][0], va[h][1]);
+                            e4m3x4_to_f16x2_scaled(r1, va[h][2], va[h][3]);
+                            e4m3x4_to_f16x2_scaled(r2, va[h + 1][0], va[h + 1][1]);
+                            e4m3x4_to_f16x2_scaled(r3, va[h + 1][2], va[h + 1][3]);
                         }
                     } else {
                         const int pnl = mm >> 2, ch = ((mm & 3) << 1) + ((lane >> 3) & 1);
