@@ -19,6 +19,7 @@
 #include "combine.cuh"
 #include "split_mma.cuh"
 #include "split_simt.cuh"
+#include "split_tc.cuh"
 #include "rope_append.cuh"
 
 namespace {
@@ -232,6 +233,73 @@ cudaError_t launch_mma_groups(const gqa_decode_params* p, const Buffers& buf,
     return launch_mma<D, 4, 2, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
 }
 
+// tcgen05 split kernel (head_dim 128): RP query columns per KV head.
+template <int RP, bool PAGED, bool OUTB, bool KV8>
+cudaError_t launch_tc(const gqa_decode_params* p, const Buffers& buf, KernelArgs args, const DeviceInfo& dev,
+                      int grid, cudaStream_t stream, bool* encode_ok) {
+    using C = TcCfg<RP, KV8>;
+    constexpr int D = 128;
+    int stages = (dev.smem_optin - C::FIXED_BYTES - 1024) / C::STAGE_BYTES;
+    if (stages > C::MAX_STAGES) stages = C::MAX_STAGES;
+    if (stages < 2) return cudaErrorInvalidConfiguration;
+    args.n_stages = stages;
+
+    CUtensorMap tmQ, tmK, tmV;
+    const uint64_t row = static_cast<uint64_t>(D) * 2;
+    {
+        const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(p->H_Q),
+                                  static_cast<uint64_t>(p->B)};
+        const uint64_t strides[2] = {row, row * p->H_Q};
+        const uint32_t box[3] = {64, static_cast<uint32_t>(RP), 1};
+        *encode_ok = encode_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, buf.q, 3, dims, strides, box);
+    }
+    // K/V boxes: 64 tokens x 64 bf16 (128 bytes), or 64 tokens x 128 E4M3 bytes.
+    const uint32_t box4[4] = {KV8 ? static_cast<uint32_t>(D) : 64u, 1, static_cast<uint32_t>(kTile), 1};
+    const uint64_t kv_row = KV8 ? static_cast<uint64_t>(D) : row;
+    if (*encode_ok) {
+        uint64_t dims[4], strides[3];
+        dims[0] = D;
+        dims[1] = p->H_KV;
+        strides[0] = kv_row;
+        strides[1] = kv_row * p->H_KV;
+        if (PAGED) {
+            dims[2] = kTile;
+            dims[3] = p->num_blocks;
+        } else {
+            dims[2] = p->max_seq_len > 0 ? p->max_seq_len : 1;
+            dims[3] = p->B;
+        }
+        strides[2] = strides[1] * dims[2];
+        const CUtensorMapDataType kv_type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+        *encode_ok = encode_map(&tmK, kv_type, buf.k, 4, dims, strides, box4) &&
+                     encode_map(&tmV, kv_type, buf.v, 4, dims, strides, box4);
+    }
+    if (!*encode_ok) return cudaErrorInvalidValue;
+    auto kernel = split_tc_kernel<RP, PAGED, OUTB, KV8>;
+    const int smem = C::smem_bytes(stages);
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), smem);
+    if (e != cudaSuccess) return e;
+    return launch_chained(kernel, grid, C::THREADS, smem, stream, tmQ, tmK, tmV, args);
+}
+
+template <bool PAGED, bool OUTB, bool KV8>
+cudaError_t launch_tc_groups(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
+                             const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
+    const int R = p->H_Q / p->H_KV;
+    if (R <= 8) return launch_tc<8, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
+    if (R <= 16) return launch_tc<16, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
+    return launch_tc<32, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
+}
+
+// Which split kernel serves a problem: the tcgen05 kernel for head_dim 128
+// with an 8-bit cache (R <= 32) or a bf16 cache with 8 < R <= 32; the
+// mma.sync kernel for the other bf16 groups up to 64; CUDA cores otherwise.
+bool use_tc(const gqa_decode_params* p, bool kv8) {
+    const int R = p->H_Q / p->H_KV;
+    if (p->head_dim != 128 || R > 32) return false;
+    return kv8 || (p->qkv_dtype == GQA_BF16 && R > 8);
+}
+
 template <typename TQ, typename TKV, int D, bool PAGED, bool OUTB>
 cudaError_t launch_simt(const Buffers& buf, const KernelArgs& args, int grid, cudaStream_t stream) {
     return launch_chained(split_simt_kernel<TQ, TKV, D, PAGED, OUTB>, grid, 32 * kSimtWarps, 0, stream,
@@ -242,13 +310,13 @@ cudaError_t launch_simt(const Buffers& buf, const KernelArgs& args, int grid, cu
 template <int D, bool PAGED, bool OUTB>
 cudaError_t launch_split(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
                          const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
-    if (buf.kv8) {
-        if constexpr (D == 128) {
-            if (p->H_Q / p->H_KV <= 8)
-                return launch_mma<128, 1, 1, PAGED, OUTB, true>(p, buf, args, dev, grid, stream, encode_ok);
+    if constexpr (D == 128) {
+        if (use_tc(p, buf.kv8)) {
+            return buf.kv8 ? launch_tc_groups<PAGED, OUTB, true>(p, buf, args, dev, grid, stream, encode_ok)
+                           : launch_tc_groups<PAGED, OUTB, false>(p, buf, args, dev, grid, stream, encode_ok);
         }
-        return launch_simt<__nv_bfloat16, __nv_fp8_e4m3, D, PAGED, OUTB>(buf, args, grid, stream);
     }
+    if (buf.kv8) return launch_simt<__nv_bfloat16, __nv_fp8_e4m3, D, PAGED, OUTB>(buf, args, grid, stream);
     if (use_tensor_cores(p)) return launch_mma_groups<D, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (p->qkv_dtype == GQA_F32) return launch_simt<float, float, D, PAGED, OUTB>(buf, args, grid, stream);
     return launch_simt<__nv_bfloat16, __nv_bfloat16, D, PAGED, OUTB>(buf, args, grid, stream);

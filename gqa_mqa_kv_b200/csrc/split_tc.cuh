@@ -1,0 +1,798 @@
+// split_tc.cuh -- split-KV decode on the 5th-generation tensor cores
+// (tcgen05, accumulators in tensor memory) for head_dim 128.
+//
+// What it computes is the split kernel's contract (schedule.cuh): for every
+// segment, the R query heads of one (sequence, KV head) pair attend over the
+// segment's tokens ("Grouped-Query Attention (GQA) and Multi-Query Attention
+// (MQA): Mathematical Foundations, ...", section 2, Head_i = softmax(Q_i
+// K_{g(i)}^T / sqrt(d_k)) V_{g(i)}), with an fp32 online softmax in base 2;
+// a whole-unit segment writes the output, others write (normalised o,
+// log2-sum-exp) partials for the combine kernel.
+//
+// Per 64-token tile:
+//   S^T = K Q^T     tcgen05.mma, M = 64 tokens, N = query columns, K = d:
+//                   A = the K tile as TMA staged it (K-major, 128-byte
+//                   swizzle), B = the query rows; S^T lands in tensor memory
+//                   (two buffers, so the next tile's product overlaps this
+//                   tile's softmax).
+//   softmax         four warps; thread = token (row of S^T): p = 2^(s - m)
+//                   against a per-head reference m shared by all tokens,
+//                   moved only when a score exceeds it by more than 8
+//                   (all threads agree through an mbarrier exchange).
+//                   P^T is written to shared memory as bf16 (or f16) hi and
+//                   lo parts -- N = 2 * RP columns -- so the product keeps
+//                   fp32-level precision of the weights.
+//   O^T += V^T P^T  tcgen05.mma, M = 128 (d), N = 2 RP, K = 64 tokens:
+//                   A = the V tile read MN-major, B = P^T; O^T accumulates in
+//                   tensor memory over the segment; hi and lo columns are
+//                   summed in the epilogue.
+//
+// 8-bit caches (KV8, OCP E4M3 with per-KV-head scales): the score product
+// runs as kind::f8f6f4 directly on the staged E4M3 key bytes.  Each query
+// head is scaled by a power of two 2^a (max |q| * 2^a in [128, 256)) and
+// split into two E4M3 terms, q 2^a = t1 + t2 / 16 (exact for every element
+// of magnitude >= 2^-6 after scaling; smaller ones err by <= 2^-14), held as
+// query columns h and RP + h; s = (S[h] + S[RP + h] / 16) 2^-a.  Four
+// converter warps widen each V tile to f16 (exact) for a kind::f16 value
+// product; P is scaled by 2^7 so its f16 hi/lo parts stay normal.
+//
+// Warp roles: 0 TMA producer, 1 score products (+ tensor-memory
+// allocation), 2 value products, 3..6 softmax and epilogue (sub-partitions
+// 3, 0, 1, 2), 7..10 V converters (KV8).  Every wait is bounded (kWaitTimeoutNs); on a timeout the CTA raises
+// GQA_FLAG_TIMEOUT, lets its copies and products drain, frees its tensor
+// memory and returns.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+#include "tcgen05.cuh"
+
+namespace gqa {
+
+template <int RP, bool KV8>
+struct TcCfg {
+    static_assert(RP == 8 || RP == 16 || RP == 32, "query columns per KV head: 8, 16 or 32");
+    static constexpr int D = 128;
+    static constexpr int NS_COLS = KV8 ? 2 * RP : RP;  // S^T columns: heads, or two query terms per head
+    static constexpr int NO_COLS = 2 * RP;             // O^T columns: P hi | P lo
+    static constexpr int S_COL = 0;                    // S^T buffer b at S_COL + b * NS_COLS
+    static constexpr int O_COL = 2 * NS_COLS;
+    static constexpr int TMEM_COLS = 512;              // the whole tensor memory of the SM
+    static constexpr int NSM = 4;                      // softmax warps
+    static constexpr int NCV = KV8 ? 4 : 0;            // converter warps
+    static constexpr int WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3, WARP_CV0 = 3 + NSM;
+    static constexpr int THREADS = 32 * (3 + NSM + NCV);
+    static constexpr int KV_TILE_BYTES = KV8 ? kTile * D : kTile * D * 2;  // one of K, V
+    static constexpr int STAGE_BYTES = 2 * KV_TILE_BYTES;
+    static constexpr int PANEL_BYTES = kTile * 128;    // bf16 tile panel: 64 tokens x 64 d
+    static constexpr int QPANEL_BYTES = RP * 128;      // bf16 query panel: RP rows x 64 d
+    static constexpr int QSLOT_BYTES = 2 * QPANEL_BYTES;
+    static constexpr int QT_BYTES = KV8 ? NS_COLS * 128 : 0;  // E4M3 query terms: 2 RP rows x 128 d
+    static constexpr int P_BYTES = (NO_COLS / 8) * 1024;      // P^T: 8-column groups x 8 token groups x 128 B
+    static constexpr int VC_BYTES = KV8 ? kTile * D * 2 : 0;  // f16 V tile (two 64-d panels)
+    static constexpr int NVC = KV8 ? 2 : 0;
+    static constexpr int MAX_STAGES = 12;
+    static constexpr int T_LAZY = 8;                   // reference slack, base 2
+    // fixed region after the stage ring; every piece 1024-aligned
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_QT = OFF_Q + 2 * QSLOT_BYTES;
+    static constexpr int OFF_P = OFF_QT + 2 * QT_BYTES;
+    static constexpr int OFF_VC = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_X = OFF_VC + NVC * VC_BYTES;       // exchange scratch
+    static constexpr int X_BYTES = 2 * NSM * 32 * 4 + 2 * 32 * 4 + 2 * NSM * 4;
+    static constexpr int OFF_CTRL = OFF_X + ((X_BYTES + 1023) / 1024) * 1024;
+    static constexpr int CTRL_BYTES = 1024;
+    static constexpr int FIXED_BYTES = OFF_CTRL + CTRL_BYTES;
+    static constexpr int smem_bytes(int stages) { return 1024 + stages * STAGE_BYTES + FIXED_BYTES; }
+};
+
+struct __align__(16) TcControl {
+    uint64_t full[12], empty[12];   // stage ring
+    uint64_t qfull[2], qempty[2];   // bf16 query slots (TMA)
+    uint64_t qtfull[2], qtempty[2]; // E4M3 query terms (KV8)
+    uint64_t sfull[2];              // S^T buffer b written
+    uint64_t pfull[2];              // P^T buffer b written (tile j uses b = j & 1)
+    uint64_t vcfull[2];             // converted V buffer b written (KV8)
+    uint64_t pvdone[2];             // value product of the last tile using buffer b completed
+    uint64_t ofull, ofree;          // O^T of a segment complete / read by the epilogue
+    uint64_t xch;                   // softmax-warp exchange (count 4)
+    uint64_t drain[2];              // final completion of each issuing warp's products
+    Plan plan;
+    uint32_t tmem_base;
+    int abort;
+};
+
+// Scratch for the softmax warps' exchanges (double-buffered by exchange parity).
+struct TcExchange {
+    float vals[2][4][32];  // per warp, per head: tile maxima or row sums
+    float qscale[2][32];   // KV8: 2^-a per head, per query-term slot
+    int flags[2][4];
+};
+
+__device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_async_smem_writes() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// Round-to-nearest-even E4M3 of two floats, packed low byte first (saturating).
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(v), __NV_E4M3);
+    return make_float2(__half2float(__ushort_as_half(h.x)), __half2float(__ushort_as_half(h.y)));
+}
+
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_raw(uint32_t two_bytes) {
+    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes), __NV_E4M3);
+    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
+}
+
+// hi + lo split of two weights into the operand type of the value product.
+template <bool F16>
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
+    if constexpr (F16) {
+        const __half2 h = __floats2half2_rn(a, b);
+        const float2 hf = __half22float2(h);
+        const __half2 l = __floats2half2_rn(a - hf.x, b - hf.y);
+        hi = *reinterpret_cast<const uint32_t*>(&h);
+        lo = *reinterpret_cast<const uint32_t*>(&l);
+    } else {
+        const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+        const float2 hf = __bfloat1622float2(h);
+        const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+        hi = *reinterpret_cast<const uint32_t*>(&h);
+        lo = *reinterpret_cast<const uint32_t*>(&l);
+    }
+}
+
+template <int RP, bool PAGED, bool OUT_BF16, bool KV8>
+__global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
+    split_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const KernelArgs a) {
+    using C = TcCfg<RP, KV8>;
+    static_assert(sizeof(TcControl) <= C::CTRL_BYTES, "control block overflows its slot");
+    static_assert(sizeof(TcExchange) <= C::X_BYTES, "exchange scratch overflows its slot");
+    constexpr uint32_t IDESC_QK = KV8 ? tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, 0, 0, 64, C::NS_COLS)
+                                      : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 64, C::NS_COLS);
+    constexpr uint32_t IDESC_PV = KV8 ? tc::instr_desc(tc::kFmtF16, tc::kFmtF16, 1, 1, 128, C::NO_COLS)
+                                      : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 1, 1, 128, C::NO_COLS);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const int NS = a.n_stages;
+    const uint32_t stages = base;
+    const uint32_t fixed = base + NS * C::STAGE_BYTES;
+    uint8_t* fixed_ptr = base_ptr + NS * C::STAGE_BYTES;
+    const uint32_t q_base = fixed + C::OFF_Q;
+    const uint32_t qt_base = fixed + C::OFF_QT;
+    const uint32_t p_base = fixed + C::OFF_P;
+    const uint32_t vc_base = fixed + C::OFF_VC;
+    TcExchange* X = reinterpret_cast<TcExchange*>(fixed_ptr + C::OFF_X);
+    TcControl* ctrl = reinterpret_cast<TcControl*>(fixed_ptr + C::OFF_CTRL);
+    volatile int* abort_flag = &ctrl->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            mbar_init(smem_addr(&ctrl->full[s]), 1);
+            mbar_init(smem_addr(&ctrl->empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&ctrl->qfull[s]), 1);
+            mbar_init(smem_addr(&ctrl->qempty[s]), KV8 ? C::NSM : 1);
+            mbar_init(smem_addr(&ctrl->qtfull[s]), C::NSM);
+            mbar_init(smem_addr(&ctrl->qtempty[s]), 1);
+            mbar_init(smem_addr(&ctrl->sfull[s]), 1);
+            mbar_init(smem_addr(&ctrl->pfull[s]), C::NSM);
+            mbar_init(smem_addr(&ctrl->vcfull[s]), KV8 ? C::NCV : 1);
+            mbar_init(smem_addr(&ctrl->pvdone[s]), 1);
+            mbar_init(smem_addr(&ctrl->drain[s]), 1);
+        }
+        mbar_init(smem_addr(&ctrl->ofull), 1);
+        mbar_init(smem_addr(&ctrl->ofree), C::NSM);
+        mbar_init(smem_addr(&ctrl->xch), C::NSM);
+        ctrl->abort = 0;
+    }
+    // Query rows past H_Q come back from TMA as zeros; the P^T buffers start
+    // zeroed so their padding columns are finite.
+    for (int i = threadIdx.x; i < (2 * C::QSLOT_BYTES + 2 * C::QT_BYTES + 2 * C::P_BYTES) / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(fixed_ptr + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
+
+    grid_dependency_wait();
+    grid_launch_dependents();
+    if (warp == 0) make_plan(a, &ctrl->plan);
+    if (warp == C::WARP_QK) {
+        tc::tmem_alloc(smem_addr(&ctrl->tmem_base), C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ctrl->tmem_base;
+
+    const int64_t lo = ctrl->plan.lo;
+    const int64_t hi = ctrl->plan.hi;
+    Walk w{ctrl->plan.b, ctrl->plan.kv, ctrl->plan.tile, ctrl->plan.n_b, ctrl->plan.L};
+    auto fail = [&]() {
+        *abort_flag = 1;
+        if (lane == 0) atomicOr(a.status, kFlagTimeout);
+    };
+
+    if (lo < hi && warp == 0) {
+        // ------------------------------------------------------------ producer
+        const uint64_t pol_kv = policy_evict_first();
+        const uint64_t pol_q = policy_evict_last();
+        int st = 0, qs = 0;
+        uint32_t ph = 0, qph = 0;
+        int64_t issued = 0, q_issued = 0;
+        int page_word = 0, page_base = -1;
+        bool ok = true;
+        for (int64_t gi = lo; gi < hi; ++gi) {
+            const bool seg_first = (gi == lo) || (w.tile == 0);
+            if (seg_first) {
+                if (!mbar_wait_warp(smem_addr(&ctrl->qempty[qs]), qph ^ 1u, abort_flag)) { ok = false; break; }
+                if (lane == 0) {
+                    const uint32_t bar = smem_addr(&ctrl->qfull[qs]);
+                    mbar_arrive_expect_tx(bar, C::QSLOT_BYTES);
+                    for (int p = 0; p < 2; ++p)
+                        tma_load_3d(q_base + qs * C::QSLOT_BYTES + p * C::QPANEL_BYTES, &tmQ, bar, 64 * p,
+                                    w.kv * a.R, w.b, pol_q);
+                }
+                ++q_issued;
+                if (++qs == 2) { qs = 0; qph ^= 1u; }
+            }
+            int c2, c3;
+            if constexpr (PAGED) {
+                const int tb = w.tile & ~31;
+                if (seg_first || tb != page_base) {
+                    page_base = tb;
+                    const int idx = tb + lane;
+                    page_word = idx < w.n_b
+                                    ? __ldg(a.block_table + static_cast<int64_t>(w.b) * a.max_blocks + idx)
+                                    : 0;
+                }
+                const int page = __shfl_sync(0xffffffffu, page_word, w.tile & 31);
+                if ((page < 0 || page >= a.num_blocks) && lane == 0) atomicOr(a.status, kFlagBadBlock);
+                c2 = 0;
+                c3 = page;  // out of range: the TMA unit fills the tile with zeros
+            } else {
+                c2 = w.tile * kTile;
+                c3 = w.b;
+            }
+            if (!mbar_wait_warp(smem_addr(&ctrl->empty[st]), ph ^ 1u, abort_flag)) { ok = false; break; }
+            if (lane == 0) {
+                const uint32_t bar = smem_addr(&ctrl->full[st]);
+                const uint32_t kb = stages + st * C::STAGE_BYTES;
+                const uint32_t vb = kb + C::KV_TILE_BYTES;
+                mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
+                if constexpr (KV8) {
+                    tma_load_4d(kb, &tmK, bar, 0, w.kv, c2, c3, pol_kv);
+                    tma_load_4d(vb, &tmV, bar, 0, w.kv, c2, c3, pol_kv);
+                } else {
+                    for (int p = 0; p < 2; ++p) {
+                        tma_load_4d(kb + p * C::PANEL_BYTES, &tmK, bar, 64 * p, w.kv, c2, c3, pol_kv);
+                        tma_load_4d(vb + p * C::PANEL_BYTES, &tmV, bar, 64 * p, w.kv, c2, c3, pol_kv);
+                    }
+                }
+            }
+            ++issued;
+            if (++st == NS) { st = 0; ph ^= 1u; }
+            if (gi + 1 < hi) w.advance(a);
+        }
+        if (!ok) {
+            fail();
+            // Let copies already in flight land before the CTA's shared memory goes away.
+            const int64_t first = issued > NS ? issued - NS : 0;
+            for (int64_t i = first; i < issued; ++i)
+                mbar_wait(smem_addr(&ctrl->full[i % NS]), static_cast<uint32_t>((i / NS) & 1), nullptr);
+            const int64_t qfirst = q_issued > 2 ? q_issued - 2 : 0;
+            for (int64_t i = qfirst; i < q_issued; ++i)
+                mbar_wait(smem_addr(&ctrl->qfull[i % 2]), static_cast<uint32_t>((i / 2) & 1), nullptr);
+        }
+    }
+
+    if (warp == C::WARP_QK) {
+        // ------------------------------------------------------------ score products
+        // Tile j: S^T(j) = K(j) Q^T into buffer b = j & 1, once the softmax
+        // warps are done with the tile that used b before (j - 2).
+        int st = 0, qs = 0, qcur = 0;
+        uint32_t ph = 0, qph = 0;
+        bool ok = true;
+        if (lo < hi) {
+            int j = 0;
+            for (int64_t gi = lo; gi < hi; ++gi, ++j) {
+                const bool seg_first = (gi == lo) || (w.tile == 0);
+                const bool seg_last = (gi == hi - 1) || (w.tile == w.n_b - 1);
+                const int b = j & 1;
+                const uint32_t bpar = static_cast<uint32_t>(j >> 1) & 1u;
+                if (seg_first) {
+                    const uint32_t qbar = KV8 ? smem_addr(&ctrl->qtfull[qs]) : smem_addr(&ctrl->qfull[qs]);
+                    if (!mbar_wait_warp(qbar, qph, abort_flag)) { ok = false; break; }
+                    qcur = qs;
+                    if (++qs == 2) { qs = 0; qph ^= 1u; }
+                }
+                if (!mbar_wait_warp(smem_addr(&ctrl->pfull[b]), bpar ^ 1u, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { ok = false; break; }
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    const uint32_t kt = stages + st * C::STAGE_BYTES;
+                    const uint32_t sd = tmem + C::S_COL + b * C::NS_COLS;
+                    if constexpr (KV8) {
+                        const uint32_t qt = qt_base + qcur * C::QT_BYTES;
+#pragma unroll
+                        for (int k = 0; k < 4; ++k) {
+                            const uint64_t da = tc::smem_desc(kt + 32 * k, 16, 1024, tc::kLayoutSw128);
+                            const uint64_t db = tc::smem_desc(qt + 32 * k, 16, 1024, tc::kLayoutSw128);
+                            tc::mma_f8(sd, da, db, IDESC_QK, k > 0);
+                        }
+                    } else {
+                        const uint32_t qt = q_base + qcur * C::QSLOT_BYTES;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t da = tc::smem_desc(kt + (k >> 2) * C::PANEL_BYTES + 32 * (k & 3), 16,
+                                                              1024, tc::kLayoutSw128);
+                            const uint64_t db = tc::smem_desc(qt + (k >> 2) * C::QPANEL_BYTES + 32 * (k & 3), 16,
+                                                              1024, tc::kLayoutSw128);
+                            tc::mma_f16(sd, da, db, IDESC_QK, k > 0);
+                        }
+                    }
+                    tc::commit(smem_addr(&ctrl->sfull[b]));
+                    if (seg_last)  // the segment's query slot is free once its last score product is done
+                        tc::commit(KV8 ? smem_addr(&ctrl->qtempty[qcur]) : smem_addr(&ctrl->qempty[qcur]));
+                }
+                __syncwarp();
+                if (++st == NS) { st = 0; ph ^= 1u; }
+                if (gi + 1 < hi) w.advance(a);
+            }
+            if (!ok) fail();
+        }
+        // Every product this warp issued has completed before tensor memory is freed.
+        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain[0]));
+        __syncwarp();
+        mbar_wait_warp(smem_addr(&ctrl->drain[0]), 0u, nullptr);
+    }
+
+    if (warp == C::WARP_PV) {
+        // ------------------------------------------------------------ value products
+        // Tile j: O^T += V^T(j) P^T(j) once the softmax warps have written P^T(j)
+        // (and, KV8, the converters the f16 V tile); a segment's first tile
+        // overwrites O^T after the epilogue has read the previous segment's.
+        int st = 0, seg = -1;
+        bool ok = true;
+        if (lo < hi) {
+            int j = 0;
+            for (int64_t gi = lo; gi < hi; ++gi, ++j) {
+                const bool seg_first = (gi == lo) || (w.tile == 0);
+                const bool seg_last = (gi == hi - 1) || (w.tile == w.n_b - 1);
+                const int b = j & 1;
+                const uint32_t bpar = static_cast<uint32_t>(j >> 1) & 1u;
+                if (seg_first) ++seg;
+                if (!mbar_wait_warp(smem_addr(&ctrl->pfull[b]), bpar, abort_flag)) { ok = false; break; }
+                if constexpr (KV8)
+                    if (!mbar_wait_warp(smem_addr(&ctrl->vcfull[b]), bpar, abort_flag)) { ok = false; break; }
+                if (seg_first && seg > 0)
+                    if (!mbar_wait_warp(smem_addr(&ctrl->ofree), static_cast<uint32_t>(seg - 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    const uint32_t vt = KV8 ? vc_base + b * C::VC_BYTES
+                                            : stages + st * C::STAGE_BYTES + C::KV_TILE_BYTES;
+                    const uint32_t pt = p_base + b * C::P_BYTES;
+#pragma unroll
+                    for (int k = 0; k < kTile / 16; ++k) {
+                        const uint64_t da = tc::smem_desc(vt + k * 2048, C::PANEL_BYTES, 1024, tc::kLayoutSw128);
+                        const uint64_t db = tc::smem_desc(pt + k * 256, 128, 1024, tc::kLayoutNone);
+                        tc::mma_f16(tmem + C::O_COL, da, db, IDESC_PV, !(seg_first && k == 0));
+                    }
+                    tc::commit(smem_addr(&ctrl->empty[st]));
+                    tc::commit(smem_addr(&ctrl->pvdone[b]));
+                    if (seg_last) tc::commit(smem_addr(&ctrl->ofull));
+                }
+                __syncwarp();
+                if (++st == NS) st = 0;
+                if (gi + 1 < hi) w.advance(a);
+            }
+            if (!ok) fail();
+        }
+        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain[1]));
+        __syncwarp();
+        mbar_wait_warp(smem_addr(&ctrl->drain[1]), 0u, nullptr);
+    }
+
+    if constexpr (KV8) {
+        if (lo < hi && warp >= C::WARP_CV0) {
+            // ------------------------------------------------------------ V converters
+            // Thread (t, hf): token row t, d half hf; E4M3 -> f16 (exact) into the
+            // bf16-style layout (two 64-d panels, 128-byte swizzle); rows past L_b
+            // are written as zeros so 0 * NaN cannot reach O^T.
+            const int ct = threadIdx.x - 32 * C::WARP_CV0;
+            const int t = ct >> 1, hf = ct & 1;
+            int st = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            int j = 0;
+            for (int64_t gi = lo; gi < hi; ++gi, ++j) {
+                const int c = j & 1;
+                const uint32_t par = static_cast<uint32_t>(j >> 1) & 1u;
+                if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[c]), par ^ 1u, abort_flag)) { ok = false; break; }
+                const bool live = (w.tile != w.n_b - 1) || (w.tile * kTile + t < w.L);
+                const uint32_t src = stages + st * C::STAGE_BYTES + C::KV_TILE_BYTES + t * 128;
+                const uint32_t dst = vc_base + c * C::VC_BYTES + hf * C::PANEL_BYTES + t * 128;
+#pragma unroll
+                for (int jj = 0; jj < 4; ++jj) {
+                    const int ch = 4 * hf + jj;
+                    uint4 v = ld_shared_v4(src + ((ch ^ (t & 7)) << 4));
+                    uint4 o0, o1;
+                    o0.x = e4m3x2_to_f16x2_raw(v.x & 0xffffu);
+                    o0.y = e4m3x2_to_f16x2_raw(v.x >> 16);
+                    o0.z = e4m3x2_to_f16x2_raw(v.y & 0xffffu);
+                    o0.w = e4m3x2_to_f16x2_raw(v.y >> 16);
+                    o1.x = e4m3x2_to_f16x2_raw(v.z & 0xffffu);
+                    o1.y = e4m3x2_to_f16x2_raw(v.z >> 16);
+                    o1.z = e4m3x2_to_f16x2_raw(v.w & 0xffffu);
+                    o1.w = e4m3x2_to_f16x2_raw(v.w >> 16);
+                    if (!live) o0 = o1 = make_uint4(0, 0, 0, 0);
+                    st_shared_v4(dst + (((2 * jj) ^ (t & 7)) << 4), o0.x, o0.y, o0.z, o0.w);
+                    st_shared_v4(dst + (((2 * jj + 1) ^ (t & 7)) << 4), o1.x, o1.y, o1.z, o1.w);
+                }
+                fence_async_smem_writes();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->vcfull[c]));
+                if (++st == NS) { st = 0; ph ^= 1u; }
+                if (gi + 1 < hi) w.advance(a);
+            }
+            if (!ok) fail();
+        }
+    }
+
+    if (lo < hi && warp >= C::WARP_SM0 && warp < C::WARP_SM0 + C::NSM) {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int sp = warp & 3;            // tensor-memory sub-partition of this warp
+        const int tok = 16 * sp + lane;     // S^T row held by this thread (lanes 0..15)
+        const bool row_lane = lane < 16;
+        const float NEG_INF = -__int_as_float(0x7f800000);
+        constexpr float PSCALE = KV8 ? 128.f : 1.f;  // keeps f16 weights normal
+        float m[RP], l[RP];
+        uint32_t xpar = 0, qph = 0;
+        int qs = 0, qcur = 0, seg = -1, seg_start_tile = 0, st = 0;
+        float vfac = 1.f, qf_uniform = a.sl2;
+        bool ok = true;
+
+        auto exchange = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->xch));
+            const bool r = mbar_wait_warp(smem_addr(&ctrl->xch), xpar, abort_flag);
+            xpar ^= 1u;
+            return r;
+        };
+
+        int j = 0;
+        for (int64_t gi = lo; gi < hi; ++gi, ++j) {
+            const bool seg_first = (gi == lo) || (w.tile == 0);
+            const bool last_tile = (w.tile == w.n_b - 1);
+            const bool seg_last = (gi == hi - 1) || last_tile;
+            if (seg_first) {
+                ++seg;
+                seg_start_tile = w.tile;
+                qcur = qs;
+                const uint32_t qpar = qph;  // phase of this use of slot qcur
+                (void)qpar;
+                if (++qs == 2) { qs = 0; qph ^= 1u; }
+#pragma unroll
+                for (int h = 0; h < RP; ++h) {
+                    m[h] = NEG_INF;
+                    l[h] = 0.f;
+                }
+                if constexpr (KV8) {
+                    vfac = __ldg(a.v_scale + w.kv) * (1.f / PSCALE);
+                    qf_uniform = a.sl2 * __ldg(a.k_scale + w.kv);
+                    if (!mbar_wait_warp(smem_addr(&ctrl->qfull[qcur]), qpar, abort_flag)) { ok = false; break; }
+                    if (!mbar_wait_warp(smem_addr(&ctrl->qtempty[qcur]), qpar ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    // Query head hh -> two E4M3 terms (rows hh and RP + hh of the term slot).
+                    const uint32_t qsrc = q_base + qcur * C::QSLOT_BYTES;
+                    const uint32_t qdst = qt_base + qcur * C::QT_BYTES;
+                    const int d0 = 4 * lane;
+                    for (int hh = sp; hh < RP; hh += 4) {
+                        const int pnl = d0 >> 6, ch = (d0 & 63) >> 3;
+                        const uint2 wq = ld_shared_v2(qsrc + pnl * C::QPANEL_BYTES + hh * 128 +
+                                                      ((ch ^ (hh & 7)) << 4) + ((d0 & 7) << 1));
+                        float q[4];
+                        q[0] = __uint_as_float(wq.x << 16);
+                        q[1] = __uint_as_float(wq.x & 0xffff0000u);
+                        q[2] = __uint_as_float(wq.y << 16);
+                        q[3] = __uint_as_float(wq.y & 0xffff0000u);
+                        if (hh >= a.R) q[0] = q[1] = q[2] = q[3] = 0.f;
+                        float mx = fmaxf(fmaxf(fabsf(q[0]), fabsf(q[1])), fmaxf(fabsf(q[2]), fabsf(q[3])));
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                        // 2^a with max |q| 2^a in [128, 256)
+                        int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+                        int sa = mx > 0.f ? 7 - e : 0;
+                        sa = sa > 120 ? 120 : (sa < -120 ? -120 : sa);
+                        const float up = __uint_as_float(static_cast<uint32_t>(sa + 127) << 23);
+                        const float down = __uint_as_float(static_cast<uint32_t>(127 - sa) << 23);
+                        float x[4], r[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) x[i] = q[i] * up;
+                        const uint16_t t1a = f32x2_to_e4m3x2(x[0], x[1]);
+                        const uint16_t t1b = f32x2_to_e4m3x2(x[2], x[3]);
+                        const float2 b1a = e4m3x2_to_f32x2(t1a), b1b = e4m3x2_to_f32x2(t1b);
+                        r[0] = (x[0] - b1a.x) * 16.f;
+                        r[1] = (x[1] - b1a.y) * 16.f;
+                        r[2] = (x[2] - b1b.x) * 16.f;
+                        r[3] = (x[3] - b1b.y) * 16.f;
+                        const uint16_t t2a = f32x2_to_e4m3x2(r[0], r[1]);
+                        const uint16_t t2b = f32x2_to_e4m3x2(r[2], r[3]);
+                        const int row2 = RP + hh;
+                        const uint32_t a1 = qdst + hh * 128 + (((d0 >> 4) ^ (hh & 7)) << 4) + (d0 & 15);
+                        const uint32_t a2 = qdst + row2 * 128 + (((d0 >> 4) ^ (row2 & 7)) << 4) + (d0 & 15);
+                        st_shared_u32(a1, static_cast<uint32_t>(t1a) | (static_cast<uint32_t>(t1b) << 16));
+                        st_shared_u32(a2, static_cast<uint32_t>(t2a) | (static_cast<uint32_t>(t2b) << 16));
+                        if (lane == 0) X->qscale[qcur][hh] = mx > 0.f ? down : 0.f;
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&ctrl->qempty[qcur]));  // bf16 query slot read
+                    fence_async_smem_writes();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&ctrl->qtfull[qcur]));
+                    if (!exchange()) { ok = false; break; }  // every head's 2^-a is in place
+                }
+            }
+            const int b = j & 1;
+            const uint32_t bpar = static_cast<uint32_t>(j >> 1) & 1u;
+            const int t0 = w.tile * kTile;
+            const bool valid = row_lane && (t0 + tok < w.L);
+
+            // ---- scores of this thread's token
+            if (!mbar_wait_warp(smem_addr(&ctrl->sfull[b]), bpar, abort_flag)) { ok = false; break; }
+            tc::fence_after_sync();
+            float s[RP];
+            {
+                const uint32_t ta = tc::tmem_addr(tmem, 32 * sp, C::S_COL + b * C::NS_COLS);
+                if constexpr (RP == 8 && !KV8) {
+                    uint32_t r[8];
+                    tc::tmem_ld8(ta, r);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) s[h] = __uint_as_float(r[h]) * qf_uniform;
+                } else if constexpr (!KV8) {
+#pragma unroll
+                    for (int c = 0; c < RP / 16; ++c) {
+                        uint32_t r[16];
+                        tc::tmem_ld16(ta + 16 * c, r);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(r[i]) * qf_uniform;
+                    }
+                } else {
+                    // columns h (term 1) and RP + h (term 2), 8 heads at a time
+#pragma unroll
+                    for (int c = 0; c < RP / 8; ++c) {
+                        uint32_t r1[8], r2[8];
+                        tc::tmem_ld8(ta + 8 * c, r1);
+                        tc::tmem_ld8(ta + RP + 8 * c, r2);
+                        tc::tmem_wait_ld();
+                        const float4 qa = *reinterpret_cast<const float4*>(&X->qscale[qcur][8 * c]);
+                        const float4 qb = *reinterpret_cast<const float4*>(&X->qscale[qcur][8 * c + 4]);
+                        const float qsc[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            s[8 * c + i] = (__uint_as_float(r1[i]) + __uint_as_float(r2[i]) * 0.0625f) *
+                                           (qf_uniform * qsc[i]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < RP; ++h)
+                if (!valid || h >= a.R) s[h] = NEG_INF;
+
+            // ---- reference check: does any score exceed its head's reference by more than T?
+            bool exceed = false;
+#pragma unroll
+            for (int h = 0; h < RP; ++h) exceed |= s[h] > m[h] + static_cast<float>(C::T_LAZY);
+            {
+                const uint32_t xb = xpar;
+                const bool any = __any_sync(0xffffffffu, exceed);
+                if (lane == 0) X->flags[xb][sp] = any ? 1 : 0;
+                if (!exchange()) { ok = false; break; }
+                const bool slow = (X->flags[xb][0] | X->flags[xb][1] | X->flags[xb][2] | X->flags[xb][3]) != 0;
+                if (slow) {
+                    float mx[RP];
+#pragma unroll
+                    for (int h = 0; h < RP; ++h) {
+                        float v = s[h];
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
+                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+                        mx[h] = v;
+                    }
+                    const uint32_t xb2 = xpar;
+                    if (lane == 0) {
+#pragma unroll
+                        for (int h = 0; h < RP; h += 4)
+                            *reinterpret_cast<float4*>(&X->vals[xb2][sp][h]) =
+                                make_float4(mx[h], mx[h + 1], mx[h + 2], mx[h + 3]);
+                    }
+                    if (!exchange()) { ok = false; break; }
+                    float alpha[RP];
+                    bool moved = false;
+#pragma unroll
+                    for (int h = 0; h < RP; ++h) {
+                        const float M = fmaxf(fmaxf(X->vals[xb2][0][h], X->vals[xb2][1][h]),
+                                              fmaxf(X->vals[xb2][2][h], X->vals[xb2][3][h]));
+                        alpha[h] = 1.f;
+                        if (M > m[h] + static_cast<float>(C::T_LAZY)) {
+                            alpha[h] = m[h] == NEG_INF ? 0.f : fast_exp2(m[h] - M);
+                            moved |= m[h] != NEG_INF;
+                            m[h] = M;
+                        }
+                        l[h] *= alpha[h];
+                    }
+                    if (moved && w.tile != seg_start_tile) {
+                        // O^T holds this segment's earlier tiles: rescale it in place once
+                        // the previous tile's value product has landed.
+                        if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[(j - 1) & 1]),
+                                            static_cast<uint32_t>((j - 1) >> 1) & 1u, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc::fence_after_sync();
+#pragma unroll
+                        for (int c = 0; c < C::NO_COLS / 8; ++c) {
+                            const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + 8 * c);
+                            uint32_t r[8];
+                            tc::tmem_ld8(oa, r);
+                            tc::tmem_wait_ld();
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha[(8 * c + e) % RP]);
+                            tc::tmem_st8(oa, r);
+                        }
+                        tc::tmem_wait_st();
+                    }
+                }
+            }
+
+            // ---- weights, row sums, P^T (hi | lo) for the value product
+            float p[RP];
+#pragma unroll
+            for (int h = 0; h < RP; ++h) {
+                const float ref = m[h] == NEG_INF ? 0.f : m[h];
+                p[h] = fast_exp2(s[h] - ref);
+                l[h] += p[h];
+            }
+            if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[b]), bpar ^ 1u, abort_flag)) { ok = false; break; }
+            if (row_lane) {
+                const uint32_t pt = p_base + b * C::P_BYTES + (tok >> 3) * 128 + (tok & 7) * 16;
+#pragma unroll
+                for (int g = 0; g < RP / 8; ++g) {
+                    uint32_t hw[4], lw[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        split_pair<KV8>(p[8 * g + 2 * e] * PSCALE, p[8 * g + 2 * e + 1] * PSCALE, hw[e], lw[e]);
+                    st_shared_v4(pt + g * 1024, hw[0], hw[1], hw[2], hw[3]);
+                    st_shared_v4(pt + (g + RP / 8) * 1024, lw[0], lw[1], lw[2], lw[3]);
+                }
+            }
+            if constexpr (!KV8) {
+                // Value rows past L_b may hold anything; 0 * NaN would poison O^T.
+                if (last_tile && row_lane && !valid) {
+                    const uint32_t vrow = stages + st * C::STAGE_BYTES + C::KV_TILE_BYTES + tok * 128;
+#pragma unroll
+                    for (int pnl = 0; pnl < 2; ++pnl)
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) st_shared_v4(vrow + pnl * C::PANEL_BYTES + 16 * c, 0u, 0u, 0u, 0u);
+                }
+            }
+            fence_async_smem_writes();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull[b]));
+
+            if (seg_last) {
+                // ---------------------------------------------------- segment end
+                float lt[RP];
+#pragma unroll
+                for (int h = 0; h < RP; ++h) {
+                    float v = l[h];
+                    v += __shfl_xor_sync(0xffffffffu, v, 8);
+                    v += __shfl_xor_sync(0xffffffffu, v, 4);
+                    v += __shfl_xor_sync(0xffffffffu, v, 2);
+                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+                    lt[h] = v;
+                }
+                const uint32_t xb3 = xpar;
+                if (lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < RP; h += 4)
+                        *reinterpret_cast<float4*>(&X->vals[xb3][sp][h]) =
+                            make_float4(lt[h], lt[h + 1], lt[h + 2], lt[h + 3]);
+                }
+                if (!exchange()) { ok = false; break; }
+#pragma unroll
+                for (int h = 0; h < RP; ++h)
+                    lt[h] = (X->vals[xb3][0][h] + X->vals[xb3][1][h]) + (X->vals[xb3][2][h] + X->vals[xb3][3][h]);
+                if (!mbar_wait_warp(smem_addr(&ctrl->ofull), static_cast<uint32_t>(seg) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const int d = 32 * sp + lane;
+                const bool whole = (seg_start_tile == 0) && last_tile;
+                const int64_t slot = 2 * static_cast<int64_t>(blockIdx.x) + (seg == 0 ? 0 : 1);
+#pragma unroll
+                for (int c = 0; c < RP / 8; ++c) {
+                    uint32_t hv[8], lv[8];
+                    tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + 8 * c), hv);
+                    tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + RP + 8 * c), lv);
+                    tc::tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int h = 8 * c + e;
+                        if (h >= a.R) continue;
+                        const float o = (__uint_as_float(hv[e]) + __uint_as_float(lv[e])) * (vfac / lt[h]);
+                        if (whole) {
+                            const int64_t i = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + h) * C::D + d;
+                            if constexpr (OUT_BF16)
+                                static_cast<__nv_bfloat16*>(a.out)[i] = __float2bfloat16_rn(o);
+                            else
+                                static_cast<float*>(a.out)[i] = o;
+                        } else {
+                            a.ws_o[(slot * a.R + h) * C::D + d] = o;
+                        }
+                    }
+                }
+                if (!whole && sp == 0 && lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < RP; ++h)
+                        if (h < a.R) a.ws_lse[slot * a.R + h] = m[h] + log2f(lt[h]);
+                }
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree));
+            }
+            if (++st == NS) st = 0;
+            if (gi + 1 < hi) w.advance(a);
+        }
+        if (!ok) fail();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == C::WARP_QK) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gqa

@@ -23,10 +23,12 @@ def run_fp8(inp, w, dev, paged=False, out_dtype=torch.float32):
     d = to_device(inp, dev)
     k = d["k_paged"] if paged else d["k"]
     v = d["v_paged"] if paged else d["v"]
-    out = gq.gqa_decode_fp8kv(d["q"], k, v, d["k_scale"], d["v_scale"], d["seq_lens"],
-                              d["block_table"] if paged else None, scale=w.softmax_scale,
-                              out_dtype=out_dtype)
-    torch.cuda.synchronize(dev)
+    table = d["block_table"] if paged else None
+    params = gq.make_params(d["q"], k, d["seq_lens"], table, out_dtype)
+    ws = gq.make_workspace(params, dev)
+    out = gq.gqa_decode_fp8kv(d["q"], k, v, d["k_scale"], d["v_scale"], d["seq_lens"], table,
+                              scale=w.softmax_scale, out_dtype=out_dtype, workspace=ws)
+    assert gq.read_status(ws) & gq.FLAG_TIMEOUT == 0, "a pipeline wait timed out"
     return out.cpu()
 
 

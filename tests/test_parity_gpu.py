@@ -23,12 +23,11 @@ pytestmark = pytest.mark.gpu
 def run_gpu(inp, w, dev, paged=False, out_dtype=torch.float32, seq_lens=None):
     d = to_device(inp, dev)
     lens = d["seq_lens"] if seq_lens is None else seq_lens.to(dev)
-    if paged:
-        out = gq.gqa_decode(d["q"], d["k_paged"], d["v_paged"], lens, d["block_table"],
-                            scale=w.softmax_scale, out_dtype=out_dtype)
-    else:
-        out = gq.gqa_decode(d["q"], d["k"], d["v"], lens, scale=w.softmax_scale, out_dtype=out_dtype)
-    torch.cuda.synchronize(dev)
+    k, v = (d["k_paged"], d["v_paged"]) if paged else (d["k"], d["v"])
+    table = d["block_table"] if paged else None
+    ws = gq.make_workspace(gq.make_params(d["q"], k, lens, table, out_dtype), dev)
+    out = gq.gqa_decode(d["q"], k, v, lens, table, scale=w.softmax_scale, out_dtype=out_dtype, workspace=ws)
+    assert gq.read_status(ws) & gq.FLAG_TIMEOUT == 0, "a pipeline wait timed out"
     return out.cpu()
 
 
