@@ -32,6 +32,8 @@ __all__ = [
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libgqa_decode.so")
 PAGE_SIZE = 64
 GQA_BF16, GQA_F32 = 0, 1
+# gqa_kernel: which split kernel serves a call (all compute the same result)
+KERNELS = {"auto": 0, "mma_sync": 1, "tcgen05": 2}
 FLAG_SEQ_LEN_CLAMPED, FLAG_BAD_BLOCK, FLAG_TIMEOUT, FLAG_BAD_POSITION = 1, 2, 4, 8
 ROPE_PAIRING = {"adjacent": 0, "halves": 1}
 
@@ -56,6 +58,7 @@ class Params(ctypes.Structure):
         ("head_dim", ctypes.c_int32), ("max_seq_len", ctypes.c_int32),
         ("page_size", ctypes.c_int32), ("max_blocks_per_seq", ctypes.c_int32),
         ("num_blocks", ctypes.c_int32), ("qkv_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int),
+        ("kernel", ctypes.c_int32),
     ]
 
     def key(self):
@@ -123,7 +126,8 @@ def _dtype_code(dtype) -> int:
     raise TypeError(f"unsupported dtype {dtype}: use torch.bfloat16 or torch.float32")
 
 
-def make_params(q, k_cache, seq_lens, block_table=None, out_dtype=None, max_seq_len=None) -> Params:
+def make_params(q, k_cache, seq_lens, block_table=None, out_dtype=None, max_seq_len=None,
+                kernel="auto") -> Params:
     """Fill gqa_decode_params from tensor shapes (no device work)."""
     import torch
 
@@ -152,6 +156,9 @@ def make_params(q, k_cache, seq_lens, block_table=None, out_dtype=None, max_seq_
                          else int(max_seq_len))
     p.qkv_dtype = _dtype_code(q.dtype)
     p.out_dtype = _dtype_code(torch.float32 if out_dtype is None else out_dtype)
+    if kernel not in KERNELS:
+        raise ValueError(f"kernel must be one of {sorted(KERNELS)}")
+    p.kernel = KERNELS[kernel]
     return p
 
 
@@ -199,12 +206,12 @@ def _check_inputs(q, k_cache, v_cache, seq_lens, block_table):
 
 
 def _call(q, k_cache, v_cache, seq_lens, block_table, scale, out, out_dtype, workspace, stream,
-          events, max_seq_len):
+          events, max_seq_len, kernel="auto"):
     import torch
 
     _check_inputs(q, k_cache, v_cache, seq_lens, block_table)
     params = make_params(q, k_cache, seq_lens, block_table, out_dtype if out is None else out.dtype,
-                         max_seq_len)
+                         max_seq_len, kernel)
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or torch.float32, device=q.device)
     elif out.shape != q.shape or not out.is_contiguous() or not out.is_cuda:
@@ -236,7 +243,7 @@ def _call(q, k_cache, v_cache, seq_lens, block_table, scale, out, out_dtype, wor
 
 
 def gqa_decode(q, k_cache, v_cache, seq_lens, block_table=None, scale=None, out=None,
-               out_dtype=None, workspace=None, stream=None, max_seq_len=None):
+               out_dtype=None, workspace=None, stream=None, max_seq_len=None, kernel="auto"):
     """One GQA decode step on the GPU.
 
     q            [B, H_Q, D] bf16 or f32 (CUDA)
@@ -246,17 +253,19 @@ def gqa_decode(q, k_cache, v_cache, seq_lens, block_table=None, scale=None, out=
     block_table  int32 [B, max_blocks_per_seq] for a paged cache
     scale        softmax scale (default 1/sqrt(D))
     out          optional [B, H_Q, D] output (f32 default, or bf16)
+    kernel       "auto", "mma_sync" or "tcgen05" (gqa_kernel)
     Returns out.  Enqueued on ``stream`` (default: the current stream); no sync.
     """
     return _call(q, k_cache, v_cache, seq_lens, block_table, scale, out, out_dtype, workspace,
-                 stream, None, max_seq_len)
+                 stream, None, max_seq_len, kernel)
 
 
 def gqa_decode_timed(events, q, k_cache, v_cache, seq_lens, block_table=None, scale=None,
-                     out=None, out_dtype=None, workspace=None, stream=None, max_seq_len=None):
+                     out=None, out_dtype=None, workspace=None, stream=None, max_seq_len=None,
+                     kernel="auto"):
     """gqa_decode with torch.cuda.Event pair ``events`` recorded around the split kernel."""
     return _call(q, k_cache, v_cache, seq_lens, block_table, scale, out, out_dtype, workspace,
-                 stream, events, max_seq_len)
+                 stream, events, max_seq_len, kernel)
 
 
 def gqa_decode_static_workspace(q, k_cache, v_cache, seq_lens, block_table=None, scale=None,
@@ -333,7 +342,7 @@ def gqa_rope_append(q, k_new, v_new, positions, k_cache, v_cache, block_table=No
 
 def gqa_decode_fp8kv(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_table=None,
                      scale=None, out=None, out_dtype=None, workspace=None, stream=None,
-                     max_seq_len=None):
+                     max_seq_len=None, kernel="auto"):
     """gqa_decode over an 8-bit cache: k_cache, v_cache hold E4M3 values
     (torch.float8_e4m3fn or their uint8 bytes) multiplied by per-KV-head
     k_scale, v_scale (float32 [H_KV]).  q is bf16."""
@@ -356,7 +365,7 @@ def gqa_decode_fp8kv(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_tabl
     if seq_lens.dtype != torch.int32 or seq_lens.shape != (q.shape[0],):
         raise ValueError("seq_lens must be int32 [B]")
     params = make_params(q, k_cache, seq_lens, block_table, out_dtype if out is None else out.dtype,
-                         max_seq_len)
+                         max_seq_len, kernel)
     params.qkv_dtype = GQA_BF16
     if out is None:
         out = torch.empty(q.shape, dtype=out_dtype or torch.float32, device=q.device)

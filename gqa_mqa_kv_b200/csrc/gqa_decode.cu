@@ -63,6 +63,7 @@ gqa_status validate_params(const gqa_decode_params* p) {
     if (p->H_Q % p->H_KV != 0) return GQA_ERR_INVALID;
     if (p->qkv_dtype != GQA_BF16 && p->qkv_dtype != GQA_F32) return GQA_ERR_INVALID;
     if (p->out_dtype != GQA_BF16 && p->out_dtype != GQA_F32) return GQA_ERR_INVALID;
+    if (p->kernel < GQA_KERNEL_AUTO || p->kernel > GQA_KERNEL_TCGEN05) return GQA_ERR_INVALID;
     if (p->page_size != 0 && p->page_size != kTile) return GQA_ERR_UNSUPPORTED;
     if (p->head_dim != 64 && p->head_dim != 128) return GQA_ERR_UNSUPPORTED;
     if (p->page_size == 0) {
@@ -77,12 +78,24 @@ gqa_status validate_params(const gqa_decode_params* p) {
     return GQA_OK;
 }
 
-bool use_tensor_cores(const gqa_decode_params* p) {
-    return p->qkv_dtype == GQA_BF16 && p->H_Q / p->H_KV <= 64;
+enum class SplitKernel { kMmaSync, kTcgen05, kSimt, kNone };
+
+// Which split kernel serves a problem (gqa_kernel in the header).
+SplitKernel select_kernel(const gqa_decode_params* p, bool kv8) {
+    const int R = p->H_Q / p->H_KV;
+    const bool tc_ok = p->head_dim == 128 && R <= 32 && p->qkv_dtype == GQA_BF16;
+    const bool mma_ok = p->qkv_dtype == GQA_BF16 && (kv8 ? (p->head_dim == 128 && R <= 8) : R <= 64);
+    switch (p->kernel) {
+        case GQA_KERNEL_TCGEN05: return tc_ok ? SplitKernel::kTcgen05 : SplitKernel::kNone;
+        case GQA_KERNEL_MMA_SYNC: return mma_ok ? SplitKernel::kMmaSync : SplitKernel::kNone;
+        default:
+            if (kv8) return tc_ok ? SplitKernel::kTcgen05 : SplitKernel::kSimt;
+            return mma_ok ? SplitKernel::kMmaSync : SplitKernel::kSimt;
+    }
 }
 
-int grid_for(const gqa_decode_params* p, const DeviceInfo& dev) {
-    return use_tensor_cores(p) ? dev.sms : dev.sms * kSimtCtasPerSm;
+int grid_for(const gqa_decode_params* p, const DeviceInfo& dev, bool kv8 = false) {
+    return select_kernel(p, kv8) == SplitKernel::kSimt && !kv8 ? dev.sms * kSimtCtasPerSm : dev.sms;
 }
 
 size_t workspace_for(const gqa_decode_params* p, int grid) {
@@ -286,18 +299,10 @@ template <bool PAGED, bool OUTB, bool KV8>
 cudaError_t launch_tc_groups(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
                              const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
     const int R = p->H_Q / p->H_KV;
-    if (R <= 8) return launch_tc<8, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
+    if constexpr (KV8)
+        if (R <= 8) return launch_tc<8, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
     if (R <= 16) return launch_tc<16, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
     return launch_tc<32, PAGED, OUTB, KV8>(p, buf, args, dev, grid, stream, encode_ok);
-}
-
-// Which split kernel serves a problem: the tcgen05 kernel for head_dim 128
-// with an 8-bit cache (R <= 32) or a bf16 cache with 8 < R <= 32; the
-// mma.sync kernel for the other bf16 groups up to 64; CUDA cores otherwise.
-bool use_tc(const gqa_decode_params* p, bool kv8) {
-    const int R = p->H_Q / p->H_KV;
-    if (p->head_dim != 128 || R > 32) return false;
-    return kv8 || (p->qkv_dtype == GQA_BF16 && R > 8);
 }
 
 template <typename TQ, typename TKV, int D, bool PAGED, bool OUTB>
@@ -310,14 +315,16 @@ cudaError_t launch_simt(const Buffers& buf, const KernelArgs& args, int grid, cu
 template <int D, bool PAGED, bool OUTB>
 cudaError_t launch_split(const gqa_decode_params* p, const Buffers& buf, const KernelArgs& args,
                          const DeviceInfo& dev, int grid, cudaStream_t stream, bool* encode_ok) {
+    const SplitKernel k = select_kernel(p, buf.kv8);
     if constexpr (D == 128) {
-        if (use_tc(p, buf.kv8)) {
+        if (k == SplitKernel::kTcgen05)
             return buf.kv8 ? launch_tc_groups<PAGED, OUTB, true>(p, buf, args, dev, grid, stream, encode_ok)
                            : launch_tc_groups<PAGED, OUTB, false>(p, buf, args, dev, grid, stream, encode_ok);
-        }
+        if (k == SplitKernel::kMmaSync && buf.kv8)
+            return launch_mma<128, 1, 1, PAGED, OUTB, true>(p, buf, args, dev, grid, stream, encode_ok);
     }
+    if (k == SplitKernel::kMmaSync) return launch_mma_groups<D, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (buf.kv8) return launch_simt<__nv_bfloat16, __nv_fp8_e4m3, D, PAGED, OUTB>(buf, args, grid, stream);
-    if (use_tensor_cores(p)) return launch_mma_groups<D, PAGED, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (p->qkv_dtype == GQA_F32) return launch_simt<float, float, D, PAGED, OUTB>(buf, args, grid, stream);
     return launch_simt<__nv_bfloat16, __nv_bfloat16, D, PAGED, OUTB>(buf, args, grid, stream);
 }
@@ -344,6 +351,7 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
     const bool kv8 = k_scale != nullptr;
     gqa_status st = validate_params(p);
     if (st != GQA_OK) return st;
+    if (select_kernel(p, kv8) == SplitKernel::kNone) return GQA_ERR_UNSUPPORTED;
     if (p->B == 0) return GQA_OK;
     if (!q || !k || !v || !seq_lens || !out) return GQA_ERR_INVALID;
     if ((p->page_size != 0) != (block_table != nullptr)) return GQA_ERR_INVALID;

@@ -9,21 +9,21 @@
 // a whole-unit segment writes the output, others write (normalised o,
 // log2-sum-exp) partials for the combine kernel.
 //
-// Per 64-token tile:
-//   S^T = K Q^T     tcgen05.mma, M = 64 tokens, N = query columns, K = d:
-//                   A = the K tile as TMA staged it (K-major, 128-byte
+// A step covers two consecutive 64-token tiles of one segment (one, zero
+// padded, when the segment's tile count is odd):
+//   S^T = K Q^T     tcgen05.mma, M = 128 tokens, N = query columns, K = d:
+//                   A = the K rows as TMA staged them (K-major, 128-byte
 //                   swizzle), B = the query rows; S^T lands in tensor memory
-//                   (two buffers, so the next tile's product overlaps this
-//                   tile's softmax).
-//   softmax         four warps; thread = token (row of S^T): p = 2^(s - m)
+//                   (two buffers, so the next step's product overlaps this
+//                   step's softmax).
+//   softmax         four warps, thread = token = TMEM lane: p = 2^(s - m)
 //                   against a per-head reference m shared by all tokens,
-//                   moved only when a score exceeds it by more than 8
-//                   (all threads agree through an mbarrier exchange).
-//                   P^T is written to shared memory as bf16 (or f16) hi and
-//                   lo parts -- N = 2 * RP columns -- so the product keeps
-//                   fp32-level precision of the weights.
-//   O^T += V^T P^T  tcgen05.mma, M = 128 (d), N = 2 RP, K = 64 tokens:
-//                   A = the V tile read MN-major, B = P^T; O^T accumulates in
+//                   moved only when a score exceeds it by more than 8 (all
+//                   threads agree through an mbarrier exchange).  P^T goes
+//                   to shared memory as bf16 (or f16) hi and lo parts -- N =
+//                   2 RP columns -- so the product keeps fp32-level weights.
+//   O^T += V^T P^T  tcgen05.mma, M = 128 (d), N = 2 RP, K = 128 tokens:
+//                   A = the V rows read MN-major, B = P^T; O^T accumulates in
 //                   tensor memory over the segment; hi and lo columns are
 //                   summed in the epilogue.
 //
@@ -33,14 +33,14 @@
 // split into two E4M3 terms, q 2^a = t1 + t2 / 16 (exact for every element
 // of magnitude >= 2^-6 after scaling; smaller ones err by <= 2^-14), held as
 // query columns h and RP + h; s = (S[h] + S[RP + h] / 16) 2^-a.  Four
-// converter warps widen each V tile to f16 (exact) for a kind::f16 value
+// converter warps widen each V step to f16 (exact) for a kind::f16 value
 // product; P is scaled by 2^7 so its f16 hi/lo parts stay normal.
 //
 // Warp roles: 0 TMA producer, 1 score products (+ tensor-memory
 // allocation), 2 value products, 3..6 softmax and epilogue (sub-partitions
-// 3, 0, 1, 2), 7..10 V converters (KV8).  Every wait is bounded (kWaitTimeoutNs); on a timeout the CTA raises
-// GQA_FLAG_TIMEOUT, lets its copies and products drain, frees its tensor
-// memory and returns.
+// 3, 0, 1, 2), 7..10 V converters (KV8).  Every wait is bounded
+// (kWaitTimeoutNs); on a timeout the CTA raises GQA_FLAG_TIMEOUT, lets its
+// copies and products drain, frees its tensor memory and returns.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -53,9 +53,13 @@
 
 namespace gqa {
 
+constexpr int kStepTiles = 2;                 // 64-token tiles per step
+constexpr int kStepTokens = kStepTiles * kTile;
+
 template <int RP, bool KV8>
 struct TcCfg {
     static_assert(RP == 8 || RP == 16 || RP == 32, "query columns per KV head: 8, 16 or 32");
+    static_assert(KV8 || RP >= 16, "an M = 128 score product needs N >= 16");
     static constexpr int D = 128;
     static constexpr int NS_COLS = KV8 ? 2 * RP : RP;  // S^T columns: heads, or two query terms per head
     static constexpr int NO_COLS = 2 * RP;             // O^T columns: P hi | P lo
@@ -66,22 +70,28 @@ struct TcCfg {
     static constexpr int NCV = KV8 ? 4 : 0;            // converter warps
     static constexpr int WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3, WARP_CV0 = 3 + NSM;
     static constexpr int THREADS = 32 * (3 + NSM + NCV);
-    static constexpr int KV_TILE_BYTES = KV8 ? kTile * D : kTile * D * 2;  // one of K, V
-    static constexpr int STAGE_BYTES = 2 * KV_TILE_BYTES;
-    static constexpr int PANEL_BYTES = kTile * 128;    // bf16 tile panel: 64 tokens x 64 d
+    static constexpr int HALF_BYTES = kTile * 128;     // one 64-row TMA box of 128-byte rows
+    static constexpr int PANEL_BYTES = kStepTokens * 128;  // 128 token rows x 128 bytes
+    static constexpr int KV_BYTES = KV8 ? PANEL_BYTES : 2 * PANEL_BYTES;  // one of K, V for a step
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
     static constexpr int QPANEL_BYTES = RP * 128;      // bf16 query panel: RP rows x 64 d
     static constexpr int QSLOT_BYTES = 2 * QPANEL_BYTES;
     static constexpr int QT_BYTES = KV8 ? NS_COLS * 128 : 0;  // E4M3 query terms: 2 RP rows x 128 d
-    static constexpr int P_BYTES = (NO_COLS / 8) * 1024;      // P^T: 8-column groups x 8 token groups x 128 B
-    static constexpr int VC_BYTES = KV8 ? kTile * D * 2 : 0;  // f16 V tile (two 64-d panels)
+    static constexpr int P_BYTES = (NO_COLS / 8) * (kStepTokens / 8) * 128;  // core matrices 8 tokens x 16 B
+    static constexpr int P_SBO = (kStepTokens / 8) * 128;     // next 8 P^T columns
+    static constexpr int VC_BYTES = KV8 ? 2 * PANEL_BYTES : 0; // f16 V rows (two 64-d panels)
+    // Buffer counts: the largest bf16 group keeps one query slot and one
+    // P^T buffer so three 64 KB stages still fit in shared memory.
+    static constexpr int NQ = (!KV8 && RP == 32) ? 1 : 2;
+    static constexpr int NP = (!KV8 && RP == 32) ? 1 : 2;
     static constexpr int NVC = KV8 ? 2 : 0;
-    static constexpr int MAX_STAGES = 12;
+    static constexpr int MAX_STAGES = 8;
     static constexpr int T_LAZY = 8;                   // reference slack, base 2
     // fixed region after the stage ring; every piece 1024-aligned
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_QT = OFF_Q + 2 * QSLOT_BYTES;
-    static constexpr int OFF_P = OFF_QT + 2 * QT_BYTES;
-    static constexpr int OFF_VC = OFF_P + 2 * P_BYTES;
+    static constexpr int OFF_QT = OFF_Q + NQ * QSLOT_BYTES;
+    static constexpr int OFF_P = OFF_QT + NQ * QT_BYTES;
+    static constexpr int OFF_VC = OFF_P + NP * P_BYTES;
     static constexpr int OFF_X = OFF_VC + NVC * VC_BYTES;       // exchange scratch
     static constexpr int X_BYTES = 2 * NSM * 32 * 4 + 2 * 32 * 4 + 2 * NSM * 4;
     static constexpr int OFF_CTRL = OFF_X + ((X_BYTES + 1023) / 1024) * 1024;
@@ -91,13 +101,13 @@ struct TcCfg {
 };
 
 struct __align__(16) TcControl {
-    uint64_t full[12], empty[12];   // stage ring
+    uint64_t full[8], empty[8];     // stage ring
     uint64_t qfull[2], qempty[2];   // bf16 query slots (TMA)
     uint64_t qtfull[2], qtempty[2]; // E4M3 query terms (KV8)
-    uint64_t sfull[2];              // S^T buffer b written
-    uint64_t pfull[2];              // P^T buffer b written (tile j uses b = j & 1)
-    uint64_t vcfull[2];             // converted V buffer b written (KV8)
-    uint64_t pvdone[2];             // value product of the last tile using buffer b completed
+    uint64_t sfull[2], sfree[2];    // S^T buffer b written / read by the softmax warps
+    uint64_t pfull[2];              // P^T buffer written
+    uint64_t vcfull[2];             // converted V buffer written (KV8)
+    uint64_t pvdone[2];             // value product of the last step using P^T buffer b completed
     uint64_t ofull, ofree;          // O^T of a segment complete / read by the epilogue
     uint64_t xch;                   // softmax-warp exchange (count 4)
     uint64_t drain[2];              // final completion of each issuing warp's products
@@ -108,10 +118,31 @@ struct __align__(16) TcControl {
 
 // Scratch for the softmax warps' exchanges (double-buffered by exchange parity).
 struct TcExchange {
-    float vals[2][4][32];  // per warp, per head: tile maxima or row sums
+    float vals[2][4][32];  // per warp, per head: step maxima or row sums
     float qscale[2][32];   // KV8: 2^-a per head, per query-term slot
     int flags[2][4];
 };
+
+// One step of a CTA's walk: tiles [tile, tile + n) of the current unit.
+struct Step {
+    int n;
+    bool seg_first, seg_last;
+};
+
+__device__ __forceinline__ Step step_at(const Walk& w, int64_t gi, int64_t lo, int64_t hi) {
+    Step s;
+    s.n = (gi + 1 < hi && w.tile + 1 < w.n_b) ? 2 : 1;
+    s.seg_first = (gi == lo) || (w.tile == 0);
+    s.seg_last = (gi + s.n == hi) || (w.tile + s.n == w.n_b);
+    return s;
+}
+
+__device__ __forceinline__ void advance_step(Walk& w, const KernelArgs& a, int64_t& gi, int n, int64_t hi) {
+    for (int i = 0; i < n; ++i) {
+        if (gi + 1 < hi) w.advance(a);
+        ++gi;
+    }
+}
 
 __device__ __forceinline__ void st_shared_u32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
@@ -163,8 +194,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     using C = TcCfg<RP, KV8>;
     static_assert(sizeof(TcControl) <= C::CTRL_BYTES, "control block overflows its slot");
     static_assert(sizeof(TcExchange) <= C::X_BYTES, "exchange scratch overflows its slot");
-    constexpr uint32_t IDESC_QK = KV8 ? tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, 0, 0, 64, C::NS_COLS)
-                                      : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 64, C::NS_COLS);
+    constexpr uint32_t IDESC_QK = KV8 ? tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, 0, 0, 128, C::NS_COLS)
+                                      : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 128, C::NS_COLS);
     constexpr uint32_t IDESC_PV = KV8 ? tc::instr_desc(tc::kFmtF16, tc::kFmtF16, 1, 1, 128, C::NO_COLS)
                                       : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 1, 1, 128, C::NO_COLS);
 
@@ -203,6 +234,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             mbar_init(smem_addr(&ctrl->qtfull[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->qtempty[s]), 1);
             mbar_init(smem_addr(&ctrl->sfull[s]), 1);
+            mbar_init(smem_addr(&ctrl->sfree[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->pfull[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->vcfull[s]), KV8 ? C::NCV : 1);
             mbar_init(smem_addr(&ctrl->pvdone[s]), 1);
@@ -215,8 +247,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     }
     // Query rows past H_Q come back from TMA as zeros; the P^T buffers start
     // zeroed so their padding columns are finite.
-    for (int i = threadIdx.x; i < (2 * C::QSLOT_BYTES + 2 * C::QT_BYTES + 2 * C::P_BYTES) / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(fixed_ptr + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < C::OFF_VC / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(fixed_ptr)[i] = make_uint4(0, 0, 0, 0);
 
     grid_dependency_wait();
     grid_launch_dependents();
@@ -247,11 +279,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         int st = 0, qs = 0;
         uint32_t ph = 0, qph = 0;
         int64_t issued = 0, q_issued = 0;
-        int page_word = 0, page_base = -1;
         bool ok = true;
-        for (int64_t gi = lo; gi < hi; ++gi) {
-            const bool seg_first = (gi == lo) || (w.tile == 0);
-            if (seg_first) {
+        for (int64_t gi = lo; gi < hi;) {
+            const Step sp = step_at(w, gi, lo, hi);
+            if (sp.seg_first) {
                 if (!mbar_wait_warp(smem_addr(&ctrl->qempty[qs]), qph ^ 1u, abort_flag)) { ok = false; break; }
                 if (lane == 0) {
                     const uint32_t bar = smem_addr(&ctrl->qfull[qs]);
@@ -261,45 +292,50 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                                     w.kv * a.R, w.b, pol_q);
                 }
                 ++q_issued;
-                if (++qs == 2) { qs = 0; qph ^= 1u; }
+                if (++qs == C::NQ) { qs = 0; qph ^= 1u; }
             }
-            int c2, c3;
-            if constexpr (PAGED) {
-                const int tb = w.tile & ~31;
-                if (seg_first || tb != page_base) {
-                    page_base = tb;
-                    const int idx = tb + lane;
-                    page_word = idx < w.n_b
-                                    ? __ldg(a.block_table + static_cast<int64_t>(w.b) * a.max_blocks + idx)
-                                    : 0;
+            // Box coordinates of the step's two tiles; a missing second tile
+            // is read from outside the tensor, which fills it with zeros.
+            int c2[2], c3[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                if constexpr (PAGED) {
+                    int page = a.num_blocks;
+                    if (h < sp.n) {
+                        page = __ldg(a.block_table + static_cast<int64_t>(w.b) * a.max_blocks + w.tile + h);
+                        if ((page < 0 || page >= a.num_blocks) && lane == 0) atomicOr(a.status, kFlagBadBlock);
+                    }
+                    c2[h] = 0;
+                    c3[h] = page;  // out of range: the TMA unit fills the tile with zeros
+                } else {
+                    c2[h] = h < sp.n ? (w.tile + h) * kTile : a.S_max;
+                    c3[h] = w.b;
                 }
-                const int page = __shfl_sync(0xffffffffu, page_word, w.tile & 31);
-                if ((page < 0 || page >= a.num_blocks) && lane == 0) atomicOr(a.status, kFlagBadBlock);
-                c2 = 0;
-                c3 = page;  // out of range: the TMA unit fills the tile with zeros
-            } else {
-                c2 = w.tile * kTile;
-                c3 = w.b;
             }
             if (!mbar_wait_warp(smem_addr(&ctrl->empty[st]), ph ^ 1u, abort_flag)) { ok = false; break; }
             if (lane == 0) {
                 const uint32_t bar = smem_addr(&ctrl->full[st]);
                 const uint32_t kb = stages + st * C::STAGE_BYTES;
-                const uint32_t vb = kb + C::KV_TILE_BYTES;
+                const uint32_t vb = kb + C::KV_BYTES;
                 mbar_arrive_expect_tx(bar, C::STAGE_BYTES);
-                if constexpr (KV8) {
-                    tma_load_4d(kb, &tmK, bar, 0, w.kv, c2, c3, pol_kv);
-                    tma_load_4d(vb, &tmV, bar, 0, w.kv, c2, c3, pol_kv);
-                } else {
-                    for (int p = 0; p < 2; ++p) {
-                        tma_load_4d(kb + p * C::PANEL_BYTES, &tmK, bar, 64 * p, w.kv, c2, c3, pol_kv);
-                        tma_load_4d(vb + p * C::PANEL_BYTES, &tmV, bar, 64 * p, w.kv, c2, c3, pol_kv);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    if constexpr (KV8) {
+                        tma_load_4d(kb + h * C::HALF_BYTES, &tmK, bar, 0, w.kv, c2[h], c3[h], pol_kv);
+                        tma_load_4d(vb + h * C::HALF_BYTES, &tmV, bar, 0, w.kv, c2[h], c3[h], pol_kv);
+                    } else {
+                        for (int p = 0; p < 2; ++p) {
+                            tma_load_4d(kb + p * C::PANEL_BYTES + h * C::HALF_BYTES, &tmK, bar, 64 * p, w.kv,
+                                        c2[h], c3[h], pol_kv);
+                            tma_load_4d(vb + p * C::PANEL_BYTES + h * C::HALF_BYTES, &tmV, bar, 64 * p, w.kv,
+                                        c2[h], c3[h], pol_kv);
+                        }
                     }
                 }
             }
             ++issued;
             if (++st == NS) { st = 0; ph ^= 1u; }
-            if (gi + 1 < hi) w.advance(a);
+            advance_step(w, a, gi, sp.n, hi);
         }
         if (!ok) {
             fail();
@@ -307,38 +343,37 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             const int64_t first = issued > NS ? issued - NS : 0;
             for (int64_t i = first; i < issued; ++i)
                 mbar_wait(smem_addr(&ctrl->full[i % NS]), static_cast<uint32_t>((i / NS) & 1), nullptr);
-            const int64_t qfirst = q_issued > 2 ? q_issued - 2 : 0;
+            const int64_t qfirst = q_issued > C::NQ ? q_issued - C::NQ : 0;
             for (int64_t i = qfirst; i < q_issued; ++i)
-                mbar_wait(smem_addr(&ctrl->qfull[i % 2]), static_cast<uint32_t>((i / 2) & 1), nullptr);
+                mbar_wait(smem_addr(&ctrl->qfull[i % C::NQ]), static_cast<uint32_t>((i / C::NQ) & 1), nullptr);
         }
     }
 
     if (warp == C::WARP_QK) {
         // ------------------------------------------------------------ score products
-        // Tile j: S^T(j) = K(j) Q^T into buffer b = j & 1, once the softmax
-        // warps are done with the tile that used b before (j - 2).
+        // Step j: S^T(j) = K(j) Q^T into buffer j & 1 once the softmax warps
+        // have read that buffer's previous contents (step j - 2).
         int st = 0, qs = 0, qcur = 0;
         uint32_t ph = 0, qph = 0;
         bool ok = true;
         if (lo < hi) {
             int j = 0;
-            for (int64_t gi = lo; gi < hi; ++gi, ++j) {
-                const bool seg_first = (gi == lo) || (w.tile == 0);
-                const bool seg_last = (gi == hi - 1) || (w.tile == w.n_b - 1);
-                const int b = j & 1;
-                const uint32_t bpar = static_cast<uint32_t>(j >> 1) & 1u;
-                if (seg_first) {
+            for (int64_t gi = lo; gi < hi; ++j) {
+                const Step sp = step_at(w, gi, lo, hi);
+                const int sb = j & 1;
+                const uint32_t spar = static_cast<uint32_t>(j >> 1) & 1u;
+                if (sp.seg_first) {
                     const uint32_t qbar = KV8 ? smem_addr(&ctrl->qtfull[qs]) : smem_addr(&ctrl->qfull[qs]);
                     if (!mbar_wait_warp(qbar, qph, abort_flag)) { ok = false; break; }
                     qcur = qs;
-                    if (++qs == 2) { qs = 0; qph ^= 1u; }
+                    if (++qs == C::NQ) { qs = 0; qph ^= 1u; }
                 }
-                if (!mbar_wait_warp(smem_addr(&ctrl->pfull[b]), bpar ^ 1u, abort_flag)) { ok = false; break; }
+                if (!mbar_wait_warp(smem_addr(&ctrl->sfree[sb]), spar ^ 1u, abort_flag)) { ok = false; break; }
                 if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { ok = false; break; }
                 tc::fence_after_sync();
                 if (tc::elect_one()) {
                     const uint32_t kt = stages + st * C::STAGE_BYTES;
-                    const uint32_t sd = tmem + C::S_COL + b * C::NS_COLS;
+                    const uint32_t sd = tmem + C::S_COL + sb * C::NS_COLS;
                     if constexpr (KV8) {
                         const uint32_t qt = qt_base + qcur * C::QT_BYTES;
 #pragma unroll
@@ -358,13 +393,13 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                             tc::mma_f16(sd, da, db, IDESC_QK, k > 0);
                         }
                     }
-                    tc::commit(smem_addr(&ctrl->sfull[b]));
-                    if (seg_last)  // the segment's query slot is free once its last score product is done
+                    tc::commit(smem_addr(&ctrl->sfull[sb]));
+                    if (sp.seg_last)  // the segment's query slot is free once its last score product is done
                         tc::commit(KV8 ? smem_addr(&ctrl->qtempty[qcur]) : smem_addr(&ctrl->qempty[qcur]));
                 }
                 __syncwarp();
                 if (++st == NS) { st = 0; ph ^= 1u; }
-                if (gi + 1 < hi) w.advance(a);
+                advance_step(w, a, gi, sp.n, hi);
             }
             if (!ok) fail();
         }
@@ -376,45 +411,49 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 
     if (warp == C::WARP_PV) {
         // ------------------------------------------------------------ value products
-        // Tile j: O^T += V^T(j) P^T(j) once the softmax warps have written P^T(j)
-        // (and, KV8, the converters the f16 V tile); a segment's first tile
+        // Step j: O^T += V^T(j) P^T(j) once the softmax warps have written P^T(j)
+        // (and, KV8, the converters the f16 V rows); a segment's first step
         // overwrites O^T after the epilogue has read the previous segment's.
         int st = 0, seg = -1;
         bool ok = true;
         if (lo < hi) {
             int j = 0;
-            for (int64_t gi = lo; gi < hi; ++gi, ++j) {
-                const bool seg_first = (gi == lo) || (w.tile == 0);
-                const bool seg_last = (gi == hi - 1) || (w.tile == w.n_b - 1);
-                const int b = j & 1;
-                const uint32_t bpar = static_cast<uint32_t>(j >> 1) & 1u;
-                if (seg_first) ++seg;
-                if (!mbar_wait_warp(smem_addr(&ctrl->pfull[b]), bpar, abort_flag)) { ok = false; break; }
-                if constexpr (KV8)
-                    if (!mbar_wait_warp(smem_addr(&ctrl->vcfull[b]), bpar, abort_flag)) { ok = false; break; }
-                if (seg_first && seg > 0)
+            for (int64_t gi = lo; gi < hi; ++j) {
+                const Step sp = step_at(w, gi, lo, hi);
+                const int pb = j % C::NP;
+                const uint32_t ppar = static_cast<uint32_t>(j / C::NP) & 1u;
+                if (sp.seg_first) ++seg;
+                if (!mbar_wait_warp(smem_addr(&ctrl->pfull[pb]), ppar, abort_flag)) { ok = false; break; }
+                if constexpr (KV8) {
+                    if (!mbar_wait_warp(smem_addr(&ctrl->vcfull[j & 1]), static_cast<uint32_t>(j >> 1) & 1u,
+                                        abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                }
+                if (sp.seg_first && seg > 0)
                     if (!mbar_wait_warp(smem_addr(&ctrl->ofree), static_cast<uint32_t>(seg - 1) & 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
                 tc::fence_after_sync();
                 if (tc::elect_one()) {
-                    const uint32_t vt = KV8 ? vc_base + b * C::VC_BYTES
-                                            : stages + st * C::STAGE_BYTES + C::KV_TILE_BYTES;
-                    const uint32_t pt = p_base + b * C::P_BYTES;
+                    const uint32_t vt = KV8 ? vc_base + (j & 1) * C::VC_BYTES
+                                            : stages + st * C::STAGE_BYTES + C::KV_BYTES;
+                    const uint32_t pt = p_base + pb * C::P_BYTES;
 #pragma unroll
-                    for (int k = 0; k < kTile / 16; ++k) {
+                    for (int k = 0; k < kStepTokens / 16; ++k) {
                         const uint64_t da = tc::smem_desc(vt + k * 2048, C::PANEL_BYTES, 1024, tc::kLayoutSw128);
-                        const uint64_t db = tc::smem_desc(pt + k * 256, 128, 1024, tc::kLayoutNone);
-                        tc::mma_f16(tmem + C::O_COL, da, db, IDESC_PV, !(seg_first && k == 0));
+                        const uint64_t db = tc::smem_desc(pt + k * 256, 128, C::P_SBO, tc::kLayoutNone);
+                        tc::mma_f16(tmem + C::O_COL, da, db, IDESC_PV, !(sp.seg_first && k == 0));
                     }
                     tc::commit(smem_addr(&ctrl->empty[st]));
-                    tc::commit(smem_addr(&ctrl->pvdone[b]));
-                    if (seg_last) tc::commit(smem_addr(&ctrl->ofull));
+                    tc::commit(smem_addr(&ctrl->pvdone[pb]));
+                    if (sp.seg_last) tc::commit(smem_addr(&ctrl->ofull));
                 }
                 __syncwarp();
                 if (++st == NS) st = 0;
-                if (gi + 1 < hi) w.advance(a);
+                advance_step(w, a, gi, sp.n, hi);
             }
             if (!ok) fail();
         }
@@ -426,45 +465,51 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     if constexpr (KV8) {
         if (lo < hi && warp >= C::WARP_CV0) {
             // ------------------------------------------------------------ V converters
-            // Thread (t, hf): token row t, d half hf; E4M3 -> f16 (exact) into the
-            // bf16-style layout (two 64-d panels, 128-byte swizzle); rows past L_b
-            // are written as zeros so 0 * NaN cannot reach O^T.
-            const int ct = threadIdx.x - 32 * C::WARP_CV0;
-            const int t = ct >> 1, hf = ct & 1;
+            // Thread t: token row t of the step; E4M3 -> f16 (exact) into the
+            // bf16-style layout (two 64-d panels, 128-byte swizzle); rows past
+            // L_b, and the zero-filled half of a one-tile step, become zeros so
+            // 0 * NaN cannot reach O^T.
+            const int t = threadIdx.x - 32 * C::WARP_CV0;
             int st = 0;
             uint32_t ph = 0;
             bool ok = true;
             int j = 0;
-            for (int64_t gi = lo; gi < hi; ++gi, ++j) {
+            for (int64_t gi = lo; gi < hi; ++j) {
+                const Step sp = step_at(w, gi, lo, hi);
                 const int c = j & 1;
                 const uint32_t par = static_cast<uint32_t>(j >> 1) & 1u;
                 if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { ok = false; break; }
                 if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[c]), par ^ 1u, abort_flag)) { ok = false; break; }
-                const bool live = (w.tile != w.n_b - 1) || (w.tile * kTile + t < w.L);
-                const uint32_t src = stages + st * C::STAGE_BYTES + C::KV_TILE_BYTES + t * 128;
-                const uint32_t dst = vc_base + c * C::VC_BYTES + hf * C::PANEL_BYTES + t * 128;
+                const bool live = t < kTile * sp.n && w.tile * kTile + t < w.L;
+                const uint32_t src = stages + st * C::STAGE_BYTES + C::KV_BYTES + t * 128;
+                const uint32_t dst = vc_base + c * C::VC_BYTES + t * 128;
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj) {
-                    const int ch = 4 * hf + jj;
-                    uint4 v = ld_shared_v4(src + ((ch ^ (t & 7)) << 4));
-                    uint4 o0, o1;
-                    o0.x = e4m3x2_to_f16x2_raw(v.x & 0xffffu);
-                    o0.y = e4m3x2_to_f16x2_raw(v.x >> 16);
-                    o0.z = e4m3x2_to_f16x2_raw(v.y & 0xffffu);
-                    o0.w = e4m3x2_to_f16x2_raw(v.y >> 16);
-                    o1.x = e4m3x2_to_f16x2_raw(v.z & 0xffffu);
-                    o1.y = e4m3x2_to_f16x2_raw(v.z >> 16);
-                    o1.z = e4m3x2_to_f16x2_raw(v.w & 0xffffu);
-                    o1.w = e4m3x2_to_f16x2_raw(v.w >> 16);
-                    if (!live) o0 = o1 = make_uint4(0, 0, 0, 0);
-                    st_shared_v4(dst + (((2 * jj) ^ (t & 7)) << 4), o0.x, o0.y, o0.z, o0.w);
-                    st_shared_v4(dst + (((2 * jj + 1) ^ (t & 7)) << 4), o1.x, o1.y, o1.z, o1.w);
+                for (int ch = 0; ch < 8; ++ch) {
+                    const uint4 v = ld_shared_v4(src + ((ch ^ (t & 7)) << 4));
+                    uint32_t o[8];
+                    o[0] = e4m3x2_to_f16x2_raw(v.x & 0xffffu);
+                    o[1] = e4m3x2_to_f16x2_raw(v.x >> 16);
+                    o[2] = e4m3x2_to_f16x2_raw(v.y & 0xffffu);
+                    o[3] = e4m3x2_to_f16x2_raw(v.y >> 16);
+                    o[4] = e4m3x2_to_f16x2_raw(v.z & 0xffffu);
+                    o[5] = e4m3x2_to_f16x2_raw(v.z >> 16);
+                    o[6] = e4m3x2_to_f16x2_raw(v.w & 0xffffu);
+                    o[7] = e4m3x2_to_f16x2_raw(v.w >> 16);
+                    if (!live) {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) o[i] = 0u;
+                    }
+                    // d = 16 ch .. 16 ch + 15: panel ch / 4, f16 chunks 2 (ch % 4), 2 (ch % 4) + 1
+                    const uint32_t pd = dst + (ch >> 2) * C::PANEL_BYTES;
+                    const int c0 = 2 * (ch & 3);
+                    st_shared_v4(pd + ((c0 ^ (t & 7)) << 4), o[0], o[1], o[2], o[3]);
+                    st_shared_v4(pd + (((c0 + 1) ^ (t & 7)) << 4), o[4], o[5], o[6], o[7]);
                 }
                 fence_async_smem_writes();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->vcfull[c]));
                 if (++st == NS) { st = 0; ph ^= 1u; }
-                if (gi + 1 < hi) w.advance(a);
+                advance_step(w, a, gi, sp.n, hi);
             }
             if (!ok) fail();
         }
@@ -473,8 +518,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     if (lo < hi && warp >= C::WARP_SM0 && warp < C::WARP_SM0 + C::NSM) {
         // ------------------------------------------------------------ softmax + epilogue
         const int sp = warp & 3;            // tensor-memory sub-partition of this warp
-        const int tok = 16 * sp + lane;     // S^T row held by this thread (lanes 0..15)
-        const bool row_lane = lane < 16;
+        const int tok = 32 * sp + lane;     // S^T row (token of the step) held by this thread
         const float NEG_INF = -__int_as_float(0x7f800000);
         constexpr float PSCALE = KV8 ? 128.f : 1.f;  // keeps f16 weights normal
         float m[RP], l[RP];
@@ -492,17 +536,16 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         };
 
         int j = 0;
-        for (int64_t gi = lo; gi < hi; ++gi, ++j) {
-            const bool seg_first = (gi == lo) || (w.tile == 0);
-            const bool last_tile = (w.tile == w.n_b - 1);
-            const bool seg_last = (gi == hi - 1) || last_tile;
-            if (seg_first) {
+        for (int64_t gi = lo; gi < hi; ++j) {
+            const Step stp = step_at(w, gi, lo, hi);
+            const bool last_of_unit = (w.tile + stp.n == w.n_b);
+            if (stp.seg_first) {
                 ++seg;
                 seg_start_tile = w.tile;
                 qcur = qs;
                 const uint32_t qpar = qph;  // phase of this use of slot qcur
                 (void)qpar;
-                if (++qs == 2) { qs = 0; qph ^= 1u; }
+                if (++qs == C::NQ) { qs = 0; qph ^= 1u; }
 #pragma unroll
                 for (int h = 0; h < RP; ++h) {
                     m[h] = NEG_INF;
@@ -534,7 +577,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
                         // 2^a with max |q| 2^a in [128, 256)
-                        int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+                        const int e = static_cast<int>((__float_as_uint(mx) >> 23) & 0xffu) - 127;
                         int sa = mx > 0.f ? 7 - e : 0;
                         sa = sa > 120 ? 120 : (sa < -120 ? -120 : sa);
                         const float up = __uint_as_float(static_cast<uint32_t>(sa + 127) << 23);
@@ -566,24 +609,21 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     if (!exchange()) { ok = false; break; }  // every head's 2^-a is in place
                 }
             }
-            const int b = j & 1;
-            const uint32_t bpar = static_cast<uint32_t>(j >> 1) & 1u;
+            const int sb = j & 1;
+            const uint32_t spar = static_cast<uint32_t>(j >> 1) & 1u;
+            const int pb = j % C::NP;
+            const uint32_t ppar = static_cast<uint32_t>(j / C::NP) & 1u;
             const int t0 = w.tile * kTile;
-            const bool valid = row_lane && (t0 + tok < w.L);
+            const bool loaded = tok < kTile * stp.n;
+            const bool valid = loaded && (t0 + tok < w.L);
 
             // ---- scores of this thread's token
-            if (!mbar_wait_warp(smem_addr(&ctrl->sfull[b]), bpar, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(smem_addr(&ctrl->sfull[sb]), spar, abort_flag)) { ok = false; break; }
             tc::fence_after_sync();
             float s[RP];
             {
-                const uint32_t ta = tc::tmem_addr(tmem, 32 * sp, C::S_COL + b * C::NS_COLS);
-                if constexpr (RP == 8 && !KV8) {
-                    uint32_t r[8];
-                    tc::tmem_ld8(ta, r);
-                    tc::tmem_wait_ld();
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) s[h] = __uint_as_float(r[h]) * qf_uniform;
-                } else if constexpr (!KV8) {
+                const uint32_t ta = tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::NS_COLS);
+                if constexpr (!KV8) {
 #pragma unroll
                     for (int c = 0; c < RP / 16; ++c) {
                         uint32_t r[16];
@@ -610,6 +650,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     }
                 }
             }
+            // S^T buffer sb may take the step after next
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
 #pragma unroll
             for (int h = 0; h < RP; ++h)
                 if (!valid || h >= a.R) s[h] = NEG_INF;
@@ -629,10 +673,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 #pragma unroll
                     for (int h = 0; h < RP; ++h) {
                         float v = s[h];
-                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 8));
-                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 4));
-                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-                        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
+#pragma unroll
+                        for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
                         mx[h] = v;
                     }
                     const uint32_t xb2 = xpar;
@@ -658,10 +700,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         l[h] *= alpha[h];
                     }
                     if (moved && w.tile != seg_start_tile) {
-                        // O^T holds this segment's earlier tiles: rescale it in place once
-                        // the previous tile's value product has landed.
-                        if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[(j - 1) & 1]),
-                                            static_cast<uint32_t>((j - 1) >> 1) & 1u, abort_flag)) {
+                        // O^T holds this segment's earlier steps: rescale it in place once
+                        // the previous step's value product has landed.
+                        if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[(j - 1) % C::NP]),
+                                            static_cast<uint32_t>((j - 1) / C::NP) & 1u, abort_flag)) {
                             ok = false;
                             break;
                         }
@@ -690,23 +732,23 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 p[h] = fast_exp2(s[h] - ref);
                 l[h] += p[h];
             }
-            if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[b]), bpar ^ 1u, abort_flag)) { ok = false; break; }
-            if (row_lane) {
-                const uint32_t pt = p_base + b * C::P_BYTES + (tok >> 3) * 128 + (tok & 7) * 16;
+            if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[pb]), ppar ^ 1u, abort_flag)) { ok = false; break; }
+            {
+                const uint32_t pt = p_base + pb * C::P_BYTES + (tok >> 3) * 128 + (tok & 7) * 16;
 #pragma unroll
                 for (int g = 0; g < RP / 8; ++g) {
                     uint32_t hw[4], lw[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e)
                         split_pair<KV8>(p[8 * g + 2 * e] * PSCALE, p[8 * g + 2 * e + 1] * PSCALE, hw[e], lw[e]);
-                    st_shared_v4(pt + g * 1024, hw[0], hw[1], hw[2], hw[3]);
-                    st_shared_v4(pt + (g + RP / 8) * 1024, lw[0], lw[1], lw[2], lw[3]);
+                    st_shared_v4(pt + g * C::P_SBO, hw[0], hw[1], hw[2], hw[3]);
+                    st_shared_v4(pt + (g + RP / 8) * C::P_SBO, lw[0], lw[1], lw[2], lw[3]);
                 }
             }
             if constexpr (!KV8) {
-                // Value rows past L_b may hold anything; 0 * NaN would poison O^T.
-                if (last_tile && row_lane && !valid) {
-                    const uint32_t vrow = stages + st * C::STAGE_BYTES + C::KV_TILE_BYTES + tok * 128;
+                // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
+                if (last_of_unit && loaded && !valid) {
+                    const uint32_t vrow = stages + st * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
 #pragma unroll
                     for (int pnl = 0; pnl < 2; ++pnl)
 #pragma unroll
@@ -716,18 +758,16 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             fence_async_smem_writes();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull[b]));
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull[pb]));
 
-            if (seg_last) {
+            if (stp.seg_last) {
                 // ---------------------------------------------------- segment end
                 float lt[RP];
 #pragma unroll
                 for (int h = 0; h < RP; ++h) {
                     float v = l[h];
-                    v += __shfl_xor_sync(0xffffffffu, v, 8);
-                    v += __shfl_xor_sync(0xffffffffu, v, 4);
-                    v += __shfl_xor_sync(0xffffffffu, v, 2);
-                    v += __shfl_xor_sync(0xffffffffu, v, 1);
+#pragma unroll
+                    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
                     lt[h] = v;
                 }
                 const uint32_t xb3 = xpar;
@@ -747,7 +787,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 }
                 tc::fence_after_sync();
                 const int d = 32 * sp + lane;
-                const bool whole = (seg_start_tile == 0) && last_tile;
+                const bool whole = (seg_start_tile == 0) && last_of_unit;
                 const int64_t slot = 2 * static_cast<int64_t>(blockIdx.x) + (seg == 0 ? 0 : 1);
 #pragma unroll
                 for (int c = 0; c < RP / 8; ++c) {
@@ -781,7 +821,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree));
             }
             if (++st == NS) st = 0;
-            if (gi + 1 < hi) w.advance(a);
+            advance_step(w, a, gi, stp.n, hi);
         }
         if (!ok) fail();
     }

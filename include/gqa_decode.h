@@ -69,6 +69,16 @@ typedef enum gqa_rope_pairing {
     GQA_ROPE_HALVES = 1     /* (i, i + head_dim/2) */
 } gqa_rope_pairing;
 
+/* Which split kernel serves a call (both compute the same result). */
+typedef enum gqa_kernel {
+    GQA_KERNEL_AUTO = 0,     /* tcgen05 for 8-bit caches (head_dim 128, R <= 32), mma.sync for bf16
+                                (R <= 64), CUDA cores otherwise */
+    GQA_KERNEL_MMA_SYNC = 1, /* warp-level mma.sync kernel: bf16 cache with R <= 64, or an 8-bit
+                                cache with head_dim 128 and R <= 8 */
+    GQA_KERNEL_TCGEN05 = 2   /* tcgen05 / tensor-memory kernel: head_dim 128, R <= 32, bf16 query,
+                                bf16 or 8-bit cache */
+} gqa_kernel;
+
 /* Device status flags, accumulated (bitwise OR) in the workspace. */
 #define GQA_FLAG_SEQ_LEN_CLAMPED 1u   /* a seq_lens entry was < 0 or > max_seq_len */
 #define GQA_FLAG_BAD_BLOCK 2u         /* a live block_table entry was outside [0, num_blocks) */
@@ -90,6 +100,8 @@ typedef enum gqa_rope_pairing {
  *                   block table, and pages held by k_cache/v_cache.
  *  qkv_dtype        element type of q, k_cache and v_cache.
  *  out_dtype        element type of out.  F32 keeps the fp32 accumulator.
+ *  kernel           gqa_kernel; 0 (automatic) for normal use.  A kernel that
+ *                   cannot serve the problem gives GQA_ERR_UNSUPPORTED.
  */
 typedef struct gqa_decode_params {
     int32_t B;
@@ -102,6 +114,7 @@ typedef struct gqa_decode_params {
     int32_t num_blocks;
     gqa_dtype qkv_dtype;
     gqa_dtype out_dtype;
+    int32_t kernel;
 } gqa_decode_params;
 
 /*

@@ -99,6 +99,8 @@ def call_decode(lib, p, q=16, k=16, v=16, lens=16, table=None, out=16, ws=256, w
         (dict(page_size=64, max_blocks_per_seq=0, num_blocks=4), GQA_ERR_INVALID),
         (dict(page_size=64, max_blocks_per_seq=2, num_blocks=4, max_seq_len=129), GQA_ERR_INVALID),
         (dict(max_blocks_per_seq=3), GQA_ERR_INVALID),   # block fields on a contiguous cache
+        (dict(kernel=3), GQA_ERR_INVALID),               # no such gqa_kernel
+        (dict(kernel=-1), GQA_ERR_INVALID),
     ],
 )
 def test_invalid_params_rejected_on_host(lib, kw, expected):
@@ -119,6 +121,31 @@ def test_null_and_misaligned_pointers_rejected(lib):
     pp = params(page_size=64, max_blocks_per_seq=4, num_blocks=8)
     assert call_decode(lib, pp, table=None) == GQA_ERR_INVALID
     assert call_decode(lib, p, scale=float("nan")) == GQA_ERR_INVALID
+
+
+@pytest.mark.parametrize(
+    "kw",
+    [
+        dict(kernel=2, head_dim=64),                    # tcgen05 serves head_dim 128 only
+        dict(kernel=2, H_Q=64, H_KV=1),                 # R = 64 > 32
+        dict(kernel=2, qkv_dtype=1),                    # f32 cache: CUDA cores only
+        dict(kernel=1, qkv_dtype=1),
+        dict(kernel=1, H_Q=128, H_KV=1),                # R = 128 > 64
+    ],
+)
+def test_unsupported_kernel_choice_refused_on_host(lib, kw):
+    assert call_decode(lib, params(**kw)) == GQA_ERR_UNSUPPORTED
+
+
+def test_fp8_kernel_choice_limits(lib):
+    vp = ctypes.c_void_p
+
+    def call(p):
+        return lib.gqa_decode_fp8kv(ctypes.byref(p), vp(16), vp(16), vp(16), vp(64), vp(64), vp(16), vp(None),
+                                    ctypes.c_float(0.1), vp(16), vp(256), ctypes.c_size_t(1 << 20), vp(None))
+
+    assert call(params(kernel=1, H_Q=32, H_KV=2)) == GQA_ERR_UNSUPPORTED  # mma.sync 8-bit path: R <= 8
+    assert call(params(kernel=2, H_Q=128, H_KV=2)) == GQA_ERR_UNSUPPORTED  # tcgen05: R <= 32
 
 
 def test_empty_batch_is_a_no_op(lib):

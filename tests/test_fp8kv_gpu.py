@@ -19,7 +19,7 @@ from tests.helpers import assert_parity, to_device
 pytestmark = pytest.mark.gpu
 
 
-def run_fp8(inp, w, dev, paged=False, out_dtype=torch.float32):
+def run_fp8(inp, w, dev, paged=False, out_dtype=torch.float32, kernel="auto"):
     d = to_device(inp, dev)
     k = d["k_paged"] if paged else d["k"]
     v = d["v_paged"] if paged else d["v"]
@@ -27,7 +27,7 @@ def run_fp8(inp, w, dev, paged=False, out_dtype=torch.float32):
     params = gq.make_params(d["q"], k, d["seq_lens"], table, out_dtype)
     ws = gq.make_workspace(params, dev)
     out = gq.gqa_decode_fp8kv(d["q"], k, v, d["k_scale"], d["v_scale"], d["seq_lens"], table,
-                              scale=w.softmax_scale, out_dtype=out_dtype, workspace=ws)
+                              scale=w.softmax_scale, out_dtype=out_dtype, workspace=ws, kernel=kernel)
     assert gq.read_status(ws) & gq.FLAG_TIMEOUT == 0, "a pipeline wait timed out"
     return out.cpu()
 

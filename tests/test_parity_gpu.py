@@ -20,13 +20,14 @@ from tests.helpers import assert_parity, to_device
 pytestmark = pytest.mark.gpu
 
 
-def run_gpu(inp, w, dev, paged=False, out_dtype=torch.float32, seq_lens=None):
+def run_gpu(inp, w, dev, paged=False, out_dtype=torch.float32, seq_lens=None, kernel="auto"):
     d = to_device(inp, dev)
     lens = d["seq_lens"] if seq_lens is None else seq_lens.to(dev)
     k, v = (d["k_paged"], d["v_paged"]) if paged else (d["k"], d["v"])
     table = d["block_table"] if paged else None
     ws = gq.make_workspace(gq.make_params(d["q"], k, lens, table, out_dtype), dev)
-    out = gq.gqa_decode(d["q"], k, v, lens, table, scale=w.softmax_scale, out_dtype=out_dtype, workspace=ws)
+    out = gq.gqa_decode(d["q"], k, v, lens, table, scale=w.softmax_scale, out_dtype=out_dtype, workspace=ws,
+                        kernel=kernel)
     assert gq.read_status(ws) & gq.FLAG_TIMEOUT == 0, "a pipeline wait timed out"
     return out.cpu()
 
