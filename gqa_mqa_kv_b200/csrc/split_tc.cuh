@@ -33,8 +33,9 @@
 // split into two E4M3 terms, q 2^a = t1 + t2 / 16 (exact for every element
 // of magnitude >= 2^-6 after scaling; smaller ones err by <= 2^-14), held as
 // query columns h and RP + h; s = (S[h] + S[RP + h] / 16) 2^-a.  Four
-// converter warps widen each V step to f16 (exact) for a kind::f16 value
-// product; P is scaled by 2^7 so its f16 hi/lo parts stay normal.
+// converter warps widen each V step to f16 by bit placement (value * 2^-8,
+// exact) for a kind::f16 value product; P is scaled by 2^7 so its f16 hi/lo
+// parts stay normal.
 //
 // Warp roles: 0 TMA producer, 1 score products (+ tensor-memory
 // allocation), 2 value products, 3..6 softmax and epilogue (sub-partitions
@@ -164,11 +165,6 @@ __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint16_t v) {
     return make_float2(__half2float(__ushort_as_half(h.x)), __half2float(__ushort_as_half(h.y)));
 }
 
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2_raw(uint32_t two_bytes) {
-    const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two_bytes), __NV_E4M3);
-    return static_cast<uint32_t>(h.x) | (static_cast<uint32_t>(h.y) << 16);
-}
-
 // hi + lo split of two weights into the operand type of the value product.
 template <bool F16>
 __device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
@@ -226,7 +222,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_addr(&ctrl->full[s]), 1);
-            mbar_init(smem_addr(&ctrl->empty[s]), 1);
+            // bf16: freed by the value product; KV8: by the score product and the converters
+            mbar_init(smem_addr(&ctrl->empty[s]), KV8 ? 1 + C::NCV : 1);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->qfull[s]), 1);
@@ -394,6 +391,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         }
                     }
                     tc::commit(smem_addr(&ctrl->sfull[sb]));
+                    if constexpr (KV8) tc::commit(smem_addr(&ctrl->empty[st]));  // keys read; converters arrive too
                     if (sp.seg_last)  // the segment's query slot is free once its last score product is done
                         tc::commit(KV8 ? smem_addr(&ctrl->qtempty[qcur]) : smem_addr(&ctrl->qempty[qcur]));
                 }
@@ -447,7 +445,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         const uint64_t db = tc::smem_desc(pt + k * 256, 128, C::P_SBO, tc::kLayoutNone);
                         tc::mma_f16(tmem + C::O_COL, da, db, IDESC_PV, !(sp.seg_first && k == 0));
                     }
-                    tc::commit(smem_addr(&ctrl->empty[st]));
+                    if constexpr (!KV8) tc::commit(smem_addr(&ctrl->empty[st]));
                     tc::commit(smem_addr(&ctrl->pvdone[pb]));
                     if (sp.seg_last) tc::commit(smem_addr(&ctrl->ofull));
                 }
@@ -465,10 +463,12 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     if constexpr (KV8) {
         if (lo < hi && warp >= C::WARP_CV0) {
             // ------------------------------------------------------------ V converters
-            // Thread t: token row t of the step; E4M3 -> f16 (exact) into the
-            // bf16-style layout (two 64-d panels, 128-byte swizzle); rows past
-            // L_b, and the zero-filled half of a one-tile step, become zeros so
-            // 0 * NaN cannot reach O^T.
+            // Thread t: token row t of the step; E4M3 -> f16 holding value * 2^-8
+            // (exact, by bit placement) into the bf16-style layout (two 64-d
+            // panels, 128-byte swizzle).  Within each group of four, d is stored
+            // in the order 4i, 4i+2, 4i+1, 4i+3 (undone when O^T is written).
+            // Rows past L_b, and the zero-filled half of a one-tile step, become
+            // zeros so 0 * NaN cannot reach O^T.
             const int t = threadIdx.x - 32 * C::WARP_CV0;
             int st = 0;
             uint32_t ph = 0;
@@ -487,14 +487,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 for (int ch = 0; ch < 8; ++ch) {
                     const uint4 v = ld_shared_v4(src + ((ch ^ (t & 7)) << 4));
                     uint32_t o[8];
-                    o[0] = e4m3x2_to_f16x2_raw(v.x & 0xffffu);
-                    o[1] = e4m3x2_to_f16x2_raw(v.x >> 16);
-                    o[2] = e4m3x2_to_f16x2_raw(v.y & 0xffffu);
-                    o[3] = e4m3x2_to_f16x2_raw(v.y >> 16);
-                    o[4] = e4m3x2_to_f16x2_raw(v.z & 0xffffu);
-                    o[5] = e4m3x2_to_f16x2_raw(v.z >> 16);
-                    o[6] = e4m3x2_to_f16x2_raw(v.w & 0xffffu);
-                    o[7] = e4m3x2_to_f16x2_raw(v.w >> 16);
+                    e4m3x4_to_f16x2_scaled(v.x, o[0], o[1]);
+                    e4m3x4_to_f16x2_scaled(v.y, o[2], o[3]);
+                    e4m3x4_to_f16x2_scaled(v.z, o[4], o[5]);
+                    e4m3x4_to_f16x2_scaled(v.w, o[6], o[7]);
                     if (!live) {
 #pragma unroll
                         for (int i = 0; i < 8; ++i) o[i] = 0u;
@@ -507,7 +503,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 }
                 fence_async_smem_writes();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&ctrl->vcfull[c]));
+                if (lane == 0) {
+                    mbar_arrive(smem_addr(&ctrl->vcfull[c]));
+                    mbar_arrive(smem_addr(&ctrl->empty[st]));  // this warp is done reading the stage
+                }
                 if (++st == NS) { st = 0; ph ^= 1u; }
                 advance_step(w, a, gi, sp.n, hi);
             }
@@ -552,7 +551,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     l[h] = 0.f;
                 }
                 if constexpr (KV8) {
-                    vfac = __ldg(a.v_scale + w.kv) * (1.f / PSCALE);
+                    vfac = __ldg(a.v_scale + w.kv) * (256.f / PSCALE);  // values were decoded as v * 2^-8
                     qf_uniform = a.sl2 * __ldg(a.k_scale + w.kv);
                     if (!mbar_wait_warp(smem_addr(&ctrl->qfull[qcur]), qpar, abort_flag)) { ok = false; break; }
                     if (!mbar_wait_warp(smem_addr(&ctrl->qtempty[qcur]), qpar ^ 1u, abort_flag)) {
@@ -659,14 +658,27 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 if (!valid || h >= a.R) s[h] = NEG_INF;
 
             // ---- reference check: does any score exceed its head's reference by more than T?
+            // The flags go out first; the weights against the current reference are
+            // computed while the other warps' flags arrive, and recomputed only when
+            // some warp found an excess (normally the first step of a segment).
             bool exceed = false;
 #pragma unroll
             for (int h = 0; h < RP; ++h) exceed |= s[h] > m[h] + static_cast<float>(C::T_LAZY);
+            float p[RP];
             {
                 const uint32_t xb = xpar;
                 const bool any = __any_sync(0xffffffffu, exceed);
                 if (lane == 0) X->flags[xb][sp] = any ? 1 : 0;
-                if (!exchange()) { ok = false; break; }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->xch));
+#pragma unroll
+                for (int h = 0; h < RP; ++h) {
+                    const float ref = m[h] == NEG_INF ? 0.f : m[h];
+                    p[h] = fast_exp2(s[h] - ref);
+                }
+                const bool xok = mbar_wait_warp(smem_addr(&ctrl->xch), xpar, abort_flag);
+                xpar ^= 1u;
+                if (!xok) { ok = false; break; }
                 const bool slow = (X->flags[xb][0] | X->flags[xb][1] | X->flags[xb][2] | X->flags[xb][3]) != 0;
                 if (slow) {
                     float mx[RP];
@@ -698,6 +710,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                             m[h] = M;
                         }
                         l[h] *= alpha[h];
+                        const float ref = m[h] == NEG_INF ? 0.f : m[h];
+                        p[h] = fast_exp2(s[h] - ref);
                     }
                     if (moved && w.tile != seg_start_tile) {
                         // O^T holds this segment's earlier steps: rescale it in place once
@@ -724,14 +738,9 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 }
             }
 
-            // ---- weights, row sums, P^T (hi | lo) for the value product
-            float p[RP];
+            // ---- row sums, P^T (hi | lo) for the value product
 #pragma unroll
-            for (int h = 0; h < RP; ++h) {
-                const float ref = m[h] == NEG_INF ? 0.f : m[h];
-                p[h] = fast_exp2(s[h] - ref);
-                l[h] += p[h];
-            }
+            for (int h = 0; h < RP; ++h) l[h] += p[h];
             if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[pb]), ppar ^ 1u, abort_flag)) { ok = false; break; }
             {
                 const uint32_t pt = p_base + pb * C::P_BYTES + (tok >> 3) * 128 + (tok & 7) * 16;
@@ -786,7 +795,9 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                const int d = 32 * sp + lane;
+                // O^T row 32 sp + lane; 8-bit values were stored with d order (0, 2, 1, 3) in each 4
+                const int drow = 32 * sp + lane;
+                const int d = KV8 ? (drow & ~3) | ((drow & 1) << 1) | ((drow >> 1) & 1) : drow;
                 const bool whole = (seg_start_tile == 0) && last_of_unit;
                 const int64_t slot = 2 * static_cast<int64_t>(blockIdx.x) + (seg == 0 ? 0 : 1);
 #pragma unroll
