@@ -20,8 +20,8 @@
 //                   against a per-head reference m shared by all tokens,
 //                   moved only when a score exceeds it by more than 8 (all
 //                   threads agree through an mbarrier exchange).  P^T goes
-//                   to shared memory as bf16 (or f16) hi and lo parts -- N =
-//                   2 RP columns -- so the product keeps fp32-level weights.
+//                   to shared memory as bf16 hi and lo parts -- N = 2 RP
+//                   columns -- so the product keeps fp32-level weights.
 //   O^T += V^T P^T  tcgen05.mma, M = 128 (d), N = 2 RP, K = 128 tokens:
 //                   A = the V rows read MN-major, B = P^T; O^T accumulates in
 //                   tensor memory over the segment; hi and lo columns are
@@ -32,14 +32,16 @@
 // head is scaled by a power of two 2^a (max |q| * 2^a in [128, 256)) and
 // split into two E4M3 terms, q 2^a = t1 + t2 / 16 (exact for every element
 // of magnitude >= 2^-6 after scaling; smaller ones err by <= 2^-14), held as
-// query columns h and RP + h; s = (S[h] + S[RP + h] / 16) 2^-a.  Four
-// converter warps widen each V step to f16 by bit placement (value * 2^-8,
-// exact) for a kind::f16 value product; P is scaled by 2^7 so its f16 hi/lo
-// parts stay normal.
+// query columns h and RP + h; s = (S[h] + S[RP + h] / 16) 2^-a.  The value
+// product is kind::f8f6f4 as well, on the staged E4M3 value rows read
+// MN-major, with each weight split into four E4M3 terms, p = t1 + t2 / 16 +
+// t3 / 256 + t4 / 4096 (relative error <= 2^-16 for p >= 2^-6, absolute
+// <= 2^-22 below), held as O^T columns [t1 | t2 | t3 | t4] and summed in
+// the epilogue.
 //
 // Warp roles: 0 TMA producer, 1 score products (+ tensor-memory
 // allocation), 2 value products, 3..6 softmax and epilogue (sub-partitions
-// 3, 0, 1, 2), 7..10 V converters (KV8).  Every wait is bounded
+// 3, 0, 1, 2).  Every wait is bounded
 // (kWaitTimeoutNs); on a timeout the CTA raises GQA_FLAG_TIMEOUT, lets its
 // copies and products drain, frees its tensor memory and returns.
 #pragma once
@@ -63,14 +65,15 @@ struct TcCfg {
     static_assert(KV8 || RP >= 16, "an M = 128 score product needs N >= 16");
     static constexpr int D = 128;
     static constexpr int NS_COLS = KV8 ? 2 * RP : RP;  // S^T columns: heads, or two query terms per head
-    static constexpr int NO_COLS = 2 * RP;             // O^T columns: P hi | P lo
+    // O^T columns: bf16 P hi | lo, or four E4M3 terms of P (KV8), each RP heads wide
+    static constexpr int NPT = KV8 ? 4 : 2;            // P terms
+    static constexpr int NO_COLS = NPT * RP;
     static constexpr int S_COL = 0;                    // S^T buffer b at S_COL + b * NS_COLS
     static constexpr int O_COL = 2 * NS_COLS;
     static constexpr int TMEM_COLS = 512;              // the whole tensor memory of the SM
     static constexpr int NSM = 4;                      // softmax warps
-    static constexpr int NCV = KV8 ? 4 : 0;            // converter warps
-    static constexpr int WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3, WARP_CV0 = 3 + NSM;
-    static constexpr int THREADS = 32 * (3 + NSM + NCV);
+    static constexpr int WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
+    static constexpr int THREADS = 32 * (3 + NSM);
     static constexpr int HALF_BYTES = kTile * 128;     // one 64-row TMA box of 128-byte rows
     static constexpr int PANEL_BYTES = kStepTokens * 128;  // 128 token rows x 128 bytes
     static constexpr int KV_BYTES = KV8 ? PANEL_BYTES : 2 * PANEL_BYTES;  // one of K, V for a step
@@ -78,22 +81,21 @@ struct TcCfg {
     static constexpr int QPANEL_BYTES = RP * 128;      // bf16 query panel: RP rows x 64 d
     static constexpr int QSLOT_BYTES = 2 * QPANEL_BYTES;
     static constexpr int QT_BYTES = KV8 ? NS_COLS * 128 : 0;  // E4M3 query terms: 2 RP rows x 128 d
-    static constexpr int P_BYTES = (NO_COLS / 8) * (kStepTokens / 8) * 128;  // core matrices 8 tokens x 16 B
-    static constexpr int P_SBO = (kStepTokens / 8) * 128;     // next 8 P^T columns
-    static constexpr int VC_BYTES = KV8 ? 2 * PANEL_BYTES : 0; // f16 V rows (two 64-d panels)
+    // P^T: core matrices of 8 tokens x 16 bytes (8 bf16 or 16 E4M3 columns)
+    static constexpr int P_COLS_PER_CORE = KV8 ? 16 : 8;
+    static constexpr int P_SBO = (kStepTokens / 8) * 128;     // next 16-byte column group
+    static constexpr int P_BYTES = (NO_COLS / P_COLS_PER_CORE) * P_SBO;
     // Buffer counts: the largest bf16 group keeps one query slot and one
     // P^T buffer so three 64 KB stages still fit in shared memory.
     static constexpr int NQ = (!KV8 && RP == 32) ? 1 : 2;
     static constexpr int NP = (!KV8 && RP == 32) ? 1 : 2;
-    static constexpr int NVC = KV8 ? 2 : 0;
     static constexpr int MAX_STAGES = 8;
     static constexpr int T_LAZY = 8;                   // reference slack, base 2
     // fixed region after the stage ring; every piece 1024-aligned
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_QT = OFF_Q + NQ * QSLOT_BYTES;
     static constexpr int OFF_P = OFF_QT + NQ * QT_BYTES;
-    static constexpr int OFF_VC = OFF_P + NP * P_BYTES;
-    static constexpr int OFF_X = OFF_VC + NVC * VC_BYTES;       // exchange scratch
+    static constexpr int OFF_X = OFF_P + NP * P_BYTES;          // exchange scratch
     static constexpr int X_BYTES = 2 * NSM * 32 * 4 + 2 * 32 * 4 + 2 * NSM * 4;
     static constexpr int OFF_CTRL = OFF_X + ((X_BYTES + 1023) / 1024) * 1024;
     static constexpr int CTRL_BYTES = 1024;
@@ -107,7 +109,6 @@ struct __align__(16) TcControl {
     uint64_t qtfull[2], qtempty[2]; // E4M3 query terms (KV8)
     uint64_t sfull[2], sfree[2];    // S^T buffer b written / read by the softmax warps
     uint64_t pfull[2];              // P^T buffer written
-    uint64_t vcfull[2];             // converted V buffer written (KV8)
     uint64_t pvdone[2];             // value product of the last step using P^T buffer b completed
     uint64_t ofull, ofree;          // O^T of a segment complete / read by the epilogue
     uint64_t xch;                   // softmax-warp exchange (count 4)
@@ -192,7 +193,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     static_assert(sizeof(TcExchange) <= C::X_BYTES, "exchange scratch overflows its slot");
     constexpr uint32_t IDESC_QK = KV8 ? tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, 0, 0, 128, C::NS_COLS)
                                       : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 128, C::NS_COLS);
-    constexpr uint32_t IDESC_PV = KV8 ? tc::instr_desc(tc::kFmtF16, tc::kFmtF16, 1, 1, 128, C::NO_COLS)
+    constexpr uint32_t IDESC_PV = KV8 ? tc::instr_desc(tc::kFmtE4M3, tc::kFmtE4M3, 1, 1, 128, C::NO_COLS)
                                       : tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 1, 1, 128, C::NO_COLS);
 
     extern __shared__ uint8_t smem_raw[];
@@ -206,7 +207,6 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     const uint32_t q_base = fixed + C::OFF_Q;
     const uint32_t qt_base = fixed + C::OFF_QT;
     const uint32_t p_base = fixed + C::OFF_P;
-    const uint32_t vc_base = fixed + C::OFF_VC;
     TcExchange* X = reinterpret_cast<TcExchange*>(fixed_ptr + C::OFF_X);
     TcControl* ctrl = reinterpret_cast<TcControl*>(fixed_ptr + C::OFF_CTRL);
     volatile int* abort_flag = &ctrl->abort;
@@ -222,8 +222,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NS; ++s) {
             mbar_init(smem_addr(&ctrl->full[s]), 1);
-            // bf16: freed by the value product; KV8: by the score product and the converters
-            mbar_init(smem_addr(&ctrl->empty[s]), KV8 ? 1 + C::NCV : 1);
+            mbar_init(smem_addr(&ctrl->empty[s]), 1);  // freed by the value product
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->qfull[s]), 1);
@@ -233,7 +232,6 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             mbar_init(smem_addr(&ctrl->sfull[s]), 1);
             mbar_init(smem_addr(&ctrl->sfree[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->pfull[s]), C::NSM);
-            mbar_init(smem_addr(&ctrl->vcfull[s]), KV8 ? C::NCV : 1);
             mbar_init(smem_addr(&ctrl->pvdone[s]), 1);
             mbar_init(smem_addr(&ctrl->drain[s]), 1);
         }
@@ -244,7 +242,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     }
     // Query rows past H_Q come back from TMA as zeros; the P^T buffers start
     // zeroed so their padding columns are finite.
-    for (int i = threadIdx.x; i < C::OFF_VC / 16; i += blockDim.x)
+    for (int i = threadIdx.x; i < C::OFF_X / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(fixed_ptr)[i] = make_uint4(0, 0, 0, 0);
 
     grid_dependency_wait();
@@ -391,7 +389,6 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         }
                     }
                     tc::commit(smem_addr(&ctrl->sfull[sb]));
-                    if constexpr (KV8) tc::commit(smem_addr(&ctrl->empty[st]));  // keys read; converters arrive too
                     if (sp.seg_last)  // the segment's query slot is free once its last score product is done
                         tc::commit(KV8 ? smem_addr(&ctrl->qtempty[qcur]) : smem_addr(&ctrl->qempty[qcur]));
                 }
@@ -422,13 +419,6 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 const uint32_t ppar = static_cast<uint32_t>(j / C::NP) & 1u;
                 if (sp.seg_first) ++seg;
                 if (!mbar_wait_warp(smem_addr(&ctrl->pfull[pb]), ppar, abort_flag)) { ok = false; break; }
-                if constexpr (KV8) {
-                    if (!mbar_wait_warp(smem_addr(&ctrl->vcfull[j & 1]), static_cast<uint32_t>(j >> 1) & 1u,
-                                        abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                }
                 if (sp.seg_first && seg > 0)
                     if (!mbar_wait_warp(smem_addr(&ctrl->ofree), static_cast<uint32_t>(seg - 1) & 1u, abort_flag)) {
                         ok = false;
@@ -436,16 +426,26 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     }
                 tc::fence_after_sync();
                 if (tc::elect_one()) {
-                    const uint32_t vt = KV8 ? vc_base + (j & 1) * C::VC_BYTES
-                                            : stages + st * C::STAGE_BYTES + C::KV_BYTES;
+                    const uint32_t vt = stages + st * C::STAGE_BYTES + C::KV_BYTES;
                     const uint32_t pt = p_base + pb * C::P_BYTES;
+                    if constexpr (KV8) {
+                        // 32 tokens per product: V^T rows read MN-major (128 d bytes per
+                        // token row), P^T as four E4M3 terms per head.
 #pragma unroll
-                    for (int k = 0; k < kStepTokens / 16; ++k) {
-                        const uint64_t da = tc::smem_desc(vt + k * 2048, C::PANEL_BYTES, 1024, tc::kLayoutSw128);
-                        const uint64_t db = tc::smem_desc(pt + k * 256, 128, C::P_SBO, tc::kLayoutNone);
-                        tc::mma_f16(tmem + C::O_COL, da, db, IDESC_PV, !(sp.seg_first && k == 0));
+                        for (int k = 0; k < kStepTokens / 32; ++k) {
+                            const uint64_t da = tc::smem_desc(vt + k * 4096, C::PANEL_BYTES, 1024, tc::kLayoutSw128);
+                            const uint64_t db = tc::smem_desc(pt + k * 512, 128, C::P_SBO, tc::kLayoutNone);
+                            tc::mma_f8(tmem + C::O_COL, da, db, IDESC_PV, !(sp.seg_first && k == 0));
+                        }
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < kStepTokens / 16; ++k) {
+                            const uint64_t da = tc::smem_desc(vt + k * 2048, C::PANEL_BYTES, 1024, tc::kLayoutSw128);
+                            const uint64_t db = tc::smem_desc(pt + k * 256, 128, C::P_SBO, tc::kLayoutNone);
+                            tc::mma_f16(tmem + C::O_COL, da, db, IDESC_PV, !(sp.seg_first && k == 0));
+                        }
                     }
-                    if constexpr (!KV8) tc::commit(smem_addr(&ctrl->empty[st]));
+                    tc::commit(smem_addr(&ctrl->empty[st]));
                     tc::commit(smem_addr(&ctrl->pvdone[pb]));
                     if (sp.seg_last) tc::commit(smem_addr(&ctrl->ofull));
                 }
@@ -460,66 +460,11 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         mbar_wait_warp(smem_addr(&ctrl->drain[1]), 0u, nullptr);
     }
 
-    if constexpr (KV8) {
-        if (lo < hi && warp >= C::WARP_CV0) {
-            // ------------------------------------------------------------ V converters
-            // Thread t: token row t of the step; E4M3 -> f16 holding value * 2^-8
-            // (exact, by bit placement) into the bf16-style layout (two 64-d
-            // panels, 128-byte swizzle).  Within each group of four, d is stored
-            // in the order 4i, 4i+2, 4i+1, 4i+3 (undone when O^T is written).
-            // Rows past L_b, and the zero-filled half of a one-tile step, become
-            // zeros so 0 * NaN cannot reach O^T.
-            const int t = threadIdx.x - 32 * C::WARP_CV0;
-            int st = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            int j = 0;
-            for (int64_t gi = lo; gi < hi; ++j) {
-                const Step sp = step_at(w, gi, lo, hi);
-                const int c = j & 1;
-                const uint32_t par = static_cast<uint32_t>(j >> 1) & 1u;
-                if (!mbar_wait_warp(smem_addr(&ctrl->full[st]), ph, abort_flag)) { ok = false; break; }
-                if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[c]), par ^ 1u, abort_flag)) { ok = false; break; }
-                const bool live = t < kTile * sp.n && w.tile * kTile + t < w.L;
-                const uint32_t src = stages + st * C::STAGE_BYTES + C::KV_BYTES + t * 128;
-                const uint32_t dst = vc_base + c * C::VC_BYTES + t * 128;
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const uint4 v = ld_shared_v4(src + ((ch ^ (t & 7)) << 4));
-                    uint32_t o[8];
-                    e4m3x4_to_f16x2_scaled(v.x, o[0], o[1]);
-                    e4m3x4_to_f16x2_scaled(v.y, o[2], o[3]);
-                    e4m3x4_to_f16x2_scaled(v.z, o[4], o[5]);
-                    e4m3x4_to_f16x2_scaled(v.w, o[6], o[7]);
-                    if (!live) {
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) o[i] = 0u;
-                    }
-                    // d = 16 ch .. 16 ch + 15: panel ch / 4, f16 chunks 2 (ch % 4), 2 (ch % 4) + 1
-                    const uint32_t pd = dst + (ch >> 2) * C::PANEL_BYTES;
-                    const int c0 = 2 * (ch & 3);
-                    st_shared_v4(pd + ((c0 ^ (t & 7)) << 4), o[0], o[1], o[2], o[3]);
-                    st_shared_v4(pd + (((c0 + 1) ^ (t & 7)) << 4), o[4], o[5], o[6], o[7]);
-                }
-                fence_async_smem_writes();
-                __syncwarp();
-                if (lane == 0) {
-                    mbar_arrive(smem_addr(&ctrl->vcfull[c]));
-                    mbar_arrive(smem_addr(&ctrl->empty[st]));  // this warp is done reading the stage
-                }
-                if (++st == NS) { st = 0; ph ^= 1u; }
-                advance_step(w, a, gi, sp.n, hi);
-            }
-            if (!ok) fail();
-        }
-    }
-
     if (lo < hi && warp >= C::WARP_SM0 && warp < C::WARP_SM0 + C::NSM) {
         // ------------------------------------------------------------ softmax + epilogue
         const int sp = warp & 3;            // tensor-memory sub-partition of this warp
         const int tok = 32 * sp + lane;     // S^T row (token of the step) held by this thread
         const float NEG_INF = -__int_as_float(0x7f800000);
-        constexpr float PSCALE = KV8 ? 128.f : 1.f;  // keeps f16 weights normal
         float m[RP], l[RP];
         uint32_t xpar = 0, qph = 0;
         int qs = 0, qcur = 0, seg = -1, seg_start_tile = 0, st = 0;
@@ -551,7 +496,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     l[h] = 0.f;
                 }
                 if constexpr (KV8) {
-                    vfac = __ldg(a.v_scale + w.kv) * (256.f / PSCALE);  // values were decoded as v * 2^-8
+                    vfac = __ldg(a.v_scale + w.kv);
                     qf_uniform = a.sl2 * __ldg(a.k_scale + w.kv);
                     if (!mbar_wait_warp(smem_addr(&ctrl->qfull[qcur]), qpar, abort_flag)) { ok = false; break; }
                     if (!mbar_wait_warp(smem_addr(&ctrl->qtempty[qcur]), qpar ^ 1u, abort_flag)) {
@@ -738,31 +683,54 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 }
             }
 
-            // ---- row sums, P^T (hi | lo) for the value product
+            // ---- row sums, P^T for the value product
 #pragma unroll
             for (int h = 0; h < RP; ++h) l[h] += p[h];
             if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[pb]), ppar ^ 1u, abort_flag)) { ok = false; break; }
             {
                 const uint32_t pt = p_base + pb * C::P_BYTES + (tok >> 3) * 128 + (tok & 7) * 16;
+                if constexpr (KV8) {
+                    // p = t1 + t2 / 16 + t3 / 256 + t4 / 4096, each term E4M3 (p <= 2^8 < 448);
+                    // columns are [t1 | t2 | t3 | t4], RP heads each.
+                    uint32_t wd[RP];  // term k, heads 4i..4i+3 -> wd[k * RP / 4 + i]
 #pragma unroll
-                for (int g = 0; g < RP / 8; ++g) {
-                    uint32_t hw[4], lw[4];
+                    for (int i = 0; i < RP / 4; ++i) {
+                        float x0 = p[4 * i], x1 = p[4 * i + 1], x2 = p[4 * i + 2], x3 = p[4 * i + 3];
 #pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        split_pair<KV8>(p[8 * g + 2 * e] * PSCALE, p[8 * g + 2 * e + 1] * PSCALE, hw[e], lw[e]);
-                    st_shared_v4(pt + g * C::P_SBO, hw[0], hw[1], hw[2], hw[3]);
-                    st_shared_v4(pt + (g + RP / 8) * C::P_SBO, lw[0], lw[1], lw[2], lw[3]);
+                        for (int k = 0; k < 4; ++k) {
+                            const uint16_t b01 = f32x2_to_e4m3x2(x0, x1);
+                            const uint16_t b23 = f32x2_to_e4m3x2(x2, x3);
+                            wd[k * (RP / 4) + i] = static_cast<uint32_t>(b01) | (static_cast<uint32_t>(b23) << 16);
+                            if (k < 3) {
+                                const float2 f01 = e4m3x2_to_f32x2(b01), f23 = e4m3x2_to_f32x2(b23);
+                                x0 = (x0 - f01.x) * 16.f;
+                                x1 = (x1 - f01.y) * 16.f;
+                                x2 = (x2 - f23.x) * 16.f;
+                                x3 = (x3 - f23.y) * 16.f;
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int g = 0; g < RP / 4; ++g)
+                        st_shared_v4(pt + g * C::P_SBO, wd[4 * g], wd[4 * g + 1], wd[4 * g + 2], wd[4 * g + 3]);
+                } else {
+#pragma unroll
+                    for (int g = 0; g < RP / 8; ++g) {
+                        uint32_t hw[4], lw[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) split_pair<false>(p[8 * g + 2 * e], p[8 * g + 2 * e + 1], hw[e], lw[e]);
+                        st_shared_v4(pt + g * C::P_SBO, hw[0], hw[1], hw[2], hw[3]);
+                        st_shared_v4(pt + (g + RP / 8) * C::P_SBO, lw[0], lw[1], lw[2], lw[3]);
+                    }
                 }
             }
-            if constexpr (!KV8) {
-                // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
-                if (last_of_unit && loaded && !valid) {
-                    const uint32_t vrow = stages + st * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
+            // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
+            if (last_of_unit && loaded && !valid) {
+                const uint32_t vrow = stages + st * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
 #pragma unroll
-                    for (int pnl = 0; pnl < 2; ++pnl)
+                for (int pnl = 0; pnl < (KV8 ? 1 : 2); ++pnl)
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) st_shared_v4(vrow + pnl * C::PANEL_BYTES + 16 * c, 0u, 0u, 0u, 0u);
-                }
+                    for (int c = 0; c < 8; ++c) st_shared_v4(vrow + pnl * C::PANEL_BYTES + 16 * c, 0u, 0u, 0u, 0u);
             }
             fence_async_smem_writes();
             tc::fence_before_sync();
@@ -795,22 +763,34 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                // O^T row 32 sp + lane; 8-bit values were stored with d order (0, 2, 1, 3) in each 4
-                const int drow = 32 * sp + lane;
-                const int d = KV8 ? (drow & ~3) | ((drow & 1) << 1) | ((drow >> 1) & 1) : drow;
+                const int d = 32 * sp + lane;  // O^T row
                 const bool whole = (seg_start_tile == 0) && last_of_unit;
                 const int64_t slot = 2 * static_cast<int64_t>(blockIdx.x) + (seg == 0 ? 0 : 1);
 #pragma unroll
                 for (int c = 0; c < RP / 8; ++c) {
-                    uint32_t hv[8], lv[8];
-                    tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + 8 * c), hv);
-                    tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + RP + 8 * c), lv);
-                    tc::tmem_wait_ld();
+                    // the P terms' columns: hi + lo, or t1 + t2 / 16 + t3 / 256 + t4 / 4096
+                    float acc[8];
+                    {
+                        uint32_t tv[8];
+                        tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + 8 * c), tv);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(tv[e]);
+                    }
+#pragma unroll
+                    for (int k = C::NPT - 1; k >= 1; --k) {
+                        uint32_t tv[8];
+                        tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + k * RP + 8 * c), tv);
+                        tc::tmem_wait_ld();
+                        const float wk = KV8 ? 1.f / static_cast<float>(1 << (4 * k)) : 1.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc[e] += __uint_as_float(tv[e]) * wk;
+                    }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         const int h = 8 * c + e;
                         if (h >= a.R) continue;
-                        const float o = (__uint_as_float(hv[e]) + __uint_as_float(lv[e])) * (vfac / lt[h]);
+                        const float o = acc[e] * (vfac / lt[h]);
                         if (whole) {
                             const int64_t i = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + h) * C::D + d;
                             if constexpr (OUT_BF16)
