@@ -91,6 +91,7 @@ struct TcCfg {
     static constexpr int NP = (!KV8 && RP == 32) ? 1 : 2;
     static constexpr int MAX_STAGES = 8;
     static constexpr int T_LAZY = 8;                   // reference slack, base 2
+    static constexpr bool PAIR = RP <= 16;             // softmax warps take two steps per pass
     // fixed region after the stage ring; every piece 1024-aligned
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_QT = OFF_Q + NQ * QSLOT_BYTES;
@@ -480,9 +481,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         };
 
         int j = 0;
-        for (int64_t gi = lo; gi < hi; ++j) {
+        for (int64_t gi = lo; gi < hi;) {
             const Step stp = step_at(w, gi, lo, hi);
-            const bool last_of_unit = (w.tile + stp.n == w.n_b);
             if (stp.seg_first) {
                 ++seg;
                 seg_start_tile = w.tile;
@@ -553,19 +553,34 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     if (!exchange()) { ok = false; break; }  // every head's 2^-a is in place
                 }
             }
-            const int sb = j & 1;
-            const uint32_t spar = static_cast<uint32_t>(j >> 1) & 1u;
-            const int pb = j % C::NP;
-            const uint32_t ppar = static_cast<uint32_t>(j / C::NP) & 1u;
-            const int t0 = w.tile * kTile;
-            const bool loaded = tok < kTile * stp.n;
-            const bool valid = loaded && (t0 + tok < w.L);
+            // The softmax warps take two steps of a segment per pass (one when the
+            // segment ends after the first), so one exchange and one round of
+            // barrier hops serve up to 256 tokens.
+            int nsub = 1, n_of[2] = {stp.n, 0}, tile_of[2] = {w.tile, 0};
+            bool seg_last = stp.seg_last;
+            if constexpr (C::PAIR) {
+                if (!stp.seg_last) {
+                    const int64_t g1 = gi + stp.n;
+                    tile_of[1] = w.tile + stp.n;
+                    n_of[1] = (g1 + 1 < hi && tile_of[1] + 1 < w.n_b) ? 2 : 1;
+                    seg_last = (g1 + n_of[1] == hi) || (tile_of[1] + n_of[1] == w.n_b);
+                    nsub = 2;
+                }
+            }
+            const bool last_of_unit = (tile_of[nsub - 1] + n_of[nsub - 1] == w.n_b);
+            constexpr int MS = C::PAIR ? 2 : 1;
 
-            // ---- scores of this thread's token
-            if (!mbar_wait_warp(smem_addr(&ctrl->sfull[sb]), spar, abort_flag)) { ok = false; break; }
-            tc::fence_after_sync();
-            float s[RP];
-            {
+            // ---- scores of this thread's token in each step
+            float s[MS][RP];
+#pragma unroll
+            for (int u = 0; u < MS; ++u) {
+                if (u >= nsub) break;
+                const int ju = j + u, sb = ju & 1;
+                if (!mbar_wait_warp(smem_addr(&ctrl->sfull[sb]), static_cast<uint32_t>(ju >> 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
                 const uint32_t ta = tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::NS_COLS);
                 if constexpr (!KV8) {
 #pragma unroll
@@ -574,7 +589,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         tc::tmem_ld16(ta + 16 * c, r);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) s[16 * c + i] = __uint_as_float(r[i]) * qf_uniform;
+                        for (int i = 0; i < 16; ++i) s[u][16 * c + i] = __uint_as_float(r[i]) * qf_uniform;
                     }
                 } else {
                     // columns h (term 1) and RP + h (term 2), 8 heads at a time
@@ -589,18 +604,20 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         const float qsc[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            s[8 * c + i] = (__uint_as_float(r1[i]) + __uint_as_float(r2[i]) * 0.0625f) *
-                                           (qf_uniform * qsc[i]);
+                            s[u][8 * c + i] = (__uint_as_float(r1[i]) + __uint_as_float(r2[i]) * 0.0625f) *
+                                              (qf_uniform * qsc[i]);
                     }
                 }
-            }
-            // S^T buffer sb may take the step after next
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
+                // S^T buffer sb may take the step after next
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
+                const bool valid = tok < kTile * n_of[u] && tile_of[u] * kTile + tok < w.L;
 #pragma unroll
-            for (int h = 0; h < RP; ++h)
-                if (!valid || h >= a.R) s[h] = NEG_INF;
+                for (int h = 0; h < RP; ++h)
+                    if (!valid || h >= a.R) s[u][h] = NEG_INF;
+            }
+            if (!ok) break;
 
             // ---- reference check: does any score exceed its head's reference by more than T?
             // The flags go out first; the weights against the current reference are
@@ -608,8 +625,12 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             // some warp found an excess (normally the first step of a segment).
             bool exceed = false;
 #pragma unroll
-            for (int h = 0; h < RP; ++h) exceed |= s[h] > m[h] + static_cast<float>(C::T_LAZY);
-            float p[RP];
+            for (int u = 0; u < MS; ++u)
+                if (u < nsub) {
+#pragma unroll
+                    for (int h = 0; h < RP; ++h) exceed |= s[u][h] > m[h] + static_cast<float>(C::T_LAZY);
+                }
+            float p[MS][RP];
             {
                 const uint32_t xb = xpar;
                 const bool any = __any_sync(0xffffffffu, exceed);
@@ -619,7 +640,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 #pragma unroll
                 for (int h = 0; h < RP; ++h) {
                     const float ref = m[h] == NEG_INF ? 0.f : m[h];
-                    p[h] = fast_exp2(s[h] - ref);
+#pragma unroll
+                    for (int u = 0; u < MS; ++u) p[u][h] = u < nsub ? fast_exp2(s[u][h] - ref) : 0.f;
                 }
                 const bool xok = mbar_wait_warp(smem_addr(&ctrl->xch), xpar, abort_flag);
                 xpar ^= 1u;
@@ -629,7 +651,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     float mx[RP];
 #pragma unroll
                     for (int h = 0; h < RP; ++h) {
-                        float v = s[h];
+                        float v = s[0][h];
+                        if (MS > 1 && nsub > 1) v = fmaxf(v, s[MS - 1][h]);
 #pragma unroll
                         for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
                         mx[h] = v;
@@ -656,7 +679,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         }
                         l[h] *= alpha[h];
                         const float ref = m[h] == NEG_INF ? 0.f : m[h];
-                        p[h] = fast_exp2(s[h] - ref);
+#pragma unroll
+                        for (int u = 0; u < MS; ++u) p[u][h] = u < nsub ? fast_exp2(s[u][h] - ref) : 0.f;
                     }
                     if (moved && w.tile != seg_start_tile) {
                         // O^T holds this segment's earlier steps: rescale it in place once
@@ -683,11 +707,20 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 }
             }
 
-            // ---- row sums, P^T for the value product
+            // ---- row sums, P^T for each step's value product
 #pragma unroll
-            for (int h = 0; h < RP; ++h) l[h] += p[h];
-            if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[pb]), ppar ^ 1u, abort_flag)) { ok = false; break; }
-            {
+            for (int h = 0; h < RP; ++h)
+#pragma unroll
+                for (int u = 0; u < MS; ++u) l[h] += p[u][h];
+#pragma unroll
+            for (int u = 0; u < MS; ++u) {
+                if (u >= nsub) break;
+                const int ju = j + u, pb = ju % C::NP;
+                if (!mbar_wait_warp(smem_addr(&ctrl->pvdone[pb]), (static_cast<uint32_t>(ju / C::NP) & 1u) ^ 1u,
+                                    abort_flag)) {
+                    ok = false;
+                    break;
+                }
                 const uint32_t pt = p_base + pb * C::P_BYTES + (tok >> 3) * 128 + (tok & 7) * 16;
                 if constexpr (KV8) {
                     // p = t1 + t2 / 16 + t3 / 256 + t4 / 4096, each term E4M3 (p <= 2^8 < 448);
@@ -695,7 +728,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     uint32_t wd[RP];  // term k, heads 4i..4i+3 -> wd[k * RP / 4 + i]
 #pragma unroll
                     for (int i = 0; i < RP / 4; ++i) {
-                        float x0 = p[4 * i], x1 = p[4 * i + 1], x2 = p[4 * i + 2], x3 = p[4 * i + 3];
+                        float x0 = p[u][4 * i], x1 = p[u][4 * i + 1], x2 = p[u][4 * i + 2], x3 = p[u][4 * i + 3];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint16_t b01 = f32x2_to_e4m3x2(x0, x1);
@@ -718,26 +751,30 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     for (int g = 0; g < RP / 8; ++g) {
                         uint32_t hw[4], lw[4];
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) split_pair<false>(p[8 * g + 2 * e], p[8 * g + 2 * e + 1], hw[e], lw[e]);
+                        for (int e = 0; e < 4; ++e)
+                            split_pair<false>(p[u][8 * g + 2 * e], p[u][8 * g + 2 * e + 1], hw[e], lw[e]);
                         st_shared_v4(pt + g * C::P_SBO, hw[0], hw[1], hw[2], hw[3]);
                         st_shared_v4(pt + (g + RP / 8) * C::P_SBO, lw[0], lw[1], lw[2], lw[3]);
                     }
                 }
-            }
-            // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
-            if (last_of_unit && loaded && !valid) {
-                const uint32_t vrow = stages + st * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
+                // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
+                const bool loaded = tok < kTile * n_of[u];
+                if (tile_of[u] + n_of[u] == w.n_b && loaded && tile_of[u] * kTile + tok >= w.L) {
+                    const int stu = (st + u) % NS;
+                    const uint32_t vrow = stages + stu * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
 #pragma unroll
-                for (int pnl = 0; pnl < (KV8 ? 1 : 2); ++pnl)
+                    for (int pnl = 0; pnl < (KV8 ? 1 : 2); ++pnl)
 #pragma unroll
-                    for (int c = 0; c < 8; ++c) st_shared_v4(vrow + pnl * C::PANEL_BYTES + 16 * c, 0u, 0u, 0u, 0u);
+                        for (int c = 0; c < 8; ++c) st_shared_v4(vrow + pnl * C::PANEL_BYTES + 16 * c, 0u, 0u, 0u, 0u);
+                }
+                fence_async_smem_writes();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull[pb]));
             }
-            fence_async_smem_writes();
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull[pb]));
+            if (!ok) break;
 
-            if (stp.seg_last) {
+            if (seg_last) {
                 // ---------------------------------------------------- segment end
                 float lt[RP];
 #pragma unroll
@@ -811,8 +848,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree));
             }
-            if (++st == NS) st = 0;
+            st = (st + nsub) % NS;
+            j += nsub;
             advance_step(w, a, gi, stp.n, hi);
+            if (nsub > 1) advance_step(w, a, gi, n_of[1], hi);
         }
         if (!ok) fail();
     }
