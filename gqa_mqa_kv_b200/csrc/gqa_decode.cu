@@ -127,8 +127,12 @@ EncodeTiledFn encode_fn() {
 }
 
 // Tiled tensor map with a 128-byte swizzle; out-of-bounds elements read as zero.
+// L2 promotion: 256-byte requests suit rows of 256 bytes or more (a bf16 head
+// row at head_dim 128); a 128-byte row (an E4M3 head row) takes 128-byte
+// requests, or every fetch would also pull the neighbouring head's row.
 bool encode_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, int rank,
-                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box) {
+                const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                CUtensorMapL2promotion promotion = CU_TENSOR_MAP_L2_PROMOTION_L2_256B) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     cuuint64_t d[5], s[4];
@@ -141,7 +145,7 @@ bool encode_map(CUtensorMap* map, CUtensorMapDataType type, const void* base, in
     }
     return fn(map, type, static_cast<cuuint32_t>(rank),
               const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_SWIZZLE_128B, promotion,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -224,8 +228,10 @@ cudaError_t launch_mma(const gqa_decode_params* p, const Buffers& buf, KernelArg
         }
         strides[2] = strides[1] * dims[2];
         const CUtensorMapDataType kv_type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-        *encode_ok = encode_map(&tmK, kv_type, buf.k, 4, dims, strides, box4) &&
-                     encode_map(&tmV, kv_type, buf.v, 4, dims, strides, box4);
+        const CUtensorMapL2promotion promo =
+            kv_row * 2 <= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+        *encode_ok = encode_map(&tmK, kv_type, buf.k, 4, dims, strides, box4, promo) &&
+                     encode_map(&tmV, kv_type, buf.v, 4, dims, strides, box4, promo);
     }
     if (!*encode_ok) return cudaErrorInvalidValue;
     auto kernel = split_mma_kernel<D, NT, HG, PAGED, OUTB, KV8>;
@@ -284,8 +290,10 @@ cudaError_t launch_tc(const gqa_decode_params* p, const Buffers& buf, KernelArgs
         }
         strides[2] = strides[1] * dims[2];
         const CUtensorMapDataType kv_type = KV8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
-        *encode_ok = encode_map(&tmK, kv_type, buf.k, 4, dims, strides, box4) &&
-                     encode_map(&tmV, kv_type, buf.v, 4, dims, strides, box4);
+        const CUtensorMapL2promotion promo =
+            kv_row * 2 <= 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B;
+        *encode_ok = encode_map(&tmK, kv_type, buf.k, 4, dims, strides, box4, promo) &&
+                     encode_map(&tmV, kv_type, buf.v, 4, dims, strides, box4, promo);
     }
     if (!*encode_ok) return cudaErrorInvalidValue;
     auto kernel = split_tc_kernel<RP, PAGED, OUTB, KV8>;
