@@ -40,7 +40,7 @@ ROPE_PAIRING = {"adjacent": 0, "halves": 1}
 EXPORTED = (
     "gqa_decode_workspace_size", "gqa_decode", "gqa_decode_timed", "gqa_read_status",
     "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version", "gqa_decode_static_workspace",
-    "gqa_rope_append", "gqa_decode_fp8kv",
+    "gqa_rope_append", "gqa_decode_fp8kv", "gqa_wait_selftest",
 )
 
 
@@ -105,6 +105,8 @@ def library() -> ctypes.CDLL:
             lib.gqa_decode_fp8kv.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz,
                                              vp]
             lib.gqa_decode_fp8kv.restype = ctypes.c_int
+            lib.gqa_wait_selftest.argtypes = [ctypes.c_uint64, ctypes.c_int, vp, vp, vp]
+            lib.gqa_wait_selftest.restype = ctypes.c_int
             _lib = lib
     return _lib
 
@@ -383,6 +385,24 @@ def gqa_decode_fp8kv(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_tabl
     if st != 0:
         raise GqaError(st, "gqa_decode_fp8kv")
     return out
+
+
+def wait_selftest(timeout_ns: int, abort_early: bool = False, device=None):
+    """Run the library's bounded-wait self test (gqa_wait_selftest) on the GPU
+    and return (flags, elapsed_ns); synchronises the stream."""
+    import torch
+
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    flags = torch.zeros(1, dtype=torch.int32, device=device)
+    elapsed = torch.zeros(1, dtype=torch.int64, device=device)
+    stream = torch.cuda.current_stream(device)
+    st = library().gqa_wait_selftest(ctypes.c_uint64(int(timeout_ns)), int(bool(abort_early)),
+                                     ctypes.c_void_p(flags.data_ptr()), ctypes.c_void_p(elapsed.data_ptr()),
+                                     ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise GqaError(st, "gqa_wait_selftest")
+    stream.synchronize()
+    return int(flags.item()) & 0xFFFFFFFF, int(elapsed.item())
 
 
 def read_status(workspace, stream=None, clear=False) -> int:

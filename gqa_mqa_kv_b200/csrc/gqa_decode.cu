@@ -464,6 +464,40 @@ cudaError_t launch_rope(const void* q, const void* k_new, const void* v_new, voi
 
 }  // namespace
 
+namespace {
+
+// One CTA: warp 0 waits on a barrier nothing arrives on (the kernels' bounded
+// wait, with the caller's limit); warp 1 optionally raises the abort flag
+// after a quarter of the limit, from a loop bounded by the same clock.
+__global__ void wait_selftest_kernel(uint64_t timeout_ns, int abort_early, uint32_t* flags, uint64_t* elapsed) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_addr(&bar), 1);
+        abort_flag = 0;
+    }
+    fence_barrier_init();
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int* af = &abort_flag;
+    if (warp == 0) {
+        const uint64_t t0 = global_timer_ns();
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_for(smem_addr(&bar), 0u, af, timeout_ns));
+        const uint64_t t1 = global_timer_ns();
+        if (lane == 0) {
+            if (!ok) atomicOr(flags, kFlagTimeout);
+            *elapsed = t1 - t0;
+        }
+    } else if (abort_early && lane == 0) {
+        const uint64_t t0 = global_timer_ns();
+        while (global_timer_ns() - t0 < timeout_ns / 4) {
+        }
+        *af = 1;
+    }
+}
+
+}  // namespace
+
 extern "C" {
 
 gqa_status gqa_decode_workspace_size(const gqa_decode_params* params, size_t* bytes) {
@@ -601,6 +635,16 @@ const char* gqa_status_string(gqa_status status) {
         case GQA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
     }
     return "unknown status";
+}
+
+gqa_status gqa_wait_selftest(uint64_t timeout_ns, int abort_early, uint32_t* flags, uint64_t* elapsed_ns,
+                             void* stream) {
+    if (timeout_ns < 1000 || timeout_ns > 10000000000ull) return GQA_ERR_INVALID;
+    if (flags == nullptr || elapsed_ns == nullptr || !aligned(flags, 4) || !aligned(elapsed_ns, 8))
+        return GQA_ERR_INVALID;
+    wait_selftest_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(timeout_ns, abort_early, flags,
+                                                                         elapsed_ns);
+    return cudaGetLastError() == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 
 int gqa_version(void) { return GQA_DECODE_VERSION; }

@@ -164,10 +164,13 @@ gqa_status gqa_decode(const gqa_decode_params* params, const void* q, const void
  * with per-KV-head fp32 factors k_scale[H_KV], v_scale[H_KV] (device).  This is
  * the bytes-per-element term of [AIT]'s cache estimate: the same attention
  * over a cache that moves half the bytes of bf16.  q stays bf16
- * (params->qkv_dtype must be GQA_BF16, |q| below 65504); layouts, seq_lens,
+ * (params->qkv_dtype must be GQA_BF16); layouts, seq_lens,
  * block_table, scale, out and the workspace (gqa_decode_workspace_size with
- * the same params suffices) are as for gqa_decode.  head_dim 128 with up to 8
- * query heads per KV head runs on tensor cores; other shapes on CUDA cores.
+ * the same params suffices) are as for gqa_decode.  head_dim 128 with up to 32
+ * query heads per KV head runs on the tcgen05 kernel (params->kernel =
+ * GQA_KERNEL_MMA_SYNC selects the mma.sync kernel for up to 8, which widens to
+ * f16 and so needs |q| < 65504); other shapes run on CUDA cores.  Cache bytes of
+ * live tokens must not be the E4M3 NaN encodings.
  */
 gqa_status gqa_decode_fp8kv(const gqa_decode_params* params, const void* q, const void* k_cache,
                             const void* v_cache, const float* k_scale, const float* v_scale,
@@ -256,6 +259,20 @@ gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const
  * synchronising `stream`; clears it when `clear` is non-zero.
  */
 gqa_status gqa_read_status(const void* workspace, void* stream, uint32_t* flags, int clear);
+
+/*
+ * Exercises, on the GPU and without any fault, the bounded wait every kernel
+ * of this library uses for its pipeline barriers.  One CTA waits on an
+ * mbarrier that nothing arrives on; the wait gives up after timeout_ns and
+ * the kernel raises GQA_FLAG_TIMEOUT in *flags (device uint32, OR-ed) and
+ * writes the nanoseconds it waited to *elapsed_ns (device uint64).  With
+ * abort_early non-zero, a second warp sets the CTA's abort flag after
+ * timeout_ns / 4 and the wait returns then (the flag is raised the same way).
+ * timeout_ns must lie in [1000, 10^10].  Enqueued on `stream`; allocates
+ * nothing.  For tests of failure detection: the context stays usable.
+ */
+gqa_status gqa_wait_selftest(uint64_t timeout_ns, int abort_early, uint32_t* flags, uint64_t* elapsed_ns,
+                             void* stream);
 
 /*
  * KV-cache size in bytes: 2 x layers x tokens x H_KV x head_dim x elem_bytes

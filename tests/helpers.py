@@ -3,7 +3,7 @@
 Tolerance (from the stated accuracy target for bf16 inputs with fp32
 accumulation): max |gpu - oracle| <= 2e-3 and max rel <= 1e-2, where
 rel_i = |gpu_i - ref_i| / max(|ref_i|, 0.2); the 0.2 floor is atol / rtol, so
-below it the relative bound is the absolute bound.  A bf16 output is judged
+below it the relative bound is the absolute bound.  A bf16 output is compared
 against the oracle value rounded to bf16: within 2e-3 or within one bf16 ulp.
 """
 

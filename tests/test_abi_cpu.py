@@ -218,3 +218,11 @@ def test_fp8kv_rejects_bad_arguments_on_host(lib):
     assert call(params(), ks=66) == GQA_ERR_INVALID          # misaligned float array
     assert call(params(qkv_dtype=1)) == GQA_ERR_UNSUPPORTED  # q must be bf16
     assert call(params(H_Q=6, H_KV=4)) == GQA_ERR_INVALID
+
+
+def test_wait_selftest_rejects_bad_arguments_on_host(lib):
+    vp = ctypes.c_void_p
+    assert lib.gqa_wait_selftest(ctypes.c_uint64(0), 0, vp(16), vp(16), vp(None)) == GQA_ERR_INVALID
+    assert lib.gqa_wait_selftest(ctypes.c_uint64(10**11), 0, vp(16), vp(16), vp(None)) == GQA_ERR_INVALID
+    assert lib.gqa_wait_selftest(ctypes.c_uint64(10**6), 0, vp(None), vp(16), vp(None)) == GQA_ERR_INVALID
+    assert lib.gqa_wait_selftest(ctypes.c_uint64(10**6), 0, vp(16), vp(12), vp(None)) == GQA_ERR_INVALID
