@@ -59,6 +59,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-sample-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--kernel", default="auto", choices=["auto", "mma_sync", "tcgen05"],
+                    help="split kernel (gqa_kernel); auto is the library's choice")
     ap.add_argument("--path", default="decode", choices=["decode", "append_decode"],
                     help="decode: gqa_decode per step; append_decode: gqa_rope_append of the "
                          "newest token (re-appended at L_b - 1) followed by gqa_decode")
@@ -337,15 +339,15 @@ def run_ours(args):
             if events is not None:
                 events[0].record(stream)
             gq.gqa_decode_fp8kv(q, k, v, ks, vs, lens, table, scale=w.softmax_scale, out=out,
-                                workspace=ws, stream=stream)
+                                workspace=ws, stream=stream, kernel=args.kernel)
             if events is not None:
                 events[1].record(stream)
         elif events is not None:
             gq.gqa_decode_timed(events, q, k, v, lens, table, scale=w.softmax_scale, out=out,
-                                workspace=ws, stream=stream)
+                                workspace=ws, stream=stream, kernel=args.kernel)
         else:
             gq.gqa_decode(q, k, v, lens, table, scale=w.softmax_scale, out=out, workspace=ws,
-                          stream=stream)
+                          stream=stream, kernel=args.kernel)
 
     def step():
         if flush is not None:
@@ -451,7 +453,7 @@ def run_ours(args):
         "pct_of_hbm_peak": 100.0 * (value / world) / peak, "peak_kind": peak_kind,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16 q, e4m3 KV" if w.kv8 else "bf16",
-        "data": "synthetic", "config": workload_config(w, world),
+        "data": "synthetic", "config": dict(workload_config(w, world), split_kernel=args.kernel),
         "algorithmic_bytes_per_step_per_gpu": step_bytes,
         "clocks": clocks.summary(),
         "e2e": {"value": world * step_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",

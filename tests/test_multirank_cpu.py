@@ -111,6 +111,29 @@ def rank_tp_shards(rank, world):
     return bool(np.array_equal(got, full))
 
 
+def rank_tp_dup_shards(rank, world):
+    import dataclasses
+
+    import numpy as np
+
+    import oracle
+    from gqa_mqa_kv_b200.sharding import tp_head_shard
+    from gqa_mqa_kv_b200.workloads import WORKLOADS, make_inputs
+
+    dist.init_process_group("gloo")
+    # 4 ranks over 2 KV heads: each KV head is held by two ranks
+    w = dataclasses.replace(WORKLOADS["tiny"], B=2, H_Q=8, H_KV=2, seq_len=96)
+    inp = make_inputs(w)
+    qs, ks = tp_head_shard(w.H_Q, w.H_KV, world, rank)
+    mine = oracle.gqa_decode(inp["q"][:, qs].contiguous(), inp["k"][:, :, ks].contiguous(),
+                             inp["v"][:, :, ks].contiguous(), inp["seq_lens"], w.softmax_scale)
+    parts = [None] * world
+    dist.all_gather_object(parts, (qs.start, mine))
+    got = np.concatenate([m for _, m in sorted(parts, key=lambda x: x[0])], axis=1)
+    full = oracle.gqa_decode(inp["q"], inp["k"], inp["v"], inp["seq_lens"], w.softmax_scale)
+    return bool(np.array_equal(got, full))
+
+
 def rank_reference_arm(rank, world):
     import bench
 
@@ -141,5 +164,26 @@ def test_shard_helpers():
 
     assert [batch_shard(7, 3, r) for r in range(3)] == [slice(0, 2), slice(2, 4), slice(4, 7)]
     assert tp_head_shard(64, 8, 8, 3) == (slice(24, 32), slice(3, 4))
+    # TP > H_KV duplicates KV heads: 8 ranks over 4 KV heads, two ranks per head
+    assert [tp_head_shard(32, 4, 8, r) for r in (0, 1, 2, 7)] == [
+        (slice(0, 4), slice(0, 1)), (slice(4, 8), slice(0, 1)), (slice(8, 12), slice(1, 2)),
+        (slice(28, 32), slice(3, 4))]
     with pytest.raises(ValueError):
-        tp_head_shard(32, 4, 8, 0)  # TP > H_KV needs duplication
+        tp_head_shard(32, 4, 3, 0)  # neither divides the other
+    with pytest.raises(ValueError):
+        tp_head_shard(24, 8, 16, 0)  # H_Q not a multiple of the TP size
+
+
+def test_duplicated_kv_shards_keep_each_query_head_on_its_own_group():
+    from gqa_mqa_kv_b200.sharding import tp_head_shard
+
+    for H_Q, H_KV, world in [(32, 4, 8), (64, 8, 16), (32, 1, 4), (64, 2, 32)]:
+        R = H_Q // H_KV
+        for rank in range(world):
+            qs, ks = tp_head_shard(H_Q, H_KV, world, rank)
+            assert ks.stop - ks.start == 1
+            assert all(h // R == ks.start for h in range(qs.start, qs.stop))
+
+
+def test_tensor_parallel_with_duplicated_kv_reassembles_the_full_step():
+    assert run_ranks("rank_tp_dup_shards", world=4) == {0: True, 1: True, 2: True, 3: True}

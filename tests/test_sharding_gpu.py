@@ -1,0 +1,41 @@
+"""Tensor-parallel head sharding on one GPU: every shard is an ordinary decode.
+
+"Grouped-Query Attention (GQA) and Multi-Query Attention (MQA): Mathematical
+Foundations, ...", section 4 "Tensor Parallelism (TP) Head Partitioning": with
+H_KV % N = 0 each rank runs GQA on its own KV heads and their query heads; with
+N > H_KV the KV heads are duplicated and each rank runs MQA on one of them.
+Here the N shards run one after another as independent calls on one GPU (no
+shard waits on another) and their outputs, concatenated along the head axis,
+must match the oracle and the unsharded call.
+"""
+
+import dataclasses
+
+import pytest
+import torch
+
+import gqa_mqa_kv_b200 as gq
+from gqa_mqa_kv_b200.sharding import tp_head_shard
+from gqa_mqa_kv_b200.workloads import WORKLOADS, make_inputs
+from tests.helpers import assert_parity, to_device
+from tests.test_parity_gpu import oracle_full, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("world,h_q,h_kv", [(2, 64, 8), (8, 64, 8), (8, 32, 4), (4, 32, 1), (4, 32, 2)])
+def test_tp_shards_reassemble_the_full_step(cuda_device, world, h_q, h_kv):
+    w = dataclasses.replace(WORKLOADS["llama2_70b_ragged"], B=3, H_Q=h_q, H_KV=h_kv, seq_len=900)
+    inp = make_inputs(w)
+    d = to_device(inp, cuda_device)
+    parts = []
+    for rank in range(world):
+        qs, ks = tp_head_shard(h_q, h_kv, world, rank)
+        q = d["q"][:, qs].contiguous()
+        k = d["k"][:, :, ks].contiguous()
+        v = d["v"][:, :, ks].contiguous()
+        parts.append(gq.gqa_decode(q, k, v, d["seq_lens"], scale=w.softmax_scale))
+    got = torch.cat(parts, dim=1).cpu()
+    assert_parity(got, oracle_full(inp, w), f"TP {world} over {h_q}/{h_kv}")
+    full = run_gpu(inp, w, cuda_device)
+    assert (got - full).abs().max().item() < 1e-4
