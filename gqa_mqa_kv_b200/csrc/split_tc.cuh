@@ -71,7 +71,11 @@ struct TcCfg {
     static constexpr int S_COL = 0;                    // S^T buffer b at S_COL + b * NS_COLS
     static constexpr int O_COL = 2 * NS_COLS;
     static constexpr int TMEM_COLS = 512;              // the whole tensor memory of the SM
-    static constexpr int NSM = 4;                      // softmax warps
+    // Softmax warps: one per tensor-memory sub-partition, two (each taking half
+    // the query columns) for 32 columns.
+    static constexpr int HSPLIT = RP == 32 ? 2 : 1;
+    static constexpr int HW = RP / HSPLIT;             // query columns per softmax warp
+    static constexpr int NSM = 4 * HSPLIT;
     static constexpr int WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
     static constexpr int THREADS = 32 * (3 + NSM);
     static constexpr int HALF_BYTES = kTile * 128;     // one 64-row TMA box of 128-byte rows
@@ -91,13 +95,13 @@ struct TcCfg {
     static constexpr int NP = (!KV8 && RP == 32) ? 1 : 2;
     static constexpr int MAX_STAGES = 8;
     static constexpr int T_LAZY = 8;                   // reference slack, base 2
-    static constexpr bool PAIR = RP <= 16;             // softmax warps take two steps per pass
+    static constexpr bool PAIR = HW <= 16 && NP == 2;  // softmax warps take two steps per pass
     // fixed region after the stage ring; every piece 1024-aligned
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_QT = OFF_Q + NQ * QSLOT_BYTES;
     static constexpr int OFF_P = OFF_QT + NQ * QT_BYTES;
     static constexpr int OFF_X = OFF_P + NP * P_BYTES;          // exchange scratch
-    static constexpr int X_BYTES = 2 * NSM * 32 * 4 + 2 * 32 * 4 + 2 * NSM * 4;
+    static constexpr int X_BYTES = 2 * 4 * 32 * 4 + 2 * 32 * 4 + 2 * 8 * 4;
     static constexpr int OFF_CTRL = OFF_X + ((X_BYTES + 1023) / 1024) * 1024;
     static constexpr int CTRL_BYTES = 1024;
     static constexpr int FIXED_BYTES = OFF_CTRL + CTRL_BYTES;
@@ -121,9 +125,9 @@ struct __align__(16) TcControl {
 
 // Scratch for the softmax warps' exchanges (double-buffered by exchange parity).
 struct TcExchange {
-    float vals[2][4][32];  // per warp, per head: step maxima or row sums
+    float vals[2][4][32];  // per sub-partition, per head: step maxima or row sums
     float qscale[2][32];   // KV8: 2^-a per head, per query-term slot
-    int flags[2][4];
+    int flags[2][8];       // per softmax warp
 };
 
 // One step of a CTA's walk: tiles [tile, tile + n) of the current unit.
@@ -464,9 +468,12 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
     if (lo < hi && warp >= C::WARP_SM0 && warp < C::WARP_SM0 + C::NSM) {
         // ------------------------------------------------------------ softmax + epilogue
         const int sp = warp & 3;            // tensor-memory sub-partition of this warp
+        const int wi = warp - C::WARP_SM0;  // softmax warp index
+        const int h0 = (wi >> 2) * C::HW;   // first query column of this warp
         const int tok = 32 * sp + lane;     // S^T row (token of the step) held by this thread
+        constexpr int HW = C::HW;
         const float NEG_INF = -__int_as_float(0x7f800000);
-        float m[RP], l[RP];
+        float m[HW], l[HW];
         uint32_t xpar = 0, qph = 0;
         int qs = 0, qcur = 0, seg = -1, seg_start_tile = 0, st = 0;
         float vfac = 1.f, qf_uniform = a.sl2;
@@ -491,7 +498,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 (void)qpar;
                 if (++qs == C::NQ) { qs = 0; qph ^= 1u; }
 #pragma unroll
-                for (int h = 0; h < RP; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     m[h] = NEG_INF;
                     l[h] = 0.f;
                 }
@@ -507,7 +514,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     const uint32_t qsrc = q_base + qcur * C::QSLOT_BYTES;
                     const uint32_t qdst = qt_base + qcur * C::QT_BYTES;
                     const int d0 = 4 * lane;
-                    for (int hh = sp; hh < RP; hh += 4) {
+                    for (int hh = wi; hh < RP; hh += C::NSM) {
                         const int pnl = d0 >> 6, ch = (d0 & 63) >> 3;
                         const uint2 wq = ld_shared_v2(qsrc + pnl * C::QPANEL_BYTES + hh * 128 +
                                                       ((ch ^ (hh & 7)) << 4) + ((d0 & 7) << 1));
@@ -571,7 +578,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             constexpr int MS = C::PAIR ? 2 : 1;
 
             // ---- scores of this thread's token in each step
-            float s[MS][RP];
+            float s[MS][HW];
 #pragma unroll
             for (int u = 0; u < MS; ++u) {
                 if (u >= nsub) break;
@@ -584,9 +591,9 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 const uint32_t ta = tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::NS_COLS);
                 if constexpr (!KV8) {
 #pragma unroll
-                    for (int c = 0; c < RP / 16; ++c) {
+                    for (int c = 0; c < HW / 16; ++c) {
                         uint32_t r[16];
-                        tc::tmem_ld16(ta + 16 * c, r);
+                        tc::tmem_ld16(ta + h0 + 16 * c, r);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 16; ++i) s[u][16 * c + i] = __uint_as_float(r[i]) * qf_uniform;
@@ -594,13 +601,13 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 } else {
                     // columns h (term 1) and RP + h (term 2), 8 heads at a time
 #pragma unroll
-                    for (int c = 0; c < RP / 8; ++c) {
+                    for (int c = 0; c < HW / 8; ++c) {
                         uint32_t r1[8], r2[8];
-                        tc::tmem_ld8(ta + 8 * c, r1);
-                        tc::tmem_ld8(ta + RP + 8 * c, r2);
+                        tc::tmem_ld8(ta + h0 + 8 * c, r1);
+                        tc::tmem_ld8(ta + RP + h0 + 8 * c, r2);
                         tc::tmem_wait_ld();
-                        const float4 qa = *reinterpret_cast<const float4*>(&X->qscale[qcur][8 * c]);
-                        const float4 qb = *reinterpret_cast<const float4*>(&X->qscale[qcur][8 * c + 4]);
+                        const float4 qa = *reinterpret_cast<const float4*>(&X->qscale[qcur][h0 + 8 * c]);
+                        const float4 qb = *reinterpret_cast<const float4*>(&X->qscale[qcur][h0 + 8 * c + 4]);
                         const float qsc[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
@@ -614,8 +621,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
                 const bool valid = tok < kTile * n_of[u] && tile_of[u] * kTile + tok < w.L;
 #pragma unroll
-                for (int h = 0; h < RP; ++h)
-                    if (!valid || h >= a.R) s[u][h] = NEG_INF;
+                for (int h = 0; h < HW; ++h)
+                    if (!valid || h0 + h >= a.R) s[u][h] = NEG_INF;
             }
             if (!ok) break;
 
@@ -628,17 +635,17 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             for (int u = 0; u < MS; ++u)
                 if (u < nsub) {
 #pragma unroll
-                    for (int h = 0; h < RP; ++h) exceed |= s[u][h] > m[h] + static_cast<float>(C::T_LAZY);
+                    for (int h = 0; h < HW; ++h) exceed |= s[u][h] > m[h] + static_cast<float>(C::T_LAZY);
                 }
-            float p[MS][RP];
+            float p[MS][HW];
             {
                 const uint32_t xb = xpar;
                 const bool any = __any_sync(0xffffffffu, exceed);
-                if (lane == 0) X->flags[xb][sp] = any ? 1 : 0;
+                if (lane == 0) X->flags[xb][wi] = any ? 1 : 0;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->xch));
 #pragma unroll
-                for (int h = 0; h < RP; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     const float ref = m[h] == NEG_INF ? 0.f : m[h];
 #pragma unroll
                     for (int u = 0; u < MS; ++u) p[u][h] = u < nsub ? fast_exp2(s[u][h] - ref) : 0.f;
@@ -646,11 +653,14 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 const bool xok = mbar_wait_warp(smem_addr(&ctrl->xch), xpar, abort_flag);
                 xpar ^= 1u;
                 if (!xok) { ok = false; break; }
-                const bool slow = (X->flags[xb][0] | X->flags[xb][1] | X->flags[xb][2] | X->flags[xb][3]) != 0;
-                if (slow) {
-                    float mx[RP];
+                int any_flag = 0;
 #pragma unroll
-                    for (int h = 0; h < RP; ++h) {
+                for (int k = 0; k < C::NSM; ++k) any_flag |= X->flags[xb][k];
+                const bool slow = any_flag != 0;
+                if (slow) {
+                    float mx[HW];
+#pragma unroll
+                    for (int h = 0; h < HW; ++h) {
                         float v = s[0][h];
                         if (MS > 1 && nsub > 1) v = fmaxf(v, s[MS - 1][h]);
 #pragma unroll
@@ -660,17 +670,17 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     const uint32_t xb2 = xpar;
                     if (lane == 0) {
 #pragma unroll
-                        for (int h = 0; h < RP; h += 4)
-                            *reinterpret_cast<float4*>(&X->vals[xb2][sp][h]) =
+                        for (int h = 0; h < HW; h += 4)
+                            *reinterpret_cast<float4*>(&X->vals[xb2][sp][h0 + h]) =
                                 make_float4(mx[h], mx[h + 1], mx[h + 2], mx[h + 3]);
                     }
                     if (!exchange()) { ok = false; break; }
-                    float alpha[RP];
+                    float alpha[HW];
                     bool moved = false;
 #pragma unroll
-                    for (int h = 0; h < RP; ++h) {
-                        const float M = fmaxf(fmaxf(X->vals[xb2][0][h], X->vals[xb2][1][h]),
-                                              fmaxf(X->vals[xb2][2][h], X->vals[xb2][3][h]));
+                    for (int h = 0; h < HW; ++h) {
+                        const float M = fmaxf(fmaxf(X->vals[xb2][0][h0 + h], X->vals[xb2][1][h0 + h]),
+                                              fmaxf(X->vals[xb2][2][h0 + h], X->vals[xb2][3][h0 + h]));
                         alpha[h] = 1.f;
                         if (M > m[h] + static_cast<float>(C::T_LAZY)) {
                             alpha[h] = m[h] == NEG_INF ? 0.f : fast_exp2(m[h] - M);
@@ -692,16 +702,18 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         }
                         tc::fence_after_sync();
 #pragma unroll
-                        for (int c = 0; c < C::NO_COLS / 8; ++c) {
-                            const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + 8 * c);
-                            uint32_t r[8];
-                            tc::tmem_ld8(oa, r);
-                            tc::tmem_wait_ld();
+                        for (int k = 0; k < C::NPT; ++k)
 #pragma unroll
-                            for (int e = 0; e < 8; ++e)
-                                r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha[(8 * c + e) % RP]);
-                            tc::tmem_st8(oa, r);
-                        }
+                            for (int c = 0; c < HW / 8; ++c) {
+                                const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + k * RP + h0 + 8 * c);
+                                uint32_t r[8];
+                                tc::tmem_ld8(oa, r);
+                                tc::tmem_wait_ld();
+#pragma unroll
+                                for (int e = 0; e < 8; ++e)
+                                    r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha[8 * c + e]);
+                                tc::tmem_st8(oa, r);
+                            }
                         tc::tmem_wait_st();
                     }
                 }
@@ -709,7 +721,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 
             // ---- row sums, P^T for each step's value product
 #pragma unroll
-            for (int h = 0; h < RP; ++h)
+            for (int h = 0; h < HW; ++h)
 #pragma unroll
                 for (int u = 0; u < MS; ++u) l[h] += p[u][h];
 #pragma unroll
@@ -725,15 +737,15 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 if constexpr (KV8) {
                     // p = t1 + t2 / 16 + t3 / 256 + t4 / 4096, each term E4M3 (p <= 2^8 < 448);
                     // columns are [t1 | t2 | t3 | t4], RP heads each.
-                    uint32_t wd[RP];  // term k, heads 4i..4i+3 -> wd[k * RP / 4 + i]
+                    uint32_t wd[HW];  // term k, heads 4i..4i+3 -> wd[k * HW / 4 + i]
 #pragma unroll
-                    for (int i = 0; i < RP / 4; ++i) {
+                    for (int i = 0; i < HW / 4; ++i) {
                         float x0 = p[u][4 * i], x1 = p[u][4 * i + 1], x2 = p[u][4 * i + 2], x3 = p[u][4 * i + 3];
 #pragma unroll
                         for (int k = 0; k < 4; ++k) {
                             const uint16_t b01 = f32x2_to_e4m3x2(x0, x1);
                             const uint16_t b23 = f32x2_to_e4m3x2(x2, x3);
-                            wd[k * (RP / 4) + i] = static_cast<uint32_t>(b01) | (static_cast<uint32_t>(b23) << 16);
+                            wd[k * (HW / 4) + i] = static_cast<uint32_t>(b01) | (static_cast<uint32_t>(b23) << 16);
                             if (k < 3) {
                                 const float2 f01 = e4m3x2_to_f32x2(b01), f23 = e4m3x2_to_f32x2(b23);
                                 x0 = (x0 - f01.x) * 16.f;
@@ -743,23 +755,36 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                             }
                         }
                     }
+                    if constexpr (HW >= 16) {
+                        // term k: columns k RP + h0 .. + HW, whole 16-column groups
 #pragma unroll
-                    for (int g = 0; g < RP / 4; ++g)
-                        st_shared_v4(pt + g * C::P_SBO, wd[4 * g], wd[4 * g + 1], wd[4 * g + 2], wd[4 * g + 3]);
+                        for (int k = 0; k < 4; ++k)
+#pragma unroll
+                            for (int gg = 0; gg < HW / 16; ++gg) {
+                                const int w0 = k * (HW / 4) + 4 * gg;
+                                st_shared_v4(pt + ((k * RP + h0) / 16 + gg) * C::P_SBO, wd[w0], wd[w0 + 1],
+                                             wd[w0 + 2], wd[w0 + 3]);
+                            }
+                    } else {
+                        // eight columns per term: two terms per 16-column group
+#pragma unroll
+                        for (int g = 0; g < HW / 4; ++g)
+                            st_shared_v4(pt + g * C::P_SBO, wd[4 * g], wd[4 * g + 1], wd[4 * g + 2], wd[4 * g + 3]);
+                    }
                 } else {
 #pragma unroll
-                    for (int g = 0; g < RP / 8; ++g) {
+                    for (int g = 0; g < HW / 8; ++g) {
                         uint32_t hw[4], lw[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
                             split_pair<false>(p[u][8 * g + 2 * e], p[u][8 * g + 2 * e + 1], hw[e], lw[e]);
-                        st_shared_v4(pt + g * C::P_SBO, hw[0], hw[1], hw[2], hw[3]);
-                        st_shared_v4(pt + (g + RP / 8) * C::P_SBO, lw[0], lw[1], lw[2], lw[3]);
+                        st_shared_v4(pt + (h0 / 8 + g) * C::P_SBO, hw[0], hw[1], hw[2], hw[3]);
+                        st_shared_v4(pt + ((RP + h0) / 8 + g) * C::P_SBO, lw[0], lw[1], lw[2], lw[3]);
                     }
                 }
                 // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
                 const bool loaded = tok < kTile * n_of[u];
-                if (tile_of[u] + n_of[u] == w.n_b && loaded && tile_of[u] * kTile + tok >= w.L) {
+                if (h0 == 0 && tile_of[u] + n_of[u] == w.n_b && loaded && tile_of[u] * kTile + tok >= w.L) {
                     const int stu = (st + u) % NS;
                     const uint32_t vrow = stages + stu * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
 #pragma unroll
@@ -776,9 +801,9 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 
             if (seg_last) {
                 // ---------------------------------------------------- segment end
-                float lt[RP];
+                float lt[HW];
 #pragma unroll
-                for (int h = 0; h < RP; ++h) {
+                for (int h = 0; h < HW; ++h) {
                     float v = l[h];
 #pragma unroll
                     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -787,14 +812,15 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 const uint32_t xb3 = xpar;
                 if (lane == 0) {
 #pragma unroll
-                    for (int h = 0; h < RP; h += 4)
-                        *reinterpret_cast<float4*>(&X->vals[xb3][sp][h]) =
+                    for (int h = 0; h < HW; h += 4)
+                        *reinterpret_cast<float4*>(&X->vals[xb3][sp][h0 + h]) =
                             make_float4(lt[h], lt[h + 1], lt[h + 2], lt[h + 3]);
                 }
                 if (!exchange()) { ok = false; break; }
 #pragma unroll
-                for (int h = 0; h < RP; ++h)
-                    lt[h] = (X->vals[xb3][0][h] + X->vals[xb3][1][h]) + (X->vals[xb3][2][h] + X->vals[xb3][3][h]);
+                for (int h = 0; h < HW; ++h)
+                    lt[h] = (X->vals[xb3][0][h0 + h] + X->vals[xb3][1][h0 + h]) +
+                            (X->vals[xb3][2][h0 + h] + X->vals[xb3][3][h0 + h]);
                 if (!mbar_wait_warp(smem_addr(&ctrl->ofull), static_cast<uint32_t>(seg) & 1u, abort_flag)) {
                     ok = false;
                     break;
@@ -804,12 +830,12 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 const bool whole = (seg_start_tile == 0) && last_of_unit;
                 const int64_t slot = 2 * static_cast<int64_t>(blockIdx.x) + (seg == 0 ? 0 : 1);
 #pragma unroll
-                for (int c = 0; c < RP / 8; ++c) {
+                for (int c = 0; c < HW / 8; ++c) {
                     // the P terms' columns: hi + lo, or t1 + t2 / 16 + t3 / 256 + t4 / 4096
                     float acc[8];
                     {
                         uint32_t tv[8];
-                        tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + 8 * c), tv);
+                        tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + h0 + 8 * c), tv);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 8; ++e) acc[e] = __uint_as_float(tv[e]);
@@ -817,7 +843,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
 #pragma unroll
                     for (int k = C::NPT - 1; k >= 1; --k) {
                         uint32_t tv[8];
-                        tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + k * RP + 8 * c), tv);
+                        tc::tmem_ld8(tc::tmem_addr(tmem, 32 * sp, C::O_COL + k * RP + h0 + 8 * c), tv);
                         tc::tmem_wait_ld();
                         const float wk = KV8 ? 1.f / static_cast<float>(1 << (4 * k)) : 1.f;
 #pragma unroll
@@ -825,9 +851,9 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     }
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int h = 8 * c + e;
+                        const int hl = 8 * c + e, h = h0 + hl;
                         if (h >= a.R) continue;
-                        const float o = acc[e] * (vfac / lt[h]);
+                        const float o = acc[e] * (vfac / lt[hl]);
                         if (whole) {
                             const int64_t i = (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R + h) * C::D + d;
                             if constexpr (OUT_BF16)
@@ -841,8 +867,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 }
                 if (!whole && sp == 0 && lane == 0) {
 #pragma unroll
-                    for (int h = 0; h < RP; ++h)
-                        if (h < a.R) a.ws_lse[slot * a.R + h] = m[h] + log2f(lt[h]);
+                    for (int h = 0; h < HW; ++h)
+                        if (h0 + h < a.R) a.ws_lse[slot * a.R + h0 + h] = m[h] + log2f(lt[h]);
                 }
                 tc::fence_before_sync();
                 __syncwarp();

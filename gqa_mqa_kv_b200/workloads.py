@@ -84,6 +84,7 @@ WORKLOADS: dict[str, Workload] = {
         _wl("sweep_hkv32", 32, 32, 32, 128, 8192, 3),
         _wl("sweep_hkv8", 32, 32, 8, 128, 8192, 3),
         _wl("sweep_hkv4", 32, 32, 4, 128, 8192, 3),
+        _wl("sweep_hkv2", 32, 32, 2, 128, 8192, 3),
         _wl("sweep_hkv1", 32, 32, 1, 128, 8192, 3),
         _wl("llama2_70b_ragged", 32, 64, 8, 128, 32768, 4, ragged=True),
         _wl("paged_long", 8, 64, 8, 128, 131072, 5, page_size=PAGE_SIZE),

@@ -71,8 +71,9 @@ typedef enum gqa_rope_pairing {
 
 /* Which split kernel serves a call (both compute the same result). */
 typedef enum gqa_kernel {
-    GQA_KERNEL_AUTO = 0,     /* tcgen05 for 8-bit caches (head_dim 128, R <= 32), mma.sync for bf16
-                                (R <= 64), CUDA cores otherwise */
+    GQA_KERNEL_AUTO = 0,     /* head_dim 128: tcgen05 for 8-bit caches (R <= 32) and for bf16 with
+                                17 <= R <= 32; mma.sync for the other bf16 groups (R <= 64);
+                                CUDA cores otherwise */
     GQA_KERNEL_MMA_SYNC = 1, /* warp-level mma.sync kernel: bf16 cache with R <= 64, or an 8-bit
                                 cache with head_dim 128 and R <= 8 */
     GQA_KERNEL_TCGEN05 = 2   /* tcgen05 / tensor-memory kernel: head_dim 128, R <= 32, bf16 query,

@@ -57,9 +57,10 @@ def test_fp8_paged_equals_contiguous_bitwise(cuda_device, out_dtype):
     assert_parity(paged, ref_fp8(inp, w), "fp8 paged")
 
 
-@pytest.mark.parametrize("h_q,h_kv,d", [(32, 8, 128), (64, 4, 128), (16, 4, 64), (8, 1, 64)])
+@pytest.mark.parametrize("h_q,h_kv,d", [(32, 8, 128), (64, 4, 128), (64, 2, 128), (32, 1, 128), (24, 1, 128),
+                                        (16, 4, 64), (8, 1, 64), (64, 1, 128)])
 def test_fp8_group_shapes(cuda_device, h_q, h_kv, d):
-    """R <= 8 at head_dim 128 runs on tensor cores; the rest on the CUDA-core kernel."""
+    """R <= 32 at head_dim 128 runs on the tcgen05 kernel; the rest on CUDA cores."""
     w = dataclasses.replace(WORKLOADS["llama2_70b_ragged_fp8"], name="shape", B=3, H_Q=h_q, H_KV=h_kv,
                             D=d, seq_len=700)
     inp = make_inputs(w)

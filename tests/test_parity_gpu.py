@@ -60,7 +60,7 @@ def test_llama3_8b_full_size(cuda_device):
     assert_parity(run_gpu(inp, w, cuda_device), oracle_full(inp, w), "llama3_8b")
 
 
-@pytest.mark.parametrize("h_kv", [32, 8, 4, 1])
+@pytest.mark.parametrize("h_kv", [32, 8, 4, 2, 1])
 def test_grouping_sweep_reduced(cuda_device, h_kv):
     w = small(f"sweep_hkv{h_kv}", B=4, seq_len=1000)  # 15 full tiles + a 40-token tail
     inp = make_inputs(w)
