@@ -469,7 +469,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         // ------------------------------------------------------------ softmax + epilogue
         const int sp = warp & 3;            // tensor-memory sub-partition of this warp
         const int wi = warp - C::WARP_SM0;  // softmax warp index
-        const int h0 = (wi >> 2) * C::HW;   // first query column of this warp
+        const int h0 = C::HSPLIT == 1 ? 0 : (wi >> 2) * C::HW;  // first query column of this warp
         const int tok = 32 * sp + lane;     // S^T row (token of the step) held by this thread
         constexpr int HW = C::HW;
         const float NEG_INF = -__int_as_float(0x7f800000);
