@@ -1,4 +1,4 @@
-"""TEST INFRASTRUCTURE -- the fp64 CPU oracle for single-token GQA decode.
+"""TEST INFRASTRUCTURE -- the fp64 CPU oracle for GQA decode and multi-token (prefill) attention.
 
 Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's
 CPU-baseline / reference arm may import this package.  The product library
@@ -72,6 +72,9 @@ def _load():
             lib.oracle_e4m3_table.argtypes = [vp]
             lib.oracle_e4m3_table.restype = None
             lib.oracle_rope.restype = i32
+            lib.oracle_gqa_prefill.argtypes = [vp, i32, vp, vp, i32, vp, vp, i32, i32, i32, i32, i64,
+                                               dbl, vp, i64, vp, i32]
+            lib.oracle_gqa_prefill.restype = i32
             lib.oracle_hardware_threads.argtypes = []
             lib.oracle_hardware_threads.restype = i32
             _lib = lib
@@ -150,6 +153,40 @@ def gqa_decode(q, k, v, seq_lens, scale, pairs=None, n_threads=0):
                                    D, S_max, float(scale), pp, n, _ptr(out), int(n_threads))
     if rc != 0:
         raise ValueError("oracle_gqa_decode rejected its arguments")
+    return out
+
+
+def gqa_prefill(q, k, v, seq_lens, cu_q, scale, rows=None, n_threads=0):
+    """fp64 multi-token causal attention.
+
+    q [total_q, H_Q, D] (rows cu_q[b] .. cu_q[b+1]-1 belong to sequence b);
+    k, v [B, S_max, H_KV, D] logical contiguous cache; seq_lens [B]; cu_q [B+1].
+    Query row j of sequence b sits at position seq_lens[b] - n_b + j and sees
+    cache positions t <= that position.  Returns float64 [total_q, H_Q, D], or
+    [n, D] for an explicit list of (row, head) pairs.
+    """
+    qa, qt = _as_array(q)
+    ka, kt = _as_array(k)
+    va, vt = _as_array(v)
+    if kt != vt:
+        raise TypeError("oracle: k and v must share a dtype")
+    lens = _lens(seq_lens)
+    cu = _lens(cu_q)
+    T, H_Q, D = qa.shape
+    B, S_max, H_KV, Dk = ka.shape
+    if Dk != D or va.shape != ka.shape or lens.shape != (B,) or cu.shape != (B + 1,) or int(cu[-1]) != T:
+        raise ValueError("oracle: inconsistent shapes")
+    if rows is None:
+        out = np.zeros((T, H_Q, D), dtype=np.float64)
+        rp, n = None, 0
+    else:
+        ra = np.ascontiguousarray(np.asarray(rows, dtype=np.int32).reshape(-1, 2))
+        out = np.zeros((ra.shape[0], D), dtype=np.float64)
+        rp, n = _ptr(ra), ra.shape[0]
+    rc = _load().oracle_gqa_prefill(_ptr(qa), qt, _ptr(ka), _ptr(va), kt, _ptr(lens), _ptr(cu), B, H_Q,
+                                    H_KV, D, S_max, float(scale), rp, n, _ptr(out), int(n_threads))
+    if rc != 0:
+        raise ValueError("oracle_gqa_prefill rejected its arguments")
     return out
 
 

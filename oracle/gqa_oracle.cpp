@@ -39,10 +39,23 @@
 // o_T = sum_{t in T} exp(s_t - lse_T) v_t; merging ranges T_1..T_n gives
 // out = sum_j exp(lse_j - LSE) o_j with LSE = log sum_j exp(lse_j).
 //
+// Multi-token step (prefill, or a chunk of a prompt after a cached prefix):
+// sequence b brings n_b = cu_q[b+1] - cu_q[b] new query tokens whose keys and
+// values are already the last n_b of its L_b cached tokens.  Its query token
+// j (0-based) therefore sits at position p = L_b - n_b + j, and the causal
+// mask M of [LLMS] section 2 (M[j][t] = 0 for t <= j, -inf after) becomes
+// "key t is visible iff t <= p": the whole cached prefix plus the new tokens
+// up to and including itself.  With no prefix (L_b = n_b) this is the s x s
+// mask as written; with n_b = 1 it is the decode step above.  [LLMS]'s
+// opening section names this prompt-processing phase (prefill) and says it
+// is compute-bound; the arithmetic is the Head_i equation unchanged.
+//
 // Layouts (row-major, innermost last):
-//   q   [B, H_Q, D]
+//   q   [B, H_Q, D]                  decode; [total_q, H_Q, D] multi-token,
+//                                    rows cu_q[b] .. cu_q[b+1]-1 for sequence b
 //   k,v [B, S_max, H_KV, D]      logical contiguous cache
 //   out [n_pairs, D] in the order of `pairs`, or [B, H_Q, D] when pairs==NULL
+//       (multi-token: [n_rows, D] for `rows`, or [total_q, H_Q, D])
 //
 // Build: g++ -O2 -std=c++17 -shared -fPIC -pthread gqa_oracle.cpp
 
@@ -351,6 +364,74 @@ int oracle_rope(const void* x, int dtype, int B, int H, int D, const int32_t* po
             }
         }
     }
+    return 0;
+}
+
+// Multi-token causal attention (see the header comment): for every listed
+// (query row i, query head h), with b the sequence whose span
+// [cu_q[b], cu_q[b+1]) holds i, j = i - cu_q[b], n_b the span length and
+// p = L_b - n_b + j:
+//     s_t = scale * <q[i,h,:], K[b,t,g,:]>                 for t in [0, p]
+//     out = sum_t softmax(s)_t * V[b,t,g,:]
+// in double, two passes (max, then exp and sum), g = floor(h / R).
+//   cu_q: [B+1], cu_q[0] = 0, non-decreasing, n_b <= L_b for every b.
+//   rows: NULL for every row (out is [cu_q[B], H_Q, D]); else n_rows pairs
+//         (i, h) and out is [n_rows, D].
+// Returns 0, or 1 on invalid arguments (nothing written).
+int oracle_gqa_prefill(const void* q, int q_dtype, const void* k, const void* v, int kv_dtype,
+                       const int32_t* seq_lens, const int32_t* cu_q, int B, int H_Q, int H_KV, int D,
+                       int64_t S_max, double scale, const int32_t* rows, int64_t n_rows, double* out,
+                       int n_threads) {
+    Problem p{q, k, v, q_dtype, kv_dtype, seq_lens, B, H_Q, H_KV, D, S_max, scale};
+    if (check_problem(p) || !out || !cu_q || cu_q[0] != 0) return 1;
+    for (int b = 0; b < B; ++b) {
+        const int n_b = cu_q[b + 1] - cu_q[b];
+        if (n_b < 0 || n_b > seq_lens[b]) return 1;
+    }
+    const int64_t total = cu_q[B];
+    const int64_t n = rows ? n_rows : total * H_Q;
+    if (n < 0) return 1;
+    if (rows) {
+        for (int64_t r = 0; r < n; ++r)
+            if (rows[2 * r] < 0 || rows[2 * r] >= total || rows[2 * r + 1] < 0 || rows[2 * r + 1] >= H_Q)
+                return 1;
+    }
+    auto one = [&](int64_t i, int h, double* o) {
+        int b = 0;
+        while (cu_q[b + 1] <= i) ++b;  // the span holding row i (spans are non-empty here)
+        const int64_t n_b = cu_q[b + 1] - cu_q[b];
+        const int64_t pos = seq_lens[b] - n_b + (i - cu_q[b]);
+        const int g = group_of(p, h);
+        std::vector<double> s(static_cast<size_t>(pos + 1));
+        double m = -std::numeric_limits<double>::infinity();
+        for (int64_t t = 0; t <= pos; ++t) {
+            double acc = 0.0;
+            for (int e = 0; e < D; ++e)
+                acc += load_elem(q, q_dtype, (i * H_Q + h) * D + e) * load_elem(k, kv_dtype, kv_index(p, b, t, g, e));
+            s[t] = scale * acc;
+            if (s[t] > m) m = s[t];
+        }
+        double sum = 0.0;
+        for (int64_t t = 0; t <= pos; ++t) {
+            s[t] = std::exp(s[t] - m);
+            sum += s[t];
+        }
+        for (int e = 0; e < D; ++e) o[e] = 0.0;
+        for (int64_t t = 0; t <= pos; ++t)
+            for (int e = 0; e < D; ++e) o[e] += (s[t] / sum) * load_elem(v, kv_dtype, kv_index(p, b, t, g, e));
+    };
+    int nt = thread_count(n_threads, n);
+    std::vector<std::thread> pool;
+    for (int w = 0; w < nt; ++w) {
+        pool.emplace_back([&, w]() {
+            for (int64_t r = w; r < n; r += nt) {
+                const int64_t i = rows ? rows[2 * r] : r / H_Q;
+                const int h = rows ? rows[2 * r + 1] : static_cast<int>(r % H_Q);
+                one(i, h, out + r * D);
+            }
+        });
+    }
+    for (auto& t : pool) t.join();
     return 0;
 }
 

@@ -39,11 +39,19 @@ MUTANTS = {
     "e4m3_bias": ("        mag = std::ldexp(1.0 + m / 8.0, e - 7);", "        mag = std::ldexp(1.0 + m / 8.0, e - 8);"),
     "e4m3_subnormal": ("        mag = std::ldexp(static_cast<double>(m), -9);", "        mag = std::ldexp(static_cast<double>(m), -10);"),
     "value_scale_dropped": ("    const double vs = p.v_scale ? p.v_scale[g] : 1.0;", "    const double vs = 1.0;"),
+    "prefill_ignores_prefix": ("        const int64_t pos = seq_lens[b] - n_b + (i - cu_q[b]);",
+                               "        const int64_t pos = i - cu_q[b];"),
+    "prefill_sees_next_key": ("        const int64_t pos = seq_lens[b] - n_b + (i - cu_q[b]);",
+                              "        const int64_t pos = seq_lens[b] - n_b + (i - cu_q[b]) + 1;"),
+    "prefill_span_lookup": ("        while (cu_q[b + 1] <= i) ++b;", "        while (cu_q[b + 1] < i) ++b;"),
+    "prefill_query_layout": ("load_elem(q, q_dtype, (i * H_Q + h) * D + e)",
+                             "load_elem(q, q_dtype, (h * cu_q[B] + i) * D + e)"),
     "rope_pairing": ("                const int i1 = pairing == 0 ? 2 * i + 1 : i + half;",
                      "                const int i1 = pairing == 0 ? 2 * i + 1 : i + half - 1;"),
 }
 
-PIN_SUITES = ["tests/test_oracle_pins.py", "tests/test_oracle_rope_pins.py", "tests/test_oracle_fp8_pins.py"]
+PIN_SUITES = ["tests/test_oracle_pins.py", "tests/test_oracle_rope_pins.py", "tests/test_oracle_fp8_pins.py",
+              "tests/test_oracle_prefill_pins.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
