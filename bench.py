@@ -37,10 +37,13 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
-from gqa_mqa_kv_b200.workloads import WORKLOADS, algorithmic_bytes, make_inputs  # noqa: E402
+from gqa_mqa_kv_b200.workloads import (PREFILL_WORKLOADS, WORKLOADS, algorithmic_bytes,  # noqa: E402
+                                       make_inputs, make_prefill_inputs, prefill_flops, prefill_lengths)
 
 METRIC = "decode-attention achieved HBM GB/s (% of B200 peak) and µs per decode step"
+PREFILL_METRIC = "prefill-attention achieved TFLOP/s (causal, algorithmic 4 d per visible query-head/key pair) and µs per step"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -52,7 +55,8 @@ def parse_args(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3000)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="llama2_70b_ragged", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="llama2_70b_ragged", choices=sorted(WORKLOADS) + sorted(PREFILL_WORKLOADS),
+                    help="a decode workload, or a multi-token (prefill) workload: prefill_*")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--soak-seconds", type=float, default=1.5,
                     help="untimed steps before the timed region so clocks settle and are sampled")
@@ -105,6 +109,16 @@ def hbm_peak():
         return v, "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 TFLOP/s: the burst figure (a kernel timed alone)."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 class ClockSampler:
@@ -484,11 +498,193 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------- multi-token (prefill) steps
+
+def prefill_config(w, n):
+    return {"workload": w.name, "B": w.B, "H_Q": w.H_Q, "H_KV": w.H_KV, "head_dim": w.D,
+            "q_len": w.q_len, "prefix": w.prefix, "ragged": w.ragged, "page_size": w.page_size,
+            "kv_dtype": "bf16", "out_dtype": "bf16", "global_batch": w.B * n,
+            "l2": "L2 flushed before every step (256 MiB written)",
+            "parallelism": f"dp{n} (independent batch per GPU, no collective)"}
+
+
+def cpu_oracle_prefill_sample(w, inp, seconds: float):
+    """Time the fp64 oracle on the last query tokens of sequence 0 (all query
+    heads; the tokens that see the most keys), sized to about `seconds`."""
+    import numpy as np
+
+    import oracle
+
+    n, lens = prefill_lengths(w)
+    cu = inp["cu_q"].numpy()
+    threads = oracle.hardware_threads()
+
+    def rows_for(count):
+        lo = int(cu[1]) - count
+        return [(i, h) for i in range(lo, int(cu[1])) for h in range(w.H_Q)]
+
+    def run(count):
+        t0 = time.perf_counter()
+        oracle.gqa_prefill(inp["q"], inp["k"], inp["v"], inp["seq_lens"], inp["cu_q"], w.softmax_scale,
+                           rows=rows_for(count))
+        return time.perf_counter() - t0
+
+    per_tok = max(run(1), 1e-6)
+    count = int(max(1, min(int(n[0]), seconds / per_tok)))
+    dt = run(count)
+    first = int(lens[0]) - count + 1  # keys seen by the first sampled token
+    pairs = count * first + count * (count - 1) // 2
+    flops = 4 * w.D * w.H_Q * pairs
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "sample": f"last {count} query tokens of sequence 0 (all {w.H_Q} query heads, "
+                      f"{first}..{int(lens[0])} visible keys each), fp64, {dt:.2f} s",
+            "seconds": dt}
+
+
+def run_reference_prefill(args):
+    world, rank, _ = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    w = PREFILL_WORKLOADS[args.workload]
+    inp = make_prefill_inputs(w)
+    t_start = time.perf_counter()
+    results = [cpu_oracle_prefill_sample(w, inp, args.cpu_sample_seconds / max(args.steps, 1))
+               for _ in range(args.steps)]
+    total = time.perf_counter() - t_start
+    value = statistics.median(r["value"] for r in results)
+    last = results[-1]
+    print(json.dumps({
+        "impl": "reference", "metric": PREFILL_METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": total * 1e3 / max(args.steps, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": prefill_config(w, args.gpus),
+        "cpu_baseline": {k: last[k] for k in ("kind", "cores", "sample")} | {"value": value, "unit": "TFLOP/s"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+    return 0
+
+
+def run_ours_prefill(args):
+    import gqa_mqa_kv_b200 as gq
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    w = PREFILL_WORKLOADS[args.workload]
+    inp = make_prefill_inputs(w)
+    n, lens_np = prefill_lengths(w)
+    flops = prefill_flops(w, n, lens_np)
+    paged = bool(w.page_size)
+    q = inp["q"].to(dev)
+    k = (inp["k_paged"] if paged else inp["k"]).to(dev)
+    v = (inp["v_paged"] if paged else inp["v"]).to(dev)
+    lens = inp["seq_lens"].to(dev)
+    cu = inp["cu_q"].to(dev)
+    table = inp["block_table"].to(dev) if paged else None
+    max_q = inp["max_q"]
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def call():
+        gq.gqa_prefill(q, k, v, lens, cu, max_q_len=max_q, block_table=table, scale=w.softmax_scale, out=out,
+                       workspace=ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        flush.zero_()
+        call()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(dev) as clocks:
+        t_soak = time.perf_counter()
+        while time.perf_counter() - t_soak < args.soak_seconds:
+            for _ in range(5):
+                flush.zero_()
+                call()
+            torch.cuda.synchronize(dev)
+        # ------------------------------------------------ timed region: K steps, L2 flushed between
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            evs[i][0].record(stream)
+            call()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+        if dist is not None:
+            dist.barrier()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    elapsed_ms = max_over_ranks(sum(step_ms), dist, dev)
+    kernel_ms = max_over_ranks(statistics.mean(step_ms), dist, dev)
+    status = gq.read_status(ws)
+
+    # ---------------------------------------------------- end to end through the public API
+    q_host = inp["q"].pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = q_host.numel() * q_host.element_size()
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        q.copy_(q_host, non_blocking=True)
+        call()
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if dist is not None:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_steps = max(1, min(args.e2e_steps, 20))
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dist, dev) / e2e_steps
+
+    peak, peak_kind = tensor_peak()
+    ms_per_step = elapsed_ms / args.steps
+    achieved = flops / (kernel_ms * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": world * flops / (ms_per_step * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "us_per_step": ms_per_step * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic", "config": prefill_config(w, world),
+        "algorithmic_flops_per_step_per_gpu": flops,
+        "clocks": clocks.summary(),
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s", "us_per_step": e2e_ms * 1e3,
+                "h2d_bytes_per_step": world * h2d, "d2h_bytes_per_step": world * d2h,
+                "path": "pinned q copied in, gqa_prefill, out copied back, every step; KV cache resident in HBM"},
+        "gpu_launches": args.steps,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(w.name),
+                     "kernel": "prefill_tc_kernel (the whole call)", "kernel_us": kernel_ms * 1e3,
+                     "peak_note": f"{peak_kind} dense bf16 GEMM TFLOP/s (burst)",
+                     "tensor_work_note": "the value product runs twice (bf16 hi and lo parts of P): "
+                                         "tensor-core work is 1.5x the algorithmic FLOPs"},
+        "device_status_flags": status,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_prefill_sample(w, inp, args.cpu_sample_seconds)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
+    prefill = args.workload in PREFILL_WORKLOADS
     if args.impl == "reference":
-        return run_reference(args)
-    return run_ours(args)
+        return run_reference_prefill(args) if prefill else run_reference(args)
+    return run_ours_prefill(args) if prefill else run_ours(args)
 
 
 if __name__ == "__main__":

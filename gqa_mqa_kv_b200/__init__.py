@@ -1,4 +1,4 @@
-"""B200-native grouped-query attention (GQA) decode.
+"""B200-native grouped-query attention (GQA): decode and multi-token (prefill) steps.
 
 A thin ctypes binding over ``libgqa_decode.so`` (the C ABI in
 ``include/gqa_decode.h``).  Every step of the computation runs in the
@@ -23,7 +23,7 @@ import threading
 
 __all__ = [
     "GqaError", "Params", "gqa_decode", "gqa_decode_timed", "gqa_decode_static_workspace",
-    "gqa_rope_append", "gqa_decode_fp8kv", "FLAG_BAD_POSITION",
+    "gqa_rope_append", "gqa_decode_fp8kv", "gqa_prefill", "FLAG_BAD_POSITION", "FLAG_BAD_QUERY_SPAN",
     "workspace_bytes", "make_workspace",
     "read_status", "kv_cache_bytes", "library", "LIB_PATH", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_BAD_BLOCK", "FLAG_TIMEOUT", "PAGE_SIZE",
@@ -34,13 +34,14 @@ PAGE_SIZE = 64
 GQA_BF16, GQA_F32 = 0, 1
 # gqa_kernel: which split kernel serves a call (all compute the same result)
 KERNELS = {"auto": 0, "mma_sync": 1, "tcgen05": 2}
-FLAG_SEQ_LEN_CLAMPED, FLAG_BAD_BLOCK, FLAG_TIMEOUT, FLAG_BAD_POSITION = 1, 2, 4, 8
+FLAG_SEQ_LEN_CLAMPED, FLAG_BAD_BLOCK, FLAG_TIMEOUT, FLAG_BAD_POSITION, FLAG_BAD_QUERY_SPAN = 1, 2, 4, 8, 16
 ROPE_PAIRING = {"adjacent": 0, "halves": 1}
 
 EXPORTED = (
     "gqa_decode_workspace_size", "gqa_decode", "gqa_decode_timed", "gqa_read_status",
     "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version", "gqa_decode_static_workspace",
-    "gqa_rope_append", "gqa_decode_fp8kv", "gqa_wait_selftest",
+    "gqa_rope_append", "gqa_decode_fp8kv", "gqa_wait_selftest", "gqa_prefill_workspace_size",
+    "gqa_prefill",
 )
 
 
@@ -105,6 +106,11 @@ def library() -> ctypes.CDLL:
             lib.gqa_decode_fp8kv.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, ctypes.c_float, vp, vp, sz,
                                              vp]
             lib.gqa_decode_fp8kv.restype = ctypes.c_int
+            lib.gqa_prefill_workspace_size.argtypes = [pp, ctypes.POINTER(sz)]
+            lib.gqa_prefill_workspace_size.restype = ctypes.c_int
+            lib.gqa_prefill.argtypes = [pp, vp, vp, ctypes.c_int32, ctypes.c_int32, vp, vp, vp, vp,
+                                        ctypes.c_float, vp, vp, sz, vp]
+            lib.gqa_prefill.restype = ctypes.c_int
             lib.gqa_wait_selftest.argtypes = [ctypes.c_uint64, ctypes.c_int, vp, vp, vp]
             lib.gqa_wait_selftest.restype = ctypes.c_int
             _lib = lib
@@ -384,6 +390,68 @@ def gqa_decode_fp8kv(q, k_cache, v_cache, k_scale, v_scale, seq_lens, block_tabl
         ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
     if st != 0:
         raise GqaError(st, "gqa_decode_fp8kv")
+    return out
+
+
+def gqa_prefill(q, k_cache, v_cache, seq_lens, cu_q_lens, max_q_len=None, block_table=None, scale=None,
+                out=None, out_dtype=None, workspace=None, stream=None, max_seq_len=None, kernel="auto"):
+    """Multi-token causal GQA (prefill, or a prompt chunk after a cached prefix) on the GPU.
+
+    q            [total_q, H_Q, 128] bf16: the new query tokens of every
+                 sequence, back to back (rows cu_q_lens[b] .. cu_q_lens[b+1]-1)
+    k_cache,     as in gqa_decode, already holding the new tokens' keys and
+    v_cache      values as the last n_b of each sequence's seq_lens[b] tokens
+    seq_lens     int32 [B]
+    cu_q_lens    int32 [B + 1], cu_q_lens[0] = 0, cu_q_lens[B] = total_q
+    max_q_len    host bound on every n_b (read from cu_q_lens, with a
+                 synchronisation, when not given)
+    Token j of sequence b sits at position seq_lens[b] - n_b + j and attends to
+    cache positions <= it.  Returns out [total_q, H_Q, 128] (f32 default, or
+    bf16), enqueued on ``stream`` (default: the current stream).
+    """
+    import torch
+
+    for name, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("seq_lens", seq_lens),
+                    ("cu_q_lens", cu_q_lens)):
+        if not isinstance(t, torch.Tensor) or not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if q.dim() != 3 or k_cache.dim() != 4:
+        raise ValueError("q must be [total_q, H_Q, D]; caches must be 4-D")
+    if k_cache.shape != v_cache.shape or not (q.dtype == k_cache.dtype == v_cache.dtype):
+        raise ValueError("q and the caches must share a dtype; k_cache and v_cache a shape")
+    B = seq_lens.shape[0]
+    if seq_lens.dtype != torch.int32 or seq_lens.dim() != 1:
+        raise ValueError("seq_lens must be int32 [B]")
+    if cu_q_lens.dtype != torch.int32 or cu_q_lens.shape != (B + 1,):
+        raise ValueError("cu_q_lens must be int32 [B + 1]")
+    if block_table is not None and (not block_table.is_cuda or not block_table.is_contiguous()
+                                    or block_table.dtype != torch.int32):
+        raise ValueError("block_table must be a contiguous int32 CUDA tensor")
+    total_q = q.shape[0]
+    if max_q_len is None:
+        cu = cu_q_lens.cpu()
+        max_q_len = int((cu[1:] - cu[:-1]).max().item()) if B > 0 else 0
+    # gqa_decode_params from the cache geometry; B comes from seq_lens.
+    proxy = torch.empty((B, q.shape[1], q.shape[2]), dtype=q.dtype, device="meta")
+    params = make_params(proxy, k_cache, seq_lens, block_table, out_dtype if out is None else out.dtype,
+                         max_seq_len, kernel)
+    if out is None:
+        out = torch.empty(q.shape, dtype=out_dtype or torch.float32, device=q.device)
+    elif out.shape != q.shape or not out.is_contiguous() or not out.is_cuda:
+        raise ValueError("out must be a contiguous CUDA tensor shaped like q")
+    if workspace is None:
+        workspace = make_workspace(params, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device)
+    opt = lambda t: ctypes.c_void_p(t.data_ptr() if t is not None else None)  # noqa: E731
+    st = library().gqa_prefill(
+        ctypes.byref(params), opt(q), opt(cu_q_lens), int(total_q), int(max_q_len), opt(k_cache), opt(v_cache),
+        opt(seq_lens), opt(block_table), ctypes.c_float(scale), opt(out), opt(workspace),
+        ctypes.c_size_t(workspace.numel()), ctypes.c_void_p(stream.cuda_stream))
+    if st != 0:
+        raise GqaError(st, "gqa_prefill")
     return out
 
 

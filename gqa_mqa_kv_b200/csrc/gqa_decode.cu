@@ -20,6 +20,7 @@
 #include "split_mma.cuh"
 #include "split_simt.cuh"
 #include "split_tc.cuh"
+#include "prefill_tc.cuh"
 #include "rope_append.cuh"
 
 namespace {
@@ -466,6 +467,54 @@ cudaError_t launch_rope(const void* q, const void* k_new, const void* v_new, voi
                           static_cast<T*>(k_cache), static_cast<T*>(v_cache), ra);
 }
 
+// ------------------------------------------------------------------ multi-token (prefill)
+
+template <bool PAGED, bool OUTB>
+cudaError_t launch_prefill(const gqa_decode_params* p, const void* q, const void* k, const void* v,
+                           const PrefillArgs& args, int grid, cudaStream_t stream, bool* encode_ok) {
+    constexpr int D = 128;
+    const uint64_t row = static_cast<uint64_t>(D) * 2;
+    CUtensorMap tmQ, tmK, tmV;
+    {
+        // q [total_q, H_Q, D]: box = 64 d x R heads x TQ tokens, rows token-major
+        const uint64_t dims[3] = {static_cast<uint64_t>(D), static_cast<uint64_t>(p->H_Q),
+                                  static_cast<uint64_t>(args.total_q)};
+        const uint64_t strides[2] = {row, row * p->H_Q};
+        const uint32_t box[3] = {64, static_cast<uint32_t>(args.R), static_cast<uint32_t>(args.TQ)};
+        *encode_ok = encode_map(&tmQ, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, q, 3, dims, strides, box);
+    }
+    if (*encode_ok) {
+        uint64_t dims[4], strides[3];
+        dims[0] = D;
+        dims[1] = p->H_KV;
+        strides[0] = row;
+        strides[1] = row * p->H_KV;
+        if (PAGED) {
+            dims[2] = kTile;
+            dims[3] = p->num_blocks;
+        } else {
+            dims[2] = p->max_seq_len > 0 ? p->max_seq_len : 1;
+            dims[3] = p->B;
+        }
+        strides[2] = strides[1] * dims[2];
+        const uint32_t box4[4] = {64, 1, static_cast<uint32_t>(kTile), 1};
+        *encode_ok = encode_map(&tmK, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, k, 4, dims, strides, box4) &&
+                     encode_map(&tmV, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, v, 4, dims, strides, box4);
+    }
+    if (!*encode_ok) return cudaErrorInvalidValue;
+    auto kernel = prefill_tc_kernel<PAGED, OUTB>;
+    cudaError_t e = ensure_smem(reinterpret_cast<const void*>(kernel), PfCfg::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    // Plain stream order (no early launch): the kernel reads what earlier work wrote.
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(PfCfg::THREADS);
+    cfg.dynamicSmemBytes = PfCfg::SMEM_BYTES;
+    cfg.stream = stream;
+    return cudaLaunchKernelEx(&cfg, kernel, tmQ, tmK, tmV, args);
+}
+
 }  // namespace
 
 namespace {
@@ -603,6 +652,79 @@ gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const
     const cudaError_t e = params->qkv_dtype == GQA_F32
                               ? launch_rope<float>(q, k_new, v_new, q_out, k_cache, v_cache, ra, s)
                               : launch_rope<__nv_bfloat16>(q, k_new, v_new, q_out, k_cache, v_cache, ra, s);
+    return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
+}
+
+gqa_status gqa_prefill_workspace_size(const gqa_decode_params* params, size_t* bytes) {
+    if (bytes == nullptr) return GQA_ERR_INVALID;
+    const gqa_status st = validate_params(params);
+    if (st != GQA_OK) return st;
+    *bytes = kHeaderBytes;
+    return GQA_OK;
+}
+
+gqa_status gqa_prefill(const gqa_decode_params* params, const void* q, const int32_t* cu_q_lens, int32_t total_q,
+                       int32_t max_q_len, const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                       const int32_t* block_table, float scale, void* out, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+    gqa_status st = validate_params(params);
+    if (st != GQA_OK) return st;
+    const gqa_decode_params* p = params;
+    if (p->head_dim != 128 || p->qkv_dtype != GQA_BF16) return GQA_ERR_UNSUPPORTED;
+    if (p->kernel == GQA_KERNEL_MMA_SYNC) return GQA_ERR_UNSUPPORTED;
+    const int R = p->H_Q / p->H_KV;
+    if (R > 128) return GQA_ERR_UNSUPPORTED;  // one tile row per head of a token at least
+    if (total_q < 0 || max_q_len < 0) return GQA_ERR_INVALID;
+    if (p->B == 0 || total_q == 0 || max_q_len == 0) return GQA_OK;
+    if (!q || !cu_q_lens || !k_cache || !v_cache || !seq_lens || !out) return GQA_ERR_INVALID;
+    if ((p->page_size != 0) != (block_table != nullptr)) return GQA_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
+        !aligned(cu_q_lens, 4) || !aligned(seq_lens, 4) || (block_table && !aligned(block_table, 4)))
+        return GQA_ERR_INVALID;
+    if (!(scale == scale)) return GQA_ERR_INVALID;
+    if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < kHeaderBytes) return GQA_ERR_WORKSPACE;
+
+    const int TQ = 128 / R;
+    const int64_t QT = (static_cast<int64_t>(max_q_len) + TQ - 1) / TQ;
+    const int64_t units = static_cast<int64_t>(p->B) * p->H_KV * QT;
+    if (units >= (int64_t(1) << 31)) return GQA_ERR_UNSUPPORTED;
+    DeviceInfo dev;
+    if ((st = device_info(&dev)) != GQA_OK) return st;
+    if (dev.smem_optin < PfCfg::SMEM_BYTES) return GQA_ERR_UNSUPPORTED;
+    const int grid = static_cast<int>(units < dev.sms ? units : dev.sms);
+
+    PrefillArgs args;
+    std::memset(&args, 0, sizeof args);
+    args.seq_lens = seq_lens;
+    args.cu_q = cu_q_lens;
+    args.block_table = block_table;
+    args.B = p->B;
+    args.H_Q = p->H_Q;
+    args.H_KV = p->H_KV;
+    args.R = R;
+    args.TQ = TQ;
+    args.QT = static_cast<int>(QT);
+    args.max_q = max_q_len;
+    args.total_q = total_q;
+    args.max_len = p->max_seq_len;
+    args.S_max = p->page_size ? 0 : p->max_seq_len;
+    args.max_blocks = p->max_blocks_per_seq;
+    args.num_blocks = p->num_blocks;
+    args.sl2 = scale * 1.4426950408889634f;  // log2(e): exponentials are taken base 2
+    args.out = out;
+    args.status = static_cast<uint32_t*>(workspace);
+
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    bool encode_ok = true;
+    const bool outb = p->out_dtype == GQA_BF16;
+    cudaError_t e;
+    if (p->page_size)
+        e = outb ? launch_prefill<true, true>(p, q, k_cache, v_cache, args, grid, s, &encode_ok)
+                 : launch_prefill<true, false>(p, q, k_cache, v_cache, args, grid, s, &encode_ok);
+    else
+        e = outb ? launch_prefill<false, true>(p, q, k_cache, v_cache, args, grid, s, &encode_ok)
+                 : launch_prefill<false, false>(p, q, k_cache, v_cache, args, grid, s, &encode_ok);
+    if (!encode_ok) return GQA_ERR_INVALID;
     return e == cudaSuccess ? GQA_OK : GQA_ERR_CUDA;
 }
 

@@ -1,0 +1,580 @@
+// prefill_tc.cuh -- multi-token (prefill, or a prompt chunk after a cached
+// prefix) grouped-query attention on the tcgen05 tensor cores, head_dim 128.
+//
+// What it computes ("Grouped-Query Attention (GQA) and Multi-Query Attention
+// (MQA): Mathematical Foundations, ...", section 2: Head_i = softmax(Q_i
+// K_{g(i)}^T / sqrt(d_k) + M) V_{g(i)} with the causal mask M; the opening
+// section names prompt processing, prefill, as the compute-bound phase):
+// sequence b brings n_b new query tokens -- rows cu_q[b] .. cu_q[b+1]-1 of q
+// -- whose keys and values are the last n_b of its L_b cached tokens.  Token
+// j sits at position p = L_b - n_b + j and attends to cache positions t <= p.
+//
+// Work unit: TQ = floor(128 / R) consecutive query tokens of one sequence
+// and one KV head kv, as one M = 128 row tile whose row r is token r / R and
+// query head kv R + r % R: every K/V row brought on chip serves all R heads
+// of the group.  The unit walks its visible keys 128 at a time:
+//   S = Q K^T       tcgen05.mma, M = 128 rows, N = 128 keys, K = d: A = the
+//                   query rows, B = the key rows, both K-major with the
+//                   128-byte swizzle as TMA stages them; S lands in tensor
+//                   memory (two buffers: the next step's product overlaps
+//                   this step's softmax).
+//   softmax         four warps, thread = row = TMEM lane, the row's 128
+//                   scores in registers: base-2 online softmax against a
+//                   per-row reference that moves only when a score exceeds
+//                   it by more than 8 (O is rescaled in tensor memory then).
+//                   P goes to shared memory as bf16 hi and lo parts, so the
+//                   product keeps ~16 bits of every weight, in the same
+//                   K-major swizzled layout TMA would produce.
+//   O += P V        tcgen05.mma, M = 128, N = d = 128, K = 128 keys, once on
+//                   the hi part and once on the lo part; B = the value rows
+//                   read MN-major; O in tensor memory (two buffers, one per
+//                   unit in flight), normalised by the row sum at the end.
+//
+// Persistent CTAs (one per SM) walk the units in a fixed interleaved order,
+// heaviest query tiles first.  Warp roles: 0 TMA producer, 1 score products
+// (+ tensor-memory allocation), 2 value products, 3..6 softmax and epilogue
+// (sub-partitions 3, 0, 1, 2).  Every wait is bounded (kWaitTimeoutNs); on a
+// timeout the CTA raises GQA_FLAG_TIMEOUT, lets its copies and products
+// drain, frees its tensor memory and returns.
+#pragma once
+
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+#include "schedule.cuh"
+#include "tcgen05.cuh"
+
+namespace gqa {
+
+struct PrefillArgs {
+    const int32_t* seq_lens;     // [B]
+    const int32_t* cu_q;         // [B + 1]: query rows of sequence b are cu_q[b] .. cu_q[b+1]-1
+    const int32_t* block_table;  // [B, max_blocks] or null
+    int B, H_Q, H_KV, R;
+    int TQ;          // query tokens per tile: floor(128 / R)
+    int QT;          // tiles per sequence: ceil(max_q / TQ)
+    int max_q;       // host bound on n_b
+    int total_q;     // rows of q and out
+    int max_len;     // seq_lens are clamped to [0, max_len]
+    int S_max;       // contiguous cache capacity; 0 when paged
+    int max_blocks, num_blocks;
+    float sl2;       // softmax scale * log2(e)
+    void* out;       // [total_q, H_Q, 128]
+    uint32_t* status;
+};
+
+struct PfCfg {
+    static constexpr int D = 128;
+    static constexpr int BN = 128;                 // keys per step
+    static constexpr int PANEL = 128 * 128;        // 128 rows x 128 bytes (64 bf16 of d, or of keys)
+    static constexpr int TILE = 2 * PANEL;         // 128 rows x 128 bf16
+    static constexpr int BOX = 64 * 128;           // one 64-row TMA box of 128-byte rows
+    static constexpr int NS = 4;                   // K/V ring entries (K and V of a step alternate)
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_P = OFF_Q + TILE;     // P hi, then P lo
+    static constexpr int OFF_RING = OFF_P + 2 * TILE;
+    static constexpr int OFF_CTRL = OFF_RING + NS * TILE;
+    static constexpr int CTRL_BYTES = 1024;
+    static constexpr int SMEM_BYTES = 1024 + OFF_CTRL + CTRL_BYTES;  // + 1024-byte alignment slack
+    static constexpr int S_COL = 0;                // S buffer b at S_COL + 128 b
+    static constexpr int O_COL = 256;              // O buffer b at O_COL + 128 b
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int WARP_TMA = 0, WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
+    static constexpr int THREADS = 32 * 7;
+    static constexpr int T_LAZY = 8;               // reference slack, base 2
+};
+
+struct __align__(16) PfControl {
+    uint64_t full[PfCfg::NS], empty[PfCfg::NS];  // K/V ring
+    uint64_t qfull, qempty;                      // query tile
+    uint64_t sfull[2], sfree[2];                 // S buffer written / read by the softmax warps
+    uint64_t pfull, pvdone;                      // P written / value product of the last step done
+    uint64_t ofull[2], ofree[2];                 // O buffer of a unit complete / read by the epilogue
+    uint64_t drain[2];                           // last products of each issuing warp complete
+    uint32_t tmem_base;
+    int abort;
+};
+
+// One work unit as every warp role derives it from the unit index.
+struct PfUnit {
+    int b, kv, qt;
+    int n_tok;   // query tokens in the tile (rows n_tok * R .. 127 are idle)
+    int q_row0;  // row of q / out of the tile's first token
+    int pos0;    // cache position of the tile's first token
+    int L;       // clamped cache length
+    int steps;   // 128-key steps: keys [0, pos0 + n_tok) are visible to some row
+};
+
+// Unit u: query tile qt = QT - 1 - u / (B H_KV) (heaviest first), then
+// sequence b, then KV head.  Returns false for a unit with no rows; *flags
+// gets the status bits the sequence's bounds raise (a clamped length, an
+// inconsistent query span -- such a sequence is skipped).
+__device__ __forceinline__ bool pf_unit(const PrefillArgs& a, int u, PfUnit& x, uint32_t* flags) {
+    const int per = a.B * a.H_KV;
+    const int t = u / per;
+    const int rem = u - t * per;
+    x.qt = a.QT - 1 - t;
+    x.b = rem / a.H_KV;
+    x.kv = rem - x.b * a.H_KV;
+    const int c0 = __ldg(a.cu_q + x.b), c1 = __ldg(a.cu_q + x.b + 1);
+    const int raw = __ldg(a.seq_lens + x.b);
+    x.L = clamp_len(raw, a.max_len);
+    uint32_t f = (raw < 0 || raw > a.max_len) ? kFlagClamped : 0u;
+    const int n = c1 - c0;
+    const bool span_ok = c0 >= 0 && c1 <= a.total_q && n >= 0 && n <= x.L && n <= a.max_q;
+    if (!span_ok) f |= kFlagBadSpan;
+    *flags = f;
+    if (!span_ok) return false;
+    const int tok0 = x.qt * a.TQ;
+    if (tok0 >= n) return false;
+    x.n_tok = min(a.TQ, n - tok0);
+    x.q_row0 = c0 + tok0;
+    x.pos0 = x.L - n + tok0;
+    x.steps = (x.pos0 + x.n_tok + PfCfg::BN - 1) / PfCfg::BN;
+    return true;
+}
+
+__device__ __forceinline__ void pf_fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+template <bool PAGED, bool OUT_BF16>
+__global__ void __launch_bounds__(PfCfg::THREADS, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
+    using C = PfCfg;
+    static_assert(sizeof(PfControl) <= C::CTRL_BYTES, "control block overflows its slot");
+    constexpr uint32_t IDESC_QK = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 128, C::BN);
+    constexpr uint32_t IDESC_PV = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 1, 128, C::D);
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_addr(smem_raw);
+    const uint32_t base = (raw + 1023u) & ~1023u;
+    uint8_t* base_ptr = smem_raw + (base - raw);
+    const uint32_t q_smem = base + C::OFF_Q;
+    const uint32_t p_smem = base + C::OFF_P;
+    const uint32_t ring = base + C::OFF_RING;
+    PfControl* ctrl = reinterpret_cast<PfControl*>(base_ptr + C::OFF_CTRL);
+    volatile int* abort_flag = &ctrl->abort;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_units = a.B * a.H_KV * a.QT;
+
+    if (warp == 0 && lane == 0) {
+        prefetch_tensormap(&tmQ);
+        prefetch_tensormap(&tmK);
+        prefetch_tensormap(&tmV);
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(smem_addr(&ctrl->full[s]), 1);
+            mbar_init(smem_addr(&ctrl->empty[s]), 1);
+        }
+        mbar_init(smem_addr(&ctrl->qfull), 1);
+        mbar_init(smem_addr(&ctrl->qempty), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_addr(&ctrl->sfull[s]), 1);
+            mbar_init(smem_addr(&ctrl->sfree[s]), 4);
+            mbar_init(smem_addr(&ctrl->ofull[s]), 1);
+            mbar_init(smem_addr(&ctrl->ofree[s]), 4);
+            mbar_init(smem_addr(&ctrl->drain[s]), 1);
+        }
+        mbar_init(smem_addr(&ctrl->pfull), 4);
+        mbar_init(smem_addr(&ctrl->pvdone), 1);
+        ctrl->abort = 0;
+    }
+    // Query rows the TMA box leaves out (R * TQ < 128) stay zero.
+    for (int i = threadIdx.x; i < C::TILE / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(base_ptr + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
+    if (warp == C::WARP_QK) {
+        tc::tmem_alloc(smem_addr(&ctrl->tmem_base), C::TMEM_COLS);
+        tc::tmem_relinquish();
+    }
+    fence_barrier_init();
+    fence_proxy_async_smem();
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = ctrl->tmem_base;
+
+    auto fail = [&]() {
+        *abort_flag = 1;
+        if (lane == 0) atomicOr(a.status, kFlagTimeout);
+    };
+
+    if (warp == C::WARP_TMA) {
+        // ------------------------------------------------------------ producer
+        // K/V rows are read again by the sequence's other query tiles: keep them in L2.
+        const uint64_t pol_kv = policy_evict_last();
+        const uint64_t pol_q = policy_evict_first();
+        int64_t ld = 0;  // K/V loads issued: K of step g is load 2g, V is 2g + 1
+        int uc = 0;      // units issued
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            PfUnit x;
+            uint32_t fl;
+            const bool has = pf_unit(a, u, x, &fl);
+            if (fl != 0u && lane == 0 && x.kv == 0 && x.qt == a.QT - 1) atomicOr(a.status, fl);
+            if (!has) continue;
+            if (!mbar_wait_warp(smem_addr(&ctrl->qempty), (static_cast<uint32_t>(uc) & 1u) ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            if (lane == 0) {
+                const uint32_t bar = smem_addr(&ctrl->qfull);
+                mbar_arrive_expect_tx(bar, 2u * 128u * static_cast<uint32_t>(a.R * a.TQ));
+                for (int p = 0; p < 2; ++p)
+                    tma_load_3d(q_smem + p * C::PANEL, &tmQ, bar, 64 * p, x.kv * a.R, x.q_row0, pol_q);
+            }
+            ++uc;
+            const int kv_end = x.pos0 + x.n_tok;
+            for (int j = 0; j < x.steps && ok; ++j) {
+                // Coordinates of the step's two 64-key tiles; a tile past the visible
+                // keys is read from outside the tensor, which fills it with zeros.
+                int c2[2], c3[2];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int t = 2 * j + h;
+                    const bool need = t * kTile < kv_end;
+                    if constexpr (PAGED) {
+                        int page = a.num_blocks;
+                        if (need) {
+                            page = __ldg(a.block_table + static_cast<int64_t>(x.b) * a.max_blocks + t);
+                            if (page < 0 || page >= a.num_blocks) {
+                                if (lane == 0) atomicOr(a.status, kFlagBadBlock);
+                                page = a.num_blocks;
+                            }
+                        }
+                        c2[h] = 0;
+                        c3[h] = page;
+                    } else {
+                        c2[h] = need ? t * kTile : a.S_max;
+                        c3[h] = x.b;
+                    }
+                }
+#pragma unroll
+                for (int which = 0; which < 2; ++which) {  // K, then V
+                    const int e = static_cast<int>(ld % C::NS);
+                    const uint32_t ph = static_cast<uint32_t>(ld / C::NS) & 1u;
+                    if (!mbar_wait_warp(smem_addr(&ctrl->empty[e]), ph ^ 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (lane == 0) {
+                        const uint32_t bar = smem_addr(&ctrl->full[e]);
+                        const uint32_t dst = ring + e * C::TILE;
+                        const CUtensorMap* map = which == 0 ? &tmK : &tmV;
+                        mbar_arrive_expect_tx(bar, C::TILE);
+#pragma unroll
+                        for (int p = 0; p < 2; ++p)
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+                                tma_load_4d(dst + p * C::PANEL + h * C::BOX, map, bar, 64 * p, x.kv, c2[h], c3[h],
+                                            pol_kv);
+                    }
+                    ++ld;
+                }
+            }
+        }
+        if (!ok) {
+            fail();
+            // Let copies already in flight land before the CTA's shared memory goes away.
+            const int64_t first = ld > C::NS ? ld - C::NS : 0;
+            for (int64_t i = first; i < ld; ++i)
+                mbar_wait(smem_addr(&ctrl->full[i % C::NS]), static_cast<uint32_t>((i / C::NS) & 1), nullptr);
+            if (uc > 0) mbar_wait(smem_addr(&ctrl->qfull), static_cast<uint32_t>(uc - 1) & 1u, nullptr);
+        }
+    }
+
+    if (warp == C::WARP_QK) {
+        // ------------------------------------------------------------ score products
+        // Global step g: S(g) = Q K(g)^T into buffer g & 1 once the softmax warps
+        // have read that buffer's previous contents (step g - 2).
+        int64_t g = 0;
+        int uc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            PfUnit x;
+            uint32_t fl;
+            if (!pf_unit(a, u, x, &fl)) continue;
+            if (!mbar_wait_warp(smem_addr(&ctrl->qfull), static_cast<uint32_t>(uc) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            for (int j = 0; j < x.steps; ++j, ++g) {
+                const int sb = static_cast<int>(g & 1);
+                const uint32_t spar = static_cast<uint32_t>(g >> 1) & 1u;
+                const int64_t ki = 2 * g;
+                const int e = static_cast<int>(ki % C::NS);
+                if (!mbar_wait_warp(smem_addr(&ctrl->sfree[sb]), spar ^ 1u, abort_flag) ||
+                    !mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(ki / C::NS) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    const uint32_t kt = ring + e * C::TILE;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const uint32_t off = (k >> 2) * C::PANEL + 32 * (k & 3);
+                        const uint64_t da = tc::smem_desc(q_smem + off, 16, 1024, tc::kLayoutSw128);
+                        const uint64_t db = tc::smem_desc(kt + off, 16, 1024, tc::kLayoutSw128);
+                        tc::mma_f16(tmem + C::S_COL + sb * C::BN, da, db, IDESC_QK, k > 0);
+                    }
+                    tc::commit(smem_addr(&ctrl->sfull[sb]));
+                    tc::commit(smem_addr(&ctrl->empty[e]));
+                    if (j == x.steps - 1) tc::commit(smem_addr(&ctrl->qempty));
+                }
+                __syncwarp();
+            }
+            ++uc;
+        }
+        if (!ok) fail();
+        // Every product this warp issued has completed before tensor memory is freed.
+        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain[0]));
+        __syncwarp();
+        mbar_wait_warp(smem_addr(&ctrl->drain[0]), 0u, nullptr);
+    }
+
+    if (warp == C::WARP_PV) {
+        // ------------------------------------------------------------ value products
+        // Global step g: O += P_hi V(g) + P_lo V(g) once the softmax warps have
+        // written P(g); a unit's first step overwrites its O buffer after the
+        // epilogue has read that buffer's previous unit.
+        int64_t g = 0;
+        int uc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            PfUnit x;
+            uint32_t fl;
+            if (!pf_unit(a, u, x, &fl)) continue;
+            const int ob = uc & 1;
+            for (int j = 0; j < x.steps; ++j, ++g) {
+                const int64_t vi = 2 * g + 1;
+                const int e = static_cast<int>(vi % C::NS);
+                if (!mbar_wait_warp(smem_addr(&ctrl->pfull), static_cast<uint32_t>(g) & 1u, abort_flag) ||
+                    (j == 0 && !mbar_wait_warp(smem_addr(&ctrl->ofree[ob]),
+                                               (static_cast<uint32_t>(uc >> 1) & 1u) ^ 1u, abort_flag)) ||
+                    !mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(vi / C::NS) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    const uint32_t vt = ring + e * C::TILE;
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            const uint64_t da = tc::smem_desc(p_smem + part * C::TILE + (k >> 2) * C::PANEL + 32 * (k & 3),
+                                                              16, 1024, tc::kLayoutSw128);
+                            const uint64_t db = tc::smem_desc(vt + k * 2048, C::PANEL, 1024, tc::kLayoutSw128);
+                            tc::mma_f16(tmem + C::O_COL + ob * C::D, da, db, IDESC_PV,
+                                        !(j == 0 && part == 0 && k == 0));
+                        }
+                    tc::commit(smem_addr(&ctrl->empty[e]));
+                    tc::commit(smem_addr(&ctrl->pvdone));
+                    if (j == x.steps - 1) tc::commit(smem_addr(&ctrl->ofull[ob]));
+                }
+                __syncwarp();
+            }
+            ++uc;
+        }
+        if (!ok) fail();
+        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain[1]));
+        __syncwarp();
+        mbar_wait_warp(smem_addr(&ctrl->drain[1]), 0u, nullptr);
+    }
+
+    if (warp >= C::WARP_SM0) {
+        // ------------------------------------------------------------ softmax + epilogue
+        const int sp = warp & 3;       // tensor-memory sub-partition of this warp
+        const int r = 32 * sp + lane;  // tile row held by this thread (= TMEM lane)
+        const float NEG_INF = -__int_as_float(0x7f800000);
+        int64_t g = 0;
+        int uc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            PfUnit x;
+            uint32_t fl;
+            if (!pf_unit(a, u, x, &fl)) continue;
+            const int ob = uc & 1;
+            const int tq = r / a.R;        // token of the row within the tile
+            const int hq = r - tq * a.R;   // query head of the row within the group
+            const bool row_ok = tq < x.n_tok;
+            const int pos = x.pos0 + tq;   // cache position of the row's token
+            float ref = NEG_INF, l = 0.f;
+            for (int j = 0; j < x.steps; ++j, ++g) {
+                const int sb = static_cast<int>(g & 1);
+                if (!mbar_wait_warp(smem_addr(&ctrl->sfull[sb]), static_cast<uint32_t>(g >> 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                uint32_t sv[C::BN];  // the row's scores, then its weights (fp32 bits)
+#pragma unroll
+                for (int c = 0; c < C::BN / 32; ++c)
+                    tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::BN + 32 * c), sv + 32 * c);
+                tc::tmem_wait_ld();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
+
+                // Base-2 scores; key 128 j + c is visible iff it is <= pos.
+                const int lim = row_ok ? pos - C::BN * j : -1;
+                float mx8[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx8[i] = NEG_INF;
+                if (lim >= C::BN - 1) {
+#pragma unroll
+                    for (int c = 0; c < C::BN; ++c) {
+                        const float v = __uint_as_float(sv[c]) * a.sl2;
+                        sv[c] = __float_as_uint(v);
+                        mx8[c & 7] = fmaxf(mx8[c & 7], v);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < C::BN; ++c) {
+                        const float v = c <= lim ? __uint_as_float(sv[c]) * a.sl2 : NEG_INF;
+                        sv[c] = __float_as_uint(v);
+                        mx8[c & 7] = fmaxf(mx8[c & 7], v);
+                    }
+                }
+                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+                // Lazy reference: weights stay <= 2^8 against it.
+                float alpha = 1.f;
+                const bool move = mx > ref + static_cast<float>(C::T_LAZY);
+                if (move) {
+                    alpha = ref == NEG_INF ? 0.f : fast_exp2(ref - mx);
+                    ref = mx;
+                    l *= alpha;
+                }
+                const float rb = ref == NEG_INF ? 0.f : ref;
+                float part[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) part[i] = 0.f;
+#pragma unroll
+                for (int c = 0; c < C::BN; ++c) {
+                    const float pc = fast_exp2(__uint_as_float(sv[c]) - rb);
+                    sv[c] = __float_as_uint(pc);
+                    part[c & 7] += pc;
+                }
+                l += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+
+                // The P buffer and O are free once the previous step's value product is done.
+                if (g > 0 &&
+                    !mbar_wait_warp(smem_addr(&ctrl->pvdone), static_cast<uint32_t>(g - 1) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                if (j > 0 && __any_sync(0xffffffffu, move)) {
+                    // O holds this unit's earlier steps: rescale the moved rows in place.
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < C::D / 32; ++c) {
+                        uint32_t o[32];
+                        const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 32 * c);
+                        tc::tmem_ld32(oa, o);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                        tc::tmem_st32(oa, o);
+                    }
+                    tc::tmem_wait_st();
+                }
+                // Value rows at or past L_b may hold anything, and 0 * NaN would poison O.
+                if (C::BN * (j + 1) > x.L) {
+                    const int64_t vi = 2 * g + 1;
+                    const int e = static_cast<int>(vi % C::NS);
+                    if (!mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(vi / C::NS) & 1u,
+                                        abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    if (C::BN * j + r >= x.L) {
+                        const uint32_t vrow = ring + e * C::TILE + r * 128;
+#pragma unroll
+                        for (int p = 0; p < 2; ++p)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c)
+                                st_shared_v4(vrow + p * C::PANEL + ((c ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                    }
+                }
+                // P = hi + lo (bf16 each), row r: keys 0..63 in the first panel, 64..127
+                // in the second, 16-byte chunks swizzled by the row's low three bits.
+#pragma unroll
+                for (int c = 0; c < C::BN / 8; ++c) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int w = 0; w < 4; ++w)
+                        split_bf16x2(__uint_as_float(sv[8 * c + 2 * w]), __uint_as_float(sv[8 * c + 2 * w + 1]), hi[w],
+                                     lo[w]);
+                    const uint32_t off = (c >> 3) * C::PANEL + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                    st_shared_v4(p_smem + off, hi[0], hi[1], hi[2], hi[3]);
+                    st_shared_v4(p_smem + C::TILE + off, lo[0], lo[1], lo[2], lo[3]);
+                }
+                pf_fence_async_smem();
+                tc::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull));
+            }
+            if (!ok) break;
+
+            // ---------------------------------------------------- unit end: O / l -> out
+            if (!mbar_wait_warp(smem_addr(&ctrl->ofull[ob]), static_cast<uint32_t>(uc >> 1) & 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const int64_t orow =
+                row_ok ? (static_cast<int64_t>(x.q_row0 + tq) * a.H_Q + x.kv * a.R + hq) * C::D : 0;
+#pragma unroll
+            for (int c = 0; c < C::D / 32; ++c) {
+                uint32_t o[32];
+                tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 32 * c), o);
+                tc::tmem_wait_ld();
+                if (row_ok) {
+                    if constexpr (OUT_BF16) {
+                        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + orow + 32 * c);
+#pragma unroll
+                        for (int q4 = 0; q4 < 4; ++q4) {
+                            uint32_t wv[4];
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const __nv_bfloat162 h2 = __floats2bfloat162_rn(__uint_as_float(o[8 * q4 + 2 * e]) * inv,
+                                                                                __uint_as_float(o[8 * q4 + 2 * e + 1]) * inv);
+                                wv[e] = *reinterpret_cast<const uint32_t*>(&h2);
+                            }
+                            dst[q4] = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+                        }
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(a.out) + orow + 32 * c);
+#pragma unroll
+                        for (int q4 = 0; q4 < 8; ++q4)
+                            dst[q4] = make_float4(__uint_as_float(o[4 * q4]) * inv, __uint_as_float(o[4 * q4 + 1]) * inv,
+                                                  __uint_as_float(o[4 * q4 + 2]) * inv,
+                                                  __uint_as_float(o[4 * q4 + 3]) * inv);
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree[ob]));
+            ++uc;
+        }
+        if (!ok) fail();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == C::WARP_QK) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
+
+}  // namespace gqa

@@ -27,6 +27,7 @@ constexpr uint32_t kFlagClamped = 1u;  // GQA_FLAG_SEQ_LEN_CLAMPED
 constexpr uint32_t kFlagBadBlock = 2u; // GQA_FLAG_BAD_BLOCK
 constexpr uint32_t kFlagTimeout = 4u;  // GQA_FLAG_TIMEOUT
 constexpr uint32_t kFlagBadPosition = 8u;  // GQA_FLAG_BAD_POSITION
+constexpr uint32_t kFlagBadSpan = 16u;     // GQA_FLAG_BAD_QUERY_SPAN
 
 struct KernelArgs {
     const int32_t* seq_lens;     // [B]

@@ -220,3 +220,123 @@ def algorithmic_bytes(w: Workload, seq_lens: torch.Tensor, out_bytes: int = 4) -
     e_kv = 1 if w.kv8 else e
     kv = int(seq_lens.to(torch.int64).sum()) * w.H_KV * w.D * e_kv * 2
     return kv + w.B * w.H_Q * w.D * e + w.B * w.H_Q * w.D * out_bytes
+
+
+# ---------------------------------------------------------------- multi-token (prefill) steps
+
+_S_QLEN, _S_PREFIX = 5, 6
+
+
+@dataclasses.dataclass(frozen=True)
+class PrefillWorkload:
+    """One multi-token step of one attention layer.
+
+    Every sequence brings ``q_len`` new query tokens (U[1, q_len] when
+    ``ragged``) after a cached prefix of ``prefix`` tokens (U[0, prefix] when
+    ragged); the new tokens' keys and values are already the last n_b of its
+    L_b = prefix_b + n_b cached tokens.  prefix 0 is a fresh prompt.
+    """
+
+    name: str
+    B: int
+    H_Q: int
+    H_KV: int
+    D: int
+    q_len: int
+    prefix: int
+    seed: int
+    ragged: bool = False
+    page_size: int = 0
+
+    @property
+    def R(self) -> int:
+        return self.H_Q // self.H_KV
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / math.sqrt(self.D)
+
+    @property
+    def capacity(self) -> int:
+        """Cache positions per sequence (a whole number of pages when paged)."""
+        n = self.prefix + self.q_len
+        return -(-n // self.page_size) * self.page_size if self.page_size else n
+
+
+PREFILL_WORKLOADS: dict[str, PrefillWorkload] = {
+    w.name: w
+    for w in [
+        # Llama 3 8B heads (32 / 8): four fresh 4096-token prompts.
+        PrefillWorkload("prefill_llama3_8b", 4, 32, 8, 128, 4096, 0, seed=11),
+        # Llama 2 70B heads (64 / 8): the last 2048-token chunk of 32K-token prompts.
+        PrefillWorkload("prefill_llama2_70b_chunk", 4, 64, 8, 128, 2048, 30720, seed=12),
+        # Mixed chunk lengths and prefixes over a paged cache.
+        PrefillWorkload("prefill_ragged_paged", 8, 64, 8, 128, 1024, 8192, seed=13, ragged=True,
+                        page_size=PAGE_SIZE),
+    ]
+}
+
+
+def prefill_lengths(w: PrefillWorkload) -> tuple[np.ndarray, np.ndarray]:
+    """(n_b, L_b) as int32 arrays [B]."""
+    if not w.ragged:
+        n = np.full(w.B, w.q_len, dtype=np.int32)
+        pre = np.full(w.B, w.prefix, dtype=np.int32)
+    else:
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence((w.seed, _S_QLEN))))
+        n = rng.integers(1, w.q_len + 1, size=w.B).astype(np.int32)
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence((w.seed, _S_PREFIX))))
+        pre = rng.integers(0, w.prefix + 1, size=w.B).astype(np.int32)
+    return n, (n + pre).astype(np.int32)
+
+
+def make_prefill_inputs(w: PrefillWorkload, pad_value: float = 0.0, lengths=None):
+    """Generate one multi-token step's inputs on the host.
+
+    ``lengths`` = (n_b, L_b) overrides the workload's length draw.
+
+    Returns a dict with
+      q          [total_q, H_Q, D] bf16, sequence b's rows at cu_q[b] .. cu_q[b+1]-1
+      k, v       [B, capacity, H_KV, D] bf16 logical contiguous cache; rows
+                 t >= L_b hold ``pad_value``
+      seq_lens   int32 [B];  cu_q  int32 [B + 1];  max_q  int
+      block_table, k_paged, v_paged   (paged workloads only), as make_inputs
+    """
+    if lengths is None:
+        n, lens = prefill_lengths(w)
+    else:
+        n, lens = (np.asarray(x, dtype=np.int32) for x in lengths)
+        assert n.shape == lens.shape == (w.B,) and (n <= lens).all()
+    cu = np.concatenate([[0], np.cumsum(n)]).astype(np.int32)
+    q = torch.empty(int(cu[-1]), w.H_Q, w.D, dtype=torch.bfloat16)
+    _fill_normal(q, (w.seed, _S_Q))
+    S = max(w.capacity, int(lens.max()) if w.B else 0)
+    if w.page_size:
+        S = -(-S // w.page_size) * w.page_size
+    k = torch.full((w.B, S, w.H_KV, w.D), pad_value, dtype=torch.bfloat16)
+    v = torch.full((w.B, S, w.H_KV, w.D), pad_value, dtype=torch.bfloat16)
+    for b in range(w.B):
+        L = int(lens[b])
+        _fill_normal(k[b, :L], (w.seed, _S_K, b))
+        _fill_normal(v[b, :L], (w.seed, _S_V, b))
+    out = {"q": q, "k": k, "v": v, "seq_lens": torch.from_numpy(lens), "cu_q": torch.from_numpy(cu),
+           "max_q": int(n.max()) if w.B else 0}
+    if w.page_size:
+        nb = S // w.page_size
+        rng = np.random.Generator(np.random.PCG64(np.random.SeedSequence((w.seed, _S_TABLE))))
+        table = torch.from_numpy(rng.permutation(w.B * nb).astype(np.int32)).view(w.B, nb)
+        out["block_table"] = table
+        out["k_paged"] = to_pages(k, table, w.page_size)
+        out["v_paged"] = to_pages(v, table, w.page_size)
+    return out
+
+
+def prefill_flops(w: PrefillWorkload, n: np.ndarray, lens: np.ndarray) -> int:
+    """Algorithmic FLOPs: 4 D per (query head, visible key) pair -- 2 D for the
+    score, 2 D for the weighted value -- where query token j of sequence b sees
+    L_b - n_b + j + 1 keys."""
+    pairs = 0
+    for n_b, L in zip(n.tolist(), lens.tolist()):
+        first = L - n_b + 1  # keys seen by the first new token
+        pairs += n_b * first + n_b * (n_b - 1) // 2
+    return 4 * w.D * w.H_Q * pairs

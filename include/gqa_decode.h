@@ -85,6 +85,8 @@ typedef enum gqa_kernel {
 #define GQA_FLAG_BAD_BLOCK 2u         /* a live block_table entry was outside [0, num_blocks) */
 #define GQA_FLAG_TIMEOUT 4u           /* an internal pipeline wait gave up; outputs invalid */
 #define GQA_FLAG_BAD_POSITION 8u      /* a rope/append position was outside [0, max_seq_len) */
+#define GQA_FLAG_BAD_QUERY_SPAN 16u   /* gqa_prefill: a cu_q_lens span was out of order, outside
+                                         [0, total_q], longer than max_q_len or than L_b */
 
 /*
  * Problem description.  All counts are element counts.
@@ -254,6 +256,51 @@ gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const
                            const void* v_new, const int32_t* positions, const int32_t* block_table,
                            double rope_base, int pairing, void* q_out, void* k_cache, void* v_cache,
                            int32_t* seq_lens_out, void* workspace, void* stream);
+
+/*
+ * Multi-token step: prefill of new prompts, or a chunk of a prompt after a
+ * cached prefix, for every sequence of the batch at once.  [LLMS] opening
+ * section: prompt processing (prefill) is the compute-bound phase; section 2:
+ * Head_i = softmax(Q_i K_{g(i)}^T / sqrt(d_k) + M) V_{g(i)} with M the causal
+ * mask.  Sequence b brings n_b = cu_q_lens[b+1] - cu_q_lens[b] new query
+ * tokens, rows cu_q_lens[b] .. cu_q_lens[b+1]-1 of q, whose keys and values
+ * are already the last n_b of its L_b = seq_lens[b] cached tokens (appended
+ * beforehand, e.g. by the caller's projection).  Its query token j sits at
+ * position p = L_b - n_b + j and attends to cache positions t <= p -- the
+ * whole cached prefix and the new tokens up to itself.  With no prefix
+ * (L_b = n_b) M is the s x s causal mask as written; n_b = 1 is gqa_decode's
+ * step.  For every row i of sequence b, query head h, g = h / R:
+ *     s_t = scale * <q[i,h,:], K_b[t,g,:]>,   t <= p
+ *     out[i,h,:] = sum_t softmax(s)_t * V_b[t,g,:]
+ *
+ *   params      as for gqa_decode; head_dim 128, qkv_dtype GQA_BF16 and
+ *               R = H_Q / H_KV <= 128 (else GQA_ERR_UNSUPPORTED); kernel AUTO
+ *               or TCGEN05 (the only implementation: tcgen05 tensor cores).
+ *   q           [total_q, H_Q, 128] bf16, 16-byte aligned, sequences' rows
+ *               back to back in the order of cu_q_lens.
+ *   cu_q_lens   int32 [B + 1] device, cu_q_lens[0] = 0, non-decreasing,
+ *               cu_q_lens[B] = total_q; 0 <= n_b <= min(L_b, max_q_len).
+ *   total_q     rows of q and out (host value).
+ *   max_q_len   host upper bound on every n_b; sizes the launch.
+ *   k_cache, v_cache, seq_lens, block_table, scale   as for gqa_decode.
+ *   out         [total_q, H_Q, 128] out_dtype, 16-byte aligned.  Rows of a
+ *               sequence whose span is invalid are left untouched.
+ *   workspace   >= gqa_prefill_workspace_size bytes (any gqa_decode
+ *               workspace will do), 256-byte aligned, zero-filled once: it
+ *               holds the status word.
+ * cu_q_lens, seq_lens and block_table are device data and are not read on the
+ * host: an invalid span skips that sequence and raises GQA_FLAG_BAD_QUERY_SPAN;
+ * lengths and pages are handled as in gqa_decode.  Argument errors return
+ * before anything is enqueued; the call allocates nothing and does not
+ * synchronise.  Weights enter the value product as bf16 hi + lo parts (about
+ * 16 significant bits), accumulation is fp32.
+ */
+gqa_status gqa_prefill_workspace_size(const gqa_decode_params* params, size_t* bytes);
+
+gqa_status gqa_prefill(const gqa_decode_params* params, const void* q, const int32_t* cu_q_lens,
+                       int32_t total_q, int32_t max_q_len, const void* k_cache, const void* v_cache,
+                       const int32_t* seq_lens, const int32_t* block_table, float scale, void* out,
+                       void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * Reads the workspace status word (GQA_FLAG_* bits) into *flags after

@@ -226,3 +226,52 @@ def test_wait_selftest_rejects_bad_arguments_on_host(lib):
     assert lib.gqa_wait_selftest(ctypes.c_uint64(10**11), 0, vp(16), vp(16), vp(None)) == GQA_ERR_INVALID
     assert lib.gqa_wait_selftest(ctypes.c_uint64(10**6), 0, vp(None), vp(16), vp(None)) == GQA_ERR_INVALID
     assert lib.gqa_wait_selftest(ctypes.c_uint64(10**6), 0, vp(16), vp(12), vp(None)) == GQA_ERR_INVALID
+
+
+def call_prefill(lib, p, q=16, cu=16, total_q=10, max_q=10, k=16, v=16, lens=16, table=None, scale=0.1,
+                 out=16, ws=256, ws_bytes=256):
+    vp = ctypes.c_void_p
+    return lib.gqa_prefill(ctypes.byref(p), vp(q), vp(cu), total_q, max_q, vp(k), vp(v), vp(lens), vp(table),
+                           ctypes.c_float(scale), vp(out), vp(ws), ctypes.c_size_t(ws_bytes), vp(None))
+
+
+def test_prefill_refuses_unsupported_problems_on_host(lib):
+    assert call_prefill(lib, params(head_dim=64)) == GQA_ERR_UNSUPPORTED
+    assert call_prefill(lib, params(qkv_dtype=1)) == GQA_ERR_UNSUPPORTED      # bf16 only
+    assert call_prefill(lib, params(kernel=1)) == GQA_ERR_UNSUPPORTED         # tcgen05 only
+    assert call_prefill(lib, params(H_Q=256, H_KV=1)) == GQA_ERR_UNSUPPORTED  # R > 128
+    assert call_prefill(lib, params(H_Q=6, H_KV=4)) == GQA_ERR_INVALID
+
+
+def test_prefill_rejects_bad_arguments_on_host(lib):
+    p = params()
+    assert call_prefill(lib, p, total_q=-1) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, max_q=-1) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, q=None) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, cu=None) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, lens=None) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, out=None) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, q=24) == GQA_ERR_INVALID           # TMA needs 16-byte alignment
+    assert call_prefill(lib, p, out=8) == GQA_ERR_INVALID          # 16-byte vector stores
+    assert call_prefill(lib, p, cu=18) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, table=16) == GQA_ERR_INVALID       # table given for a contiguous cache
+    pp = params(page_size=64, max_blocks_per_seq=4, num_blocks=8)
+    assert call_prefill(lib, pp, table=None) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, scale=float("nan")) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, ws=None) == GQA_ERR_WORKSPACE
+    assert call_prefill(lib, p, ws=128) == GQA_ERR_WORKSPACE       # not 256-byte aligned
+    assert call_prefill(lib, p, ws_bytes=64) == GQA_ERR_WORKSPACE   # no room for the status word
+
+
+def test_prefill_with_nothing_to_do_is_a_no_op(lib):
+    none = dict(q=None, cu=None, k=None, v=None, lens=None, out=None, ws=None)
+    assert call_prefill(lib, params(B=0), **none) == GQA_OK
+    assert call_prefill(lib, params(), total_q=0, **none) == GQA_OK
+    assert call_prefill(lib, params(), max_q=0, **none) == GQA_OK
+
+
+def test_prefill_workspace_size(lib):
+    n = ctypes.c_size_t(0)
+    assert lib.gqa_prefill_workspace_size(ctypes.byref(params()), ctypes.byref(n)) == GQA_OK
+    assert n.value == 256
+    assert lib.gqa_prefill_workspace_size(ctypes.byref(params(H_Q=6, H_KV=4)), ctypes.byref(n)) == GQA_ERR_INVALID
