@@ -681,7 +681,7 @@ gqa_status gqa_prefill(const gqa_decode_params* params, const void* q, const int
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
         !aligned(cu_q_lens, 4) || !aligned(seq_lens, 4) || (block_table && !aligned(block_table, 4)))
         return GQA_ERR_INVALID;
-    if (!(scale == scale)) return GQA_ERR_INVALID;
+    if (!(scale > 0.f) || !std::isfinite(scale)) return GQA_ERR_INVALID;  // a positive scale keeps the score order
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < kHeaderBytes) return GQA_ERR_WORKSPACE;
 
     const int TQ = 128 / R;

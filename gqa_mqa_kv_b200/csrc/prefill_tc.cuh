@@ -18,11 +18,14 @@
 //                   128-byte swizzle as TMA stages them; S lands in tensor
 //                   memory (two buffers: the next step's product overlaps
 //                   this step's softmax).
-//   softmax         four warps, thread = row = TMEM lane, the row's 128
-//                   scores in registers: base-2 online softmax against a
-//                   per-row reference that moves only when a score exceeds
-//                   it by more than 8 (O is rescaled in tensor memory then).
-//                   P goes to shared memory as bf16 hi and lo parts, so the
+//   softmax         eight warps, two per tensor-memory sub-partition:
+//                   thread = row = TMEM lane, each warp of a pair taking 64
+//                   of the step's keys in registers.  Base-2 online softmax
+//                   against a per-row reference that moves only when a score
+//                   exceeds it by more than 8 (O is rescaled in tensor memory
+//                   then); the pair agrees on the reference through a
+//                   shared-memory exchange of partial maxima each step.  P
+//                   goes to shared memory as bf16 hi and lo parts, so the
 //                   product keeps ~16 bits of every weight, in the same
 //                   K-major swizzled layout TMA would produce.
 //   O += P V        tcgen05.mma, M = 128, N = d = 128, K = 128 keys, once on
@@ -32,8 +35,9 @@
 //
 // Persistent CTAs (one per SM) walk the units in a fixed interleaved order,
 // heaviest query tiles first.  Warp roles: 0 TMA producer, 1 score products
-// (+ tensor-memory allocation), 2 value products, 3..6 softmax and epilogue
-// (sub-partitions 3, 0, 1, 2).  Every wait is bounded (kWaitTimeoutNs); on a
+// (+ tensor-memory allocation), 2 value products, 3..10 softmax and epilogue
+// (warp w on sub-partition w % 4, keys 64 ((w - 3) / 4) ..).  Every wait is
+// bounded (kWaitTimeoutNs); on a
 // timeout the CTA raises GQA_FLAG_TIMEOUT, lets its copies and products
 // drain, frees its tensor memory and returns.
 #pragma once
@@ -74,13 +78,14 @@ struct PfCfg {
     static constexpr int OFF_P = OFF_Q + TILE;     // P hi, then P lo
     static constexpr int OFF_RING = OFF_P + 2 * TILE;
     static constexpr int OFF_CTRL = OFF_RING + NS * TILE;
-    static constexpr int CTRL_BYTES = 1024;
+    static constexpr int CTRL_BYTES = 2048;
     static constexpr int SMEM_BYTES = 1024 + OFF_CTRL + CTRL_BYTES;  // + 1024-byte alignment slack
     static constexpr int S_COL = 0;                // S buffer b at S_COL + 128 b
     static constexpr int O_COL = 256;              // O buffer b at O_COL + 128 b
     static constexpr int TMEM_COLS = 512;
     static constexpr int WARP_TMA = 0, WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
-    static constexpr int THREADS = 32 * 7;
+    static constexpr int NSM = 8;                  // softmax warps: two per sub-partition, 64 keys each
+    static constexpr int THREADS = 32 * (3 + NSM);
     static constexpr int T_LAZY = 8;               // reference slack, base 2
 };
 
@@ -91,8 +96,10 @@ struct __align__(16) PfControl {
     uint64_t pfull, pvdone;                      // P written / value product of the last step done
     uint64_t ofull[2], ofree[2];                 // O buffer of a unit complete / read by the epilogue
     uint64_t drain[2];                           // last products of each issuing warp complete
+    uint64_t xfull[4], xfree[4];                 // per sub-partition: both halves wrote / read xval
     uint32_t tmem_base;
     int abort;
+    float xval[2][128];                          // per key half, per row: a partial row max or row sum
 };
 
 // One work unit as every warp role derives it from the unit index.
@@ -138,6 +145,50 @@ __device__ __forceinline__ void pf_fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// Packed fp32 pairs (sm_100 f32x2 arithmetic: one instruction for two lanes of work).
+__device__ __forceinline__ uint64_t pf_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+__device__ __forceinline__ float2 pf_unpack(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+
+__device__ __forceinline__ uint64_t pf_fma2(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
+__device__ __forceinline__ uint64_t pf_add2(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+__device__ __forceinline__ float pf_max3(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// p0, p1 -> bf16 hi parts (truncated: the top 16 bits of each fp32) and bf16
+// lo parts (round to nearest of the exact remainder); hi + lo is within
+// 2^-15 of each weight.  p0 lands in the low half of each packed word.
+__device__ __forceinline__ void pf_split(float p0, float p1, uint64_t neg1, uint32_t& hi, uint32_t& lo) {
+    const uint32_t a = __float_as_uint(p0), b = __float_as_uint(p1);
+    hi = __byte_perm(a, b, 0x7632);
+    const uint64_t rem = pf_fma2(pf_pack(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u)), neg1,
+                                 pf_pack(p0, p1));
+    const float2 r = pf_unpack(rem);
+    const __nv_bfloat162 l2 = __floats2bfloat162_rn(r.x, r.y);
+    lo = *reinterpret_cast<const uint32_t*>(&l2);
+}
+
 template <bool PAGED, bool OUT_BF16>
 __global__ void __launch_bounds__(PfCfg::THREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -175,12 +226,16 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         mbar_init(smem_addr(&ctrl->qempty), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->sfull[s]), 1);
-            mbar_init(smem_addr(&ctrl->sfree[s]), 4);
+            mbar_init(smem_addr(&ctrl->sfree[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->ofull[s]), 1);
-            mbar_init(smem_addr(&ctrl->ofree[s]), 4);
+            mbar_init(smem_addr(&ctrl->ofree[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->drain[s]), 1);
         }
-        mbar_init(smem_addr(&ctrl->pfull), 4);
+        for (int s = 0; s < 4; ++s) {
+            mbar_init(smem_addr(&ctrl->xfull[s]), 2);
+            mbar_init(smem_addr(&ctrl->xfree[s]), 2);
+        }
+        mbar_init(smem_addr(&ctrl->pfull), C::NSM);
         mbar_init(smem_addr(&ctrl->pvdone), 1);
         ctrl->abort = 0;
     }
@@ -389,9 +444,30 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
 
     if (warp >= C::WARP_SM0) {
         // ------------------------------------------------------------ softmax + epilogue
-        const int sp = warp & 3;       // tensor-memory sub-partition of this warp
-        const int r = 32 * sp + lane;  // tile row held by this thread (= TMEM lane)
+        // Two warps per tensor-memory sub-partition: warp half hf takes keys
+        // 64 hf .. 64 hf + 63 of every step (and d columns 64 hf .. of O).  The
+        // halves of a row share one reference, agreed each step from their
+        // partial maxima.
+        const int sp = warp & 3;                    // sub-partition of this warp
+        const int hf = (warp - C::WARP_SM0) >> 2;   // key half
+        const int r = 32 * sp + lane;               // tile row held by this thread (= TMEM lane)
         const float NEG_INF = -__int_as_float(0x7f800000);
+        const uint64_t neg1 = pf_pack(-1.f, -1.f);
+        const uint64_t sl2x2 = pf_pack(a.sl2, a.sl2);
+        uint32_t xpar = 0;
+        // Both halves post a per-row value and read the other's; bounded waits.
+        auto exchange = [&](float mine, float& other) -> bool {
+            if (!mbar_wait_warp(smem_addr(&ctrl->xfree[sp]), xpar ^ 1u, abort_flag)) return false;
+            ctrl->xval[hf][r] = mine;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->xfull[sp]));
+            if (!mbar_wait_warp(smem_addr(&ctrl->xfull[sp]), xpar, abort_flag)) return false;
+            other = ctrl->xval[hf ^ 1][r];
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->xfree[sp]));
+            xpar ^= 1u;
+            return true;
+        };
         int64_t g = 0;
         int uc = 0;
         bool ok = true;
@@ -404,7 +480,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
             const int hq = r - tq * a.R;   // query head of the row within the group
             const bool row_ok = tq < x.n_tok;
             const int pos = x.pos0 + tq;   // cache position of the row's token
-            float ref = NEG_INF, l = 0.f;
+            float ref = NEG_INF, l = 0.f;  // l: this half's share of the row sum
             for (int j = 0; j < x.steps; ++j, ++g) {
                 const int sb = static_cast<int>(g & 1);
                 if (!mbar_wait_warp(smem_addr(&ctrl->sfull[sb]), static_cast<uint32_t>(g >> 1) & 1u, abort_flag)) {
@@ -412,38 +488,35 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                uint32_t sv[C::BN];  // the row's scores, then its weights (fp32 bits)
+                uint32_t sv[64];  // this half's raw scores, then its weights (fp32 bits)
 #pragma unroll
-                for (int c = 0; c < C::BN / 32; ++c)
-                    tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::BN + 32 * c), sv + 32 * c);
+                for (int c = 0; c < 2; ++c)
+                    tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::BN + 64 * hf + 32 * c), sv + 32 * c);
                 tc::tmem_wait_ld();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
 
-                // Base-2 scores; key 128 j + c is visible iff it is <= pos.
-                const int lim = row_ok ? pos - C::BN * j : -1;
-                float mx8[8];
+                // Key 128 j + 64 hf + c is visible iff it is <= pos.
+                const int lim = row_ok ? pos - C::BN * j - 64 * hf : -1;
+                if (lim < 63) {
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mx8[i] = NEG_INF;
-                if (lim >= C::BN - 1) {
-#pragma unroll
-                    for (int c = 0; c < C::BN; ++c) {
-                        const float v = __uint_as_float(sv[c]) * a.sl2;
-                        sv[c] = __float_as_uint(v);
-                        mx8[c & 7] = fmaxf(mx8[c & 7], v);
-                    }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < C::BN; ++c) {
-                        const float v = c <= lim ? __uint_as_float(sv[c]) * a.sl2 : NEG_INF;
-                        sv[c] = __float_as_uint(v);
-                        mx8[c & 7] = fmaxf(mx8[c & 7], v);
-                    }
+                    for (int c = 0; c < 64; ++c)
+                        if (c > lim) sv[c] = __float_as_uint(NEG_INF);
                 }
-                const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-                // Lazy reference: weights stay <= 2^8 against it.
+                float m4[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
+#pragma unroll
+                for (int c = 0; c < 64; c += 2)
+                    m4[(c >> 1) & 3] = pf_max3(m4[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
+                float mo;
+                const float mp = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
+                if (!exchange(mp, mo)) {
+                    ok = false;
+                    break;
+                }
+                // Base-2 row maximum (scale > 0 keeps the order); lazy reference:
+                // weights stay <= 2^8 against it.
+                const float mx = fmaxf(mp, mo) * a.sl2;
                 float alpha = 1.f;
                 const bool move = mx > ref + static_cast<float>(C::T_LAZY);
                 if (move) {
@@ -452,16 +525,21 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                     l *= alpha;
                 }
                 const float rb = ref == NEG_INF ? 0.f : ref;
-                float part[8];
+                const uint64_t nrb = pf_pack(-rb, -rb);
+                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int i = 0; i < 8; ++i) part[i] = 0.f;
-#pragma unroll
-                for (int c = 0; c < C::BN; ++c) {
-                    const float pc = fast_exp2(__uint_as_float(sv[c]) - rb);
-                    sv[c] = __float_as_uint(pc);
-                    part[c & 7] += pc;
+                for (int i = 0; i < 32; ++i) {
+                    const float2 t = pf_unpack(
+                        pf_fma2(pf_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2, nrb));
+                    const float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
+                    sv[2 * i] = __float_as_uint(p0);
+                    sv[2 * i + 1] = __float_as_uint(p1);
+                    acc[i & 3] = pf_add2(acc[i & 3], pf_pack(p0, p1));
                 }
-                l += ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+                {
+                    const float2 s2 = pf_unpack(pf_add2(pf_add2(acc[0], acc[1]), pf_add2(acc[2], acc[3])));
+                    l += s2.x + s2.y;
+                }
 
                 // The P buffer and O are free once the previous step's value product is done.
                 if (g > 0 &&
@@ -470,12 +548,13 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                     break;
                 }
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
-                    // O holds this unit's earlier steps: rescale the moved rows in place.
+                    // O holds this unit's earlier steps: rescale the moved rows in place
+                    // (this half's d columns).
                     tc::fence_after_sync();
 #pragma unroll
-                    for (int c = 0; c < C::D / 32; ++c) {
+                    for (int c = 0; c < 2; ++c) {
                         uint32_t o[32];
-                        const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 32 * c);
+                        const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 64 * hf + 32 * c);
                         tc::tmem_ld32(oa, o);
                         tc::tmem_wait_ld();
 #pragma unroll
@@ -494,24 +573,21 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                         break;
                     }
                     if (C::BN * j + r >= x.L) {
-                        const uint32_t vrow = ring + e * C::TILE + r * 128;
+                        const uint32_t vrow = ring + e * C::TILE + hf * C::PANEL + r * 128;
 #pragma unroll
-                        for (int p = 0; p < 2; ++p)
-#pragma unroll
-                            for (int c = 0; c < 8; ++c)
-                                st_shared_v4(vrow + p * C::PANEL + ((c ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                        for (int c = 0; c < 8; ++c) st_shared_v4(vrow + ((c ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
                     }
                 }
-                // P = hi + lo (bf16 each), row r: keys 0..63 in the first panel, 64..127
-                // in the second, 16-byte chunks swizzled by the row's low three bits.
+                // P = hi + lo (bf16 each): this half's 64 keys fill panel hf of row r,
+                // 16-byte chunks swizzled by the row's low three bits.
 #pragma unroll
-                for (int c = 0; c < C::BN / 8; ++c) {
+                for (int c = 0; c < 8; ++c) {
                     uint32_t hi[4], lo[4];
 #pragma unroll
                     for (int w = 0; w < 4; ++w)
-                        split_bf16x2(__uint_as_float(sv[8 * c + 2 * w]), __uint_as_float(sv[8 * c + 2 * w + 1]), hi[w],
-                                     lo[w]);
-                    const uint32_t off = (c >> 3) * C::PANEL + r * 128 + (((c & 7) ^ (r & 7)) << 4);
+                        pf_split(__uint_as_float(sv[8 * c + 2 * w]), __uint_as_float(sv[8 * c + 2 * w + 1]), neg1, hi[w],
+                                 lo[w]);
+                    const uint32_t off = hf * C::PANEL + r * 128 + ((c ^ (r & 7)) << 4);
                     st_shared_v4(p_smem + off, hi[0], hi[1], hi[2], hi[3]);
                     st_shared_v4(p_smem + C::TILE + off, lo[0], lo[1], lo[2], lo[3]);
                 }
@@ -523,18 +599,21 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
             if (!ok) break;
 
             // ---------------------------------------------------- unit end: O / l -> out
-            if (!mbar_wait_warp(smem_addr(&ctrl->ofull[ob]), static_cast<uint32_t>(uc >> 1) & 1u, abort_flag)) {
+            float lo_half;
+            if (!exchange(l, lo_half) ||
+                !mbar_wait_warp(smem_addr(&ctrl->ofull[ob]), static_cast<uint32_t>(uc >> 1) & 1u, abort_flag)) {
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            const float inv = l > 0.f ? 1.f / l : 0.f;
+            const float lt = l + lo_half;
+            const float inv = lt > 0.f ? 1.f / lt : 0.f;
             const int64_t orow =
-                row_ok ? (static_cast<int64_t>(x.q_row0 + tq) * a.H_Q + x.kv * a.R + hq) * C::D : 0;
+                row_ok ? (static_cast<int64_t>(x.q_row0 + tq) * a.H_Q + x.kv * a.R + hq) * C::D + 64 * hf : 0;
 #pragma unroll
-            for (int c = 0; c < C::D / 32; ++c) {
+            for (int c = 0; c < 2; ++c) {
                 uint32_t o[32];
-                tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 32 * c), o);
+                tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 64 * hf + 32 * c), o);
                 tc::tmem_wait_ld();
                 if (row_ok) {
                     if constexpr (OUT_BF16) {

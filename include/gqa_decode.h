@@ -282,7 +282,8 @@ gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const
  *               cu_q_lens[B] = total_q; 0 <= n_b <= min(L_b, max_q_len).
  *   total_q     rows of q and out (host value).
  *   max_q_len   host upper bound on every n_b; sizes the launch.
- *   k_cache, v_cache, seq_lens, block_table, scale   as for gqa_decode.
+ *   k_cache, v_cache, seq_lens, block_table   as for gqa_decode.
+ *   scale       softmax scale, finite and > 0 (usually 1/sqrt(128)).
  *   out         [total_q, H_Q, 128] out_dtype, 16-byte aligned.  Rows of a
  *               sequence whose span is invalid are left untouched.
  *   workspace   >= gqa_prefill_workspace_size bytes (any gqa_decode
@@ -292,8 +293,8 @@ gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const
  * host: an invalid span skips that sequence and raises GQA_FLAG_BAD_QUERY_SPAN;
  * lengths and pages are handled as in gqa_decode.  Argument errors return
  * before anything is enqueued; the call allocates nothing and does not
- * synchronise.  Weights enter the value product as bf16 hi + lo parts (about
- * 16 significant bits), accumulation is fp32.
+ * synchronise.  Weights enter the value product as bf16 hi + lo parts (within
+ * 2^-15 of each weight), accumulation is fp32.
  */
 gqa_status gqa_prefill_workspace_size(const gqa_decode_params* params, size_t* bytes);
 

@@ -258,6 +258,9 @@ def test_prefill_rejects_bad_arguments_on_host(lib):
     pp = params(page_size=64, max_blocks_per_seq=4, num_blocks=8)
     assert call_prefill(lib, pp, table=None) == GQA_ERR_INVALID
     assert call_prefill(lib, p, scale=float("nan")) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, scale=0.0) == GQA_ERR_INVALID       # the scale must be positive
+    assert call_prefill(lib, p, scale=-0.1) == GQA_ERR_INVALID
+    assert call_prefill(lib, p, scale=float("inf")) == GQA_ERR_INVALID
     assert call_prefill(lib, p, ws=None) == GQA_ERR_WORKSPACE
     assert call_prefill(lib, p, ws=128) == GQA_ERR_WORKSPACE       # not 256-byte aligned
     assert call_prefill(lib, p, ws_bytes=64) == GQA_ERR_WORKSPACE   # no room for the status word
