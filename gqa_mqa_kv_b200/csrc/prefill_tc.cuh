@@ -25,13 +25,17 @@
 //                   exceeds it by more than 8 (O is rescaled in tensor memory
 //                   then); the pair agrees on the reference through a
 //                   shared-memory exchange of partial maxima each step.  P
-//                   goes to shared memory as bf16 hi and lo parts, so the
-//                   product keeps ~16 bits of every weight, in the same
-//                   K-major swizzled layout TMA would produce.
+//                   replaces S in its own tensor-memory columns as bf16 hi
+//                   and lo parts (two per 32-bit column), so the product
+//                   keeps ~16 bits of every weight and the two S buffers
+//                   double as two P buffers.
 //   O += P V        tcgen05.mma, M = 128, N = d = 128, K = 128 keys, once on
-//                   the hi part and once on the lo part; B = the value rows
-//                   read MN-major; O in tensor memory (two buffers, one per
-//                   unit in flight), normalised by the row sum at the end.
+//                   the hi part and once on the lo part; A = P read from
+//                   tensor memory, B = the value rows read MN-major; O in
+//                   tensor memory (two buffers, one per unit in flight),
+//                   normalised by the row sum at the end.  The value product
+//                   of a step releases its S/P buffer to the score product
+//                   two steps later.
 //
 // Persistent CTAs (one per SM) walk the units in a fixed interleaved order,
 // heaviest query tiles first.  Warp roles: 0 TMA producer, 1 score products
@@ -73,14 +77,13 @@ struct PfCfg {
     static constexpr int PANEL = 128 * 128;        // 128 rows x 128 bytes (64 bf16 of d, or of keys)
     static constexpr int TILE = 2 * PANEL;         // 128 rows x 128 bf16
     static constexpr int BOX = 64 * 128;           // one 64-row TMA box of 128-byte rows
-    static constexpr int NS = 4;                   // K/V ring entries (K and V of a step alternate)
+    static constexpr int NS = 6;                   // K/V ring entries (K and V of a step alternate)
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_P = OFF_Q + TILE;     // P hi, then P lo
-    static constexpr int OFF_RING = OFF_P + 2 * TILE;
+    static constexpr int OFF_RING = OFF_Q + TILE;
     static constexpr int OFF_CTRL = OFF_RING + NS * TILE;
     static constexpr int CTRL_BYTES = 2048;
     static constexpr int SMEM_BYTES = 1024 + OFF_CTRL + CTRL_BYTES;  // + 1024-byte alignment slack
-    static constexpr int S_COL = 0;                // S buffer b at S_COL + 128 b
+    static constexpr int S_COL = 0;                // S buffer b at S_COL + 128 b; P hi | lo replaces S there
     static constexpr int O_COL = 256;              // O buffer b at O_COL + 128 b
     static constexpr int TMEM_COLS = 512;
     static constexpr int WARP_TMA = 0, WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
@@ -92,7 +95,7 @@ struct PfCfg {
 struct __align__(16) PfControl {
     uint64_t full[PfCfg::NS], empty[PfCfg::NS];  // K/V ring
     uint64_t qfull, qempty;                      // query tile
-    uint64_t sfull[2], sfree[2];                 // S buffer written / read by the softmax warps
+    uint64_t sfull[2], sfree[2];                 // S buffer written / its P read by the value product
     uint64_t pfull, pvdone;                      // P written / value product of the last step done
     uint64_t ofull[2], ofree[2];                 // O buffer of a unit complete / read by the epilogue
     uint64_t drain[2];                           // last products of each issuing warp complete
@@ -203,7 +206,6 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* base_ptr = smem_raw + (base - raw);
     const uint32_t q_smem = base + C::OFF_Q;
-    const uint32_t p_smem = base + C::OFF_P;
     const uint32_t ring = base + C::OFF_RING;
     PfControl* ctrl = reinterpret_cast<PfControl*>(base_ptr + C::OFF_CTRL);
     volatile int* abort_flag = &ctrl->abort;
@@ -226,7 +228,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         mbar_init(smem_addr(&ctrl->qempty), 1);
         for (int s = 0; s < 2; ++s) {
             mbar_init(smem_addr(&ctrl->sfull[s]), 1);
-            mbar_init(smem_addr(&ctrl->sfree[s]), C::NSM);
+            mbar_init(smem_addr(&ctrl->sfree[s]), 1);  // committed by the value product
             mbar_init(smem_addr(&ctrl->ofull[s]), 1);
             mbar_init(smem_addr(&ctrl->ofree[s]), C::NSM);
             mbar_init(smem_addr(&ctrl->drain[s]), 1);
@@ -344,8 +346,8 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
 
     if (warp == C::WARP_QK) {
         // ------------------------------------------------------------ score products
-        // Global step g: S(g) = Q K(g)^T into buffer g & 1 once the softmax warps
-        // have read that buffer's previous contents (step g - 2).
+        // Global step g: S(g) = Q K(g)^T into buffer g & 1 once the value product
+        // of step g - 2 has read the P that replaced that buffer's S.
         int64_t g = 0;
         int uc = 0;
         bool ok = true;
@@ -394,9 +396,10 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
 
     if (warp == C::WARP_PV) {
         // ------------------------------------------------------------ value products
-        // Global step g: O += P_hi V(g) + P_lo V(g) once the softmax warps have
-        // written P(g); a unit's first step overwrites its O buffer after the
-        // epilogue has read that buffer's previous unit.
+        // Global step g: O += P_hi V(g) + P_lo V(g), A read from tensor memory
+        // (the P that replaced S(g)), once the softmax warps have written P(g);
+        // a unit's first step overwrites its O buffer after the epilogue has
+        // read that buffer's previous unit.
         int64_t g = 0;
         int uc = 0;
         bool ok = true;
@@ -418,17 +421,19 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                 tc::fence_after_sync();
                 if (tc::elect_one()) {
                     const uint32_t vt = ring + e * C::TILE;
+                    const int sb = static_cast<int>(g & 1);
 #pragma unroll
                     for (int part = 0; part < 2; ++part)
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
-                            const uint64_t da = tc::smem_desc(p_smem + part * C::TILE + (k >> 2) * C::PANEL + 32 * (k & 3),
-                                                              16, 1024, tc::kLayoutSw128);
+                            // 16 keys = 8 packed columns of P; 16 value rows
+                            const uint32_t pa = tmem + C::S_COL + sb * C::BN + part * 64 + 8 * k;
                             const uint64_t db = tc::smem_desc(vt + k * 2048, C::PANEL, 1024, tc::kLayoutSw128);
-                            tc::mma_f16(tmem + C::O_COL + ob * C::D, da, db, IDESC_PV,
-                                        !(j == 0 && part == 0 && k == 0));
+                            tc::mma_f16_ts(tmem + C::O_COL + ob * C::D, pa, db, IDESC_PV,
+                                           !(j == 0 && part == 0 && k == 0));
                         }
                     tc::commit(smem_addr(&ctrl->empty[e]));
+                    tc::commit(smem_addr(&ctrl->sfree[sb]));
                     tc::commit(smem_addr(&ctrl->pvdone));
                     if (j == x.steps - 1) tc::commit(smem_addr(&ctrl->ofull[ob]));
                 }
@@ -456,12 +461,16 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         const uint64_t sl2x2 = pf_pack(a.sl2, a.sl2);
         uint32_t xpar = 0;
         // Both halves post a per-row value and read the other's; bounded waits.
+        // It also orders each half's tensor-memory reads of S before the other
+        // half's writes of P over the same columns.
         auto exchange = [&](float mine, float& other) -> bool {
             if (!mbar_wait_warp(smem_addr(&ctrl->xfree[sp]), xpar ^ 1u, abort_flag)) return false;
             ctrl->xval[hf][r] = mine;
+            tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&ctrl->xfull[sp]));
             if (!mbar_wait_warp(smem_addr(&ctrl->xfull[sp]), xpar, abort_flag)) return false;
+            tc::fence_after_sync();
             other = ctrl->xval[hf ^ 1][r];
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(&ctrl->xfree[sp]));
@@ -493,9 +502,6 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                 for (int c = 0; c < 2; ++c)
                     tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::BN + 64 * hf + 32 * c), sv + 32 * c);
                 tc::tmem_wait_ld();
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&ctrl->sfree[sb]));
 
                 // Key 128 j + 64 hf + c is visible iff it is <= pos.
                 const int lim = row_ok ? pos - C::BN * j - 64 * hf : -1;
@@ -541,15 +547,14 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                     l += s2.x + s2.y;
                 }
 
-                // The P buffer and O are free once the previous step's value product is done.
-                if (g > 0 &&
-                    !mbar_wait_warp(smem_addr(&ctrl->pvdone), static_cast<uint32_t>(g - 1) & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
-                    // O holds this unit's earlier steps: rescale the moved rows in place
-                    // (this half's d columns).
+                    // O holds this unit's earlier steps: once the previous step's value
+                    // product is done, rescale the moved rows in place (this half's d
+                    // columns).
+                    if (!mbar_wait_warp(smem_addr(&ctrl->pvdone), static_cast<uint32_t>(g - 1) & 1u, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
                     tc::fence_after_sync();
 #pragma unroll
                     for (int c = 0; c < 2; ++c) {
@@ -577,21 +582,21 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
 #pragma unroll
                         for (int c = 0; c < 8; ++c) st_shared_v4(vrow + ((c ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
                     }
+                    pf_fence_async_smem();
                 }
-                // P = hi + lo (bf16 each): this half's 64 keys fill panel hf of row r,
-                // 16-byte chunks swizzled by the row's low three bits.
+                // P = hi + lo (bf16 pairs) over S's own columns: hi of keys
+                // 64 hf .. at columns 32 hf .., lo at 64 + 32 hf .. (both halves have
+                // read their scores: the exchange above orders it).
+                {
+                    uint32_t hi[32], lo[32];
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int w = 0; w < 4; ++w)
-                        pf_split(__uint_as_float(sv[8 * c + 2 * w]), __uint_as_float(sv[8 * c + 2 * w + 1]), neg1, hi[w],
-                                 lo[w]);
-                    const uint32_t off = hf * C::PANEL + r * 128 + ((c ^ (r & 7)) << 4);
-                    st_shared_v4(p_smem + off, hi[0], hi[1], hi[2], hi[3]);
-                    st_shared_v4(p_smem + C::TILE + off, lo[0], lo[1], lo[2], lo[3]);
+                    for (int w = 0; w < 32; ++w)
+                        pf_split(__uint_as_float(sv[2 * w]), __uint_as_float(sv[2 * w + 1]), neg1, hi[w], lo[w]);
+                    const uint32_t pcol = C::S_COL + sb * C::BN + 32 * hf;
+                    tc::tmem_st32(tc::tmem_addr(tmem, 32 * sp, pcol), hi);
+                    tc::tmem_st32(tc::tmem_addr(tmem, 32 * sp, pcol + 64), lo);
+                    tc::tmem_wait_st();
                 }
-                pf_fence_async_smem();
                 tc::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull));
