@@ -178,24 +178,37 @@ class ClockSampler:
                 "power_w_max": max(power), "reasons": sorted(reasons), "samples": len(sm)}
 
 
-def kernel_source_hash() -> str:
+# Sources each measured kernel is built from (the host file gqa_decode.cu and
+# the shared headers count for both).
+_PREFILL_ONLY = {"prefill_tc.cuh"}
+_DECODE_ONLY = {"split_mma.cuh", "split_tc.cuh", "split_simt.cuh", "combine.cuh", "rope_append.cuh"}
+
+
+def kernel_source_hash(kind: str = "decode") -> str:
+    """sha256 (first 16 hex digits) over the csrc files of the decode or the
+    prefill kernels."""
+    skip = _PREFILL_ONLY if kind == "decode" else _DECODE_ONLY
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gqa_mqa_kv_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
+        if name in skip:
+            continue
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(workload: str):
-    """DRAM bytes per split-kernel launch from the committed ncu summary, if it
-    was taken on the current kernel source; else None."""
+    """DRAM bytes per launch of the workload's dominant kernel from the
+    committed ncu summary, if it was taken on the current source of that
+    kernel; else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    kind = "prefill" if workload in PREFILL_WORKLOADS else "decode"
     try:
         with open(path) as f:
             rec = json.load(f)
         ent = rec.get(workload)
-        if ent and ent.get("kernel_source_hash") == kernel_source_hash():
+        if ent and ent.get("kernel_source_hash") == kernel_source_hash(kind):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         pass
