@@ -18,7 +18,9 @@ SRC = os.path.join(ROOT, "oracle", "gqa_oracle.cpp")
 MUTANTS = {
     "strided_group_map": ("    return h / R;", "    return h % p.H_KV;"),
     "dropped_scale": ("    return p.scale * ks * acc;", "    return ks * acc;"),
-    "exponent_sign": ("        s[t] = std::exp(s[t] - m);", "        s[t] = std::exp(m - s[t]);"),
+    "exponent_sign": ("    for (int64_t t = 0; t < L; ++t) {\n        s[t] = std::exp(s[t] - m);",
+                      "    for (int64_t t = 0; t < L; ++t) {\n        s[t] = std::exp(m - s[t]);"),
+    "prefill_exponent_sign": ("            s[t] = std::exp(s[t] - m);", "            s[t] = std::exp(m - s[t]);"),
     "drops_last_token": ("    int64_t L = p.seq_lens[b];\n    std::vector<double> s(",
                          "    int64_t L = p.seq_lens[b] > 1 ? p.seq_lens[b] - 1 : p.seq_lens[b];\n    std::vector<double> s("),
     "values_from_keys": ("            out[i] += w[t] * vs * load_elem(p.v, p.kv_dtype, kv_index(p, b, t, g, i));",
