@@ -1,11 +1,14 @@
 /*
- * gqa_decode.h -- C ABI of the B200 grouped-query attention decode library.
+ * gqa_decode.h -- C ABI of the B200 grouped-query attention library.
  *
- * One call computes one decode step of one attention layer: every query head
- * of every sequence attends, with a single new query token, over that
- * sequence's cached keys and values.  Key/value head g of the cache serves
- * the R = H_Q / H_KV query heads h with g = floor(h / R) and is read from HBM
- * once for all of them.
+ * One gqa_decode call computes one decode step of one attention layer: every
+ * query head of every sequence attends, with a single new query token, over
+ * that sequence's cached keys and values.  Key/value head g of the cache
+ * serves the R = H_Q / H_KV query heads h with g = floor(h / R) and is read
+ * from HBM once for all of them.  gqa_prefill computes the multi-token step
+ * (fresh prompts, or prompt chunks after a cached prefix) with the causal
+ * mask; gqa_rope_append and gqa_decode_fp8kv cover the step before decode and
+ * an 8-bit cache.
  *
  * Defining passages (cited by page title and section):
  *   [LLMS] "Grouped-Query Attention (GQA) and Multi-Query Attention (MQA):

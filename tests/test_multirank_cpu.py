@@ -134,6 +134,29 @@ def rank_tp_dup_shards(rank, world):
     return bool(np.array_equal(got, full))
 
 
+def rank_tp_prefill_shards(rank, world):
+    # The multi-token step shards by heads the same way: each rank runs the
+    # causal step on its query heads and their (possibly duplicated) KV heads.
+    import numpy as np
+
+    import oracle
+    from gqa_mqa_kv_b200.sharding import tp_head_shard
+    from gqa_mqa_kv_b200.workloads import PrefillWorkload, make_prefill_inputs
+
+    dist.init_process_group("gloo")
+    w = PrefillWorkload("tp", 3, 8, 2, 16, 1, 0, seed=31)
+    n, L = np.array([5, 1, 9]), np.array([12, 7, 9])
+    inp = make_prefill_inputs(w, lengths=(n, L))
+    qs, ks = tp_head_shard(w.H_Q, w.H_KV, world, rank)
+    mine = oracle.gqa_prefill(inp["q"][:, qs].contiguous(), inp["k"][:, :, ks].contiguous(),
+                              inp["v"][:, :, ks].contiguous(), inp["seq_lens"], inp["cu_q"], w.softmax_scale)
+    parts = [None] * world
+    dist.all_gather_object(parts, (qs.start, mine))
+    got = np.concatenate([m for _, m in sorted(parts, key=lambda x: x[0])], axis=1)
+    full = oracle.gqa_prefill(inp["q"], inp["k"], inp["v"], inp["seq_lens"], inp["cu_q"], w.softmax_scale)
+    return bool(np.array_equal(got, full))
+
+
 def rank_reference_arm(rank, world):
     import bench
 
@@ -187,3 +210,9 @@ def test_duplicated_kv_shards_keep_each_query_head_on_its_own_group():
 
 def test_tensor_parallel_with_duplicated_kv_reassembles_the_full_step():
     assert run_ranks("rank_tp_dup_shards", world=4) == {0: True, 1: True, 2: True, 3: True}
+
+
+def test_tensor_parallel_prefill_shards_reassemble_the_full_step():
+    assert run_ranks("rank_tp_prefill_shards") == {0: True, 1: True}
+    # four ranks over two KV heads: duplicated KV, one group slice per rank
+    assert run_ranks("rank_tp_prefill_shards", world=4) == {0: True, 1: True, 2: True, 3: True}

@@ -39,3 +39,28 @@ def test_tp_shards_reassemble_the_full_step(cuda_device, world, h_q, h_kv):
     assert_parity(got, oracle_full(inp, w), f"TP {world} over {h_q}/{h_kv}")
     full = run_gpu(inp, w, cuda_device)
     assert (got - full).abs().max().item() < 1e-4
+
+
+@pytest.mark.parametrize("world,h_q,h_kv", [(2, 64, 8), (8, 32, 4), (4, 32, 2)])
+def test_tp_prefill_shards_reassemble_the_full_step(cuda_device, world, h_q, h_kv):
+    # The multi-token step shards the same way; every shard is an ordinary
+    # gqa_prefill call on its query heads and their (possibly duplicated) KV heads.
+    import numpy as np
+
+    import oracle
+    from gqa_mqa_kv_b200.workloads import PrefillWorkload, make_prefill_inputs
+
+    w = PrefillWorkload("tp", 3, h_q, h_kv, 128, 1, 0, seed=32)
+    n, L = np.array([150, 1, 70]), np.array([150, 260, 300])
+    inp = make_prefill_inputs(w, pad_value=float("nan"), lengths=(n, L))
+    d = to_device(inp, cuda_device)
+    parts = []
+    for rank in range(world):
+        qs, ks = tp_head_shard(h_q, h_kv, world, rank)
+        parts.append(gq.gqa_prefill(d["q"][:, qs].contiguous(), d["k"][:, :, ks].contiguous(),
+                                    d["v"][:, :, ks].contiguous(), d["seq_lens"], d["cu_q"], max_q_len=d["max_q"]))
+    got = torch.cat(parts, dim=1).cpu()
+    ref = oracle.gqa_prefill(inp["q"], inp["k"], inp["v"], inp["seq_lens"], inp["cu_q"], w.softmax_scale)
+    assert_parity(got, ref, f"TP prefill {world} over {h_q}/{h_kv}")
+    full = gq.gqa_prefill(d["q"], d["k"], d["v"], d["seq_lens"], d["cu_q"], max_q_len=d["max_q"]).cpu()
+    assert (got - full).abs().max().item() < 1e-4
