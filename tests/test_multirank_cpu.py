@@ -182,6 +182,18 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert run_ranks("rank_reference_arm") == {0: 0, 1: 0}
 
 
+def rank_reference_arm_prefill(rank, world):
+    import bench
+
+    if rank != 0:
+        return bench.main(["--impl", "reference", "--gpus", str(world), "--workload", "prefill_llama3_8b"])
+    return 0  # only the non-zero ranks' early exit is checked here
+
+
+def test_prefill_reference_arm_runs_on_rank_zero_only():
+    assert run_ranks("rank_reference_arm_prefill") == {0: 0, 1: 0}
+
+
 def test_shard_helpers():
     from gqa_mqa_kv_b200.sharding import batch_shard, tp_head_shard
 
