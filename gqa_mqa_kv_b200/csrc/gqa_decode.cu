@@ -684,8 +684,8 @@ gqa_status gqa_prefill(const gqa_decode_params* params, const void* q, const int
     if (!(scale > 0.f) || !std::isfinite(scale)) return GQA_ERR_INVALID;  // a positive scale keeps the score order
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < kHeaderBytes) return GQA_ERR_WORKSPACE;
 
-    const int TQ = 128 / R;
-    const int64_t QT = (static_cast<int64_t>(max_q_len) + TQ - 1) / TQ;
+    const int TQ = 128 / R;  // query tokens per 128-row tile; a unit is two tiles
+    const int64_t QT = (static_cast<int64_t>(max_q_len) + 2 * TQ - 1) / (2 * TQ);
     const int64_t units = static_cast<int64_t>(p->B) * p->H_KV * QT;
     if (units >= (int64_t(1) << 31)) return GQA_ERR_UNSUPPORTED;
     DeviceInfo dev;

@@ -9,41 +9,44 @@
 // -- whose keys and values are the last n_b of its L_b cached tokens.  Token
 // j sits at position p = L_b - n_b + j and attends to cache positions t <= p.
 //
-// Work unit: TQ = floor(128 / R) consecutive query tokens of one sequence
+// Query tile: TQ = floor(128 / R) consecutive query tokens of one sequence
 // and one KV head kv, as one M = 128 row tile whose row r is token r / R and
-// query head kv R + r % R: every K/V row brought on chip serves all R heads
-// of the group.  The unit walks its visible keys 128 at a time:
-//   S = Q K^T       tcgen05.mma, M = 128 rows, N = 128 keys, K = d: A = the
+// query head kv R + r % R, so every K/V row brought on chip serves all R
+// heads of the group.  Work unit: two consecutive query tiles (tile 0 and
+// tile 1, 2 TQ tokens) that share every K/V step, so each staged K/V row
+// serves 256 rows and one tile's softmax runs while the tensor cores work on
+// the other tile.  The unit walks its visible keys 128 at a time:
+//   S_t = Q_t K^T   tcgen05.mma, M = 128 rows, N = 128 keys, K = d: A = the
 //                   query rows, B = the key rows, both K-major with the
-//                   128-byte swizzle as TMA stages them; S lands in tensor
-//                   memory (two buffers: the next step's product overlaps
-//                   this step's softmax).
-//   softmax         eight warps, two per tensor-memory sub-partition:
-//                   thread = row = TMEM lane, each warp of a pair taking 64
-//                   of the step's keys in registers.  Base-2 online softmax
-//                   against a per-row reference that moves only when a score
-//                   exceeds it by more than 8 (O is rescaled in tensor memory
-//                   then); the pair agrees on the reference through a
-//                   shared-memory exchange of partial maxima each step.  P
-//                   replaces S in its own tensor-memory columns as bf16 hi
-//                   and lo parts (two per 32-bit column), so the product
-//                   keeps ~16 bits of every weight and the two S buffers
-//                   double as two P buffers.
-//   O += P V        tcgen05.mma, M = 128, N = d = 128, K = 128 keys, once on
+//                   128-byte swizzle as TMA stages them; S_t in tensor memory.
+//   softmax         four warps per tile, one per tensor-memory sub-partition:
+//                   thread = row = TMEM lane, all 128 keys of the step in
+//                   registers, so the row maximum needs no exchange.  Base-2
+//                   online softmax against a per-row reference that moves
+//                   only when a score exceeds it by more than 8 (O_t is
+//                   rescaled in tensor memory then).  P replaces S_t in its
+//                   own columns as bf16 hi and lo parts: keys 32c .. 32c+31
+//                   go to columns 32c .. 32c+15 (hi, two keys per column) and
+//                   32c+16 .. 32c+31 (lo), so the product keeps ~16 bits of
+//                   every weight.
+//   O_t += P V      tcgen05.mma, M = 128, N = d = 128, K = 128 keys, once on
 //                   the hi part and once on the lo part; A = P read from
-//                   tensor memory, B = the value rows read MN-major; O in
-//                   tensor memory (two buffers, one per unit in flight),
-//                   normalised by the row sum at the end.  The value product
-//                   of a step releases its S/P buffer to the score product
-//                   two steps later.
+//                   tensor memory, B = the value rows read MN-major; O_t in
+//                   tensor memory, normalised by the row sum at the unit end.
+//
+// One thread issues every product, per step i in the order
+//   S_0(i), O_1 += P_1(i-1) V(i-1), S_1(i), O_0 += P_0(i) V(i)
+// so each tile's softmax is covered by two products of the other tile.  The
+// score product that overwrites S_t columns still holding P_t of the step
+// before is issued after the value product that reads them: tcgen05.mma
+// operations of one thread execute in issue order.
 //
 // Persistent CTAs (one per SM) walk the units in a fixed interleaved order,
-// heaviest query tiles first.  Warp roles: 0 TMA producer, 1 score products
-// (+ tensor-memory allocation), 2 value products, 3..10 softmax and epilogue
-// (warp w on sub-partition w % 4, keys 64 ((w - 3) / 4) ..).  Every wait is
-// bounded (kWaitTimeoutNs); on a
-// timeout the CTA raises GQA_FLAG_TIMEOUT, lets its copies and products
-// drain, frees its tensor memory and returns.
+// heaviest first.  Warp roles: 0 TMA producer, 1 tensor-core issue
+// (+ tensor-memory allocation), 2..3 idle, 4..7 softmax and epilogue of
+// tile 0, 8..11 of tile 1 (warp w on sub-partition w % 4).  Every wait is bounded
+// (kWaitTimeoutNs); on a timeout the CTA raises GQA_FLAG_TIMEOUT, lets its
+// copies and products drain, frees its tensor memory and returns.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -60,7 +63,7 @@ struct PrefillArgs {
     const int32_t* block_table;  // [B, max_blocks] or null
     int B, H_Q, H_KV, R;
     int TQ;          // query tokens per tile: floor(128 / R)
-    int QT;          // tiles per sequence: ceil(max_q / TQ)
+    int QT;          // units (tile pairs) per sequence: ceil(max_q / (2 TQ))
     int max_q;       // host bound on n_b
     int total_q;     // rows of q and out
     int max_len;     // seq_lens are clamped to [0, max_len]
@@ -77,48 +80,52 @@ struct PfCfg {
     static constexpr int PANEL = 128 * 128;        // 128 rows x 128 bytes (64 bf16 of d, or of keys)
     static constexpr int TILE = 2 * PANEL;         // 128 rows x 128 bf16
     static constexpr int BOX = 64 * 128;           // one 64-row TMA box of 128-byte rows
-    static constexpr int NS = 6;                   // K/V ring entries (K and V of a step alternate)
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_RING = OFF_Q + TILE;
+    static constexpr int NS = 5;                   // K/V ring entries (K and V of a step alternate)
+    static constexpr int OFF_Q = 0;                // query tile t at OFF_Q + t TILE
+    static constexpr int OFF_RING = OFF_Q + 2 * TILE;
     static constexpr int OFF_CTRL = OFF_RING + NS * TILE;
     static constexpr int CTRL_BYTES = 2048;
     static constexpr int SMEM_BYTES = 1024 + OFF_CTRL + CTRL_BYTES;  // + 1024-byte alignment slack
-    static constexpr int S_COL = 0;                // S buffer b at S_COL + 128 b; P hi | lo replaces S there
-    static constexpr int O_COL = 256;              // O buffer b at O_COL + 128 b
+    static constexpr int S_COL = 0;                // S_t at S_COL + 128 t; P_t hi | lo replaces it
+    static constexpr int O_COL = 256;              // O_t at O_COL + 128 t
     static constexpr int TMEM_COLS = 512;
-    static constexpr int WARP_TMA = 0, WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
-    static constexpr int NSM = 8;                  // softmax warps: two per sub-partition, 64 keys each
-    static constexpr int THREADS = 32 * (3 + NSM);
+    // Three warpgroups: 0 = TMA producer, tensor-core issue and two idle warps;
+    // 1 and 2 = softmax of tile 0 and tile 1.  Registers move from group 0 to
+    // the softmax groups (setmaxnreg): 128 x REG_LOW + 256 x REG_HIGH must not
+    // exceed the 384 x 168 the block is launched with.
+    static constexpr int WARP_TMA = 0, WARP_MMA = 1, WARP_SM0 = 4;
+    static constexpr int NSM = 8;                  // softmax warps: four per tile
+    static constexpr int THREADS = 32 * (WARP_SM0 + NSM);
+    static constexpr int REG_LAUNCH = 168, REG_LOW = 88, REG_HIGH = 208;
     static constexpr int T_LAZY = 8;               // reference slack, base 2
 };
 
 struct __align__(16) PfControl {
     uint64_t full[PfCfg::NS], empty[PfCfg::NS];  // K/V ring
-    uint64_t qfull, qempty;                      // query tile
-    uint64_t sfull[2], sfree[2];                 // S buffer written / its P read by the value product
-    uint64_t pfull, pvdone;                      // P written / value product of the last step done
-    uint64_t ofull[2], ofree[2];                 // O buffer of a unit complete / read by the epilogue
-    uint64_t drain[2];                           // last products of each issuing warp complete
-    uint64_t xfull[4], xfree[4];                 // per sub-partition: both halves wrote / read xval
+    uint64_t qfull, qempty;                      // the unit's two query tiles
+    uint64_t sfull[2];                           // S_t of a step written
+    uint64_t pfull[2];                           // P_t of a step written (four softmax warps)
+    uint64_t ofull[2], ofree[2];                 // O_t of a unit complete / read by the epilogue
+    uint64_t drain;                              // every issued product complete
     uint32_t tmem_base;
     int abort;
-    float xval[2][128];                          // per key half, per row: a partial row max or row sum
 };
 
-// One work unit as every warp role derives it from the unit index.
+// One work unit (a pair of query tiles) as every warp role derives it from
+// the unit index.
 struct PfUnit {
     int b, kv, qt;
-    int n_tok;   // query tokens in the tile (rows n_tok * R .. 127 are idle)
-    int q_row0;  // row of q / out of the tile's first token
-    int pos0;    // cache position of the tile's first token
+    int n_tok;   // query tokens in the pair (tokens past it in a tile are idle rows)
+    int q_row0;  // row of q / out of the pair's first token
+    int pos0;    // cache position of the pair's first token
     int L;       // clamped cache length
     int steps;   // 128-key steps: keys [0, pos0 + n_tok) are visible to some row
 };
 
-// Unit u: query tile qt = QT - 1 - u / (B H_KV) (heaviest first), then
-// sequence b, then KV head.  Returns false for a unit with no rows; *flags
-// gets the status bits the sequence's bounds raise (a clamped length, an
-// inconsistent query span -- such a sequence is skipped).
+// Unit u: pair qt = QT - 1 - u / (B H_KV) (heaviest first), then sequence b,
+// then KV head.  Returns false for a unit with no rows; *flags gets the status
+// bits the sequence's bounds raise (a clamped length, an inconsistent query
+// span -- such a sequence is skipped).
 __device__ __forceinline__ bool pf_unit(const PrefillArgs& a, int u, PfUnit& x, uint32_t* flags) {
     const int per = a.B * a.H_KV;
     const int t = u / per;
@@ -135,9 +142,9 @@ __device__ __forceinline__ bool pf_unit(const PrefillArgs& a, int u, PfUnit& x, 
     if (!span_ok) f |= kFlagBadSpan;
     *flags = f;
     if (!span_ok) return false;
-    const int tok0 = x.qt * a.TQ;
+    const int tok0 = x.qt * 2 * a.TQ;
     if (tok0 >= n) return false;
-    x.n_tok = min(a.TQ, n - tok0);
+    x.n_tok = min(2 * a.TQ, n - tok0);
     x.q_row0 = c0 + tok0;
     x.pos0 = x.L - n + tok0;
     x.steps = (x.pos0 + x.n_tok + PfCfg::BN - 1) / PfCfg::BN;
@@ -192,12 +199,24 @@ __device__ __forceinline__ void pf_split(float p0, float p1, uint64_t neg1, uint
     lo = *reinterpret_cast<const uint32_t*>(&l2);
 }
 
+// Warpgroup-wide register budget changes (every warp of the warpgroup executes them).
+template <int N>
+__device__ __forceinline__ void reg_alloc() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dealloc() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 template <bool PAGED, bool OUT_BF16>
 __global__ void __launch_bounds__(PfCfg::THREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const PrefillArgs a) {
     using C = PfCfg;
     static_assert(sizeof(PfControl) <= C::CTRL_BYTES, "control block overflows its slot");
+    static_assert(128 * C::REG_LOW + 256 * C::REG_HIGH <= C::THREADS * C::REG_LAUNCH,
+                  "the register split must fit the registers the block is launched with");
     constexpr uint32_t IDESC_QK = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 128, C::BN);
     constexpr uint32_t IDESC_PV = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 1, 128, C::D);
 
@@ -226,25 +245,19 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         }
         mbar_init(smem_addr(&ctrl->qfull), 1);
         mbar_init(smem_addr(&ctrl->qempty), 1);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_addr(&ctrl->sfull[s]), 1);
-            mbar_init(smem_addr(&ctrl->sfree[s]), 1);  // committed by the value product
-            mbar_init(smem_addr(&ctrl->ofull[s]), 1);
-            mbar_init(smem_addr(&ctrl->ofree[s]), C::NSM);
-            mbar_init(smem_addr(&ctrl->drain[s]), 1);
+        for (int t = 0; t < 2; ++t) {
+            mbar_init(smem_addr(&ctrl->sfull[t]), 1);
+            mbar_init(smem_addr(&ctrl->pfull[t]), 4);
+            mbar_init(smem_addr(&ctrl->ofull[t]), 1);
+            mbar_init(smem_addr(&ctrl->ofree[t]), 4);
         }
-        for (int s = 0; s < 4; ++s) {
-            mbar_init(smem_addr(&ctrl->xfull[s]), 2);
-            mbar_init(smem_addr(&ctrl->xfree[s]), 2);
-        }
-        mbar_init(smem_addr(&ctrl->pfull), C::NSM);
-        mbar_init(smem_addr(&ctrl->pvdone), 1);
+        mbar_init(smem_addr(&ctrl->drain), 1);
         ctrl->abort = 0;
     }
-    // Query rows the TMA box leaves out (R * TQ < 128) stay zero.
-    for (int i = threadIdx.x; i < C::TILE / 16; i += blockDim.x)
+    // Query rows the TMA boxes leave out (R * TQ < 128) stay zero.
+    for (int i = threadIdx.x; i < 2 * C::TILE / 16; i += blockDim.x)
         reinterpret_cast<uint4*>(base_ptr + C::OFF_Q)[i] = make_uint4(0, 0, 0, 0);
-    if (warp == C::WARP_QK) {
+    if (warp == C::WARP_MMA) {
         tc::tmem_alloc(smem_addr(&ctrl->tmem_base), C::TMEM_COLS);
         tc::tmem_relinquish();
     }
@@ -260,9 +273,11 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         if (lane == 0) atomicOr(a.status, kFlagTimeout);
     };
 
+    if (warp < C::WARP_SM0) {
+    reg_dealloc<C::REG_LOW>();
     if (warp == C::WARP_TMA) {
         // ------------------------------------------------------------ producer
-        // K/V rows are read again by the sequence's other query tiles: keep them in L2.
+        // K/V rows are read again by the sequence's other units: keep them in L2.
         const uint64_t pol_kv = policy_evict_last();
         const uint64_t pol_q = policy_evict_first();
         int64_t ld = 0;  // K/V loads issued: K of step g is load 2g, V is 2g + 1
@@ -279,10 +294,13 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                 break;
             }
             if (lane == 0) {
+                // Both tiles: TQ tokens x R heads each; a box reaching past total_q reads zeros.
                 const uint32_t bar = smem_addr(&ctrl->qfull);
-                mbar_arrive_expect_tx(bar, 2u * 128u * static_cast<uint32_t>(a.R * a.TQ));
-                for (int p = 0; p < 2; ++p)
-                    tma_load_3d(q_smem + p * C::PANEL, &tmQ, bar, 64 * p, x.kv * a.R, x.q_row0, pol_q);
+                mbar_arrive_expect_tx(bar, 2u * 2u * 128u * static_cast<uint32_t>(a.R * a.TQ));
+                for (int t = 0; t < 2; ++t)
+                    for (int p = 0; p < 2; ++p)
+                        tma_load_3d(q_smem + t * C::TILE + p * C::PANEL, &tmQ, bar, 64 * p, x.kv * a.R,
+                                    x.q_row0 + t * a.TQ, pol_q);
             }
             ++uc;
             const int kv_end = x.pos0 + x.n_tok;
@@ -344,138 +362,44 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         }
     }
 
-    if (warp == C::WARP_QK) {
-        // ------------------------------------------------------------ score products
-        // Global step g: S(g) = Q K(g)^T into buffer g & 1 once the value product
-        // of step g - 2 has read the P that replaced that buffer's S.
-        int64_t g = 0;
-        int uc = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-            PfUnit x;
-            uint32_t fl;
-            if (!pf_unit(a, u, x, &fl)) continue;
-            if (!mbar_wait_warp(smem_addr(&ctrl->qfull), static_cast<uint32_t>(uc) & 1u, abort_flag)) {
-                ok = false;
-                break;
+    if (warp == C::WARP_MMA) {
+        // ------------------------------------------------------------ tensor-core issue
+        // Global step g of this CTA: K(g) is ring load 2g, V(g) load 2g + 1.
+        auto stage = [&](int64_t li) { return ring + static_cast<uint32_t>(li % C::NS) * C::TILE; };
+        auto loaded = [&](int64_t li) {
+            return mbar_wait_warp(smem_addr(&ctrl->full[li % C::NS]), static_cast<uint32_t>((li / C::NS) & 1),
+                                  abort_flag);
+        };
+        // S_t = Q_t K^T (8 products of K = 16).  Descriptor start addresses are
+        // advanced by adding (offset >> 4) to the descriptor: every operand lies
+        // below 256 KB, so the 14-bit address field never carries.
+        auto issue_qk = [&](int t, uint32_t kt) {
+            const uint64_t da0 = tc::smem_desc(q_smem + t * C::TILE, 16, 1024, tc::kLayoutSw128);
+            const uint64_t db0 = tc::smem_desc(kt, 16, 1024, tc::kLayoutSw128);
+            const uint32_t d = tmem + C::S_COL + 128 * t;
+#pragma unroll 1
+            for (int k = 0; k < 8; ++k) {
+                const uint64_t off = static_cast<uint64_t>(((k >> 2) * C::PANEL + 32 * (k & 3)) >> 4);
+                tc::mma_f16(d, da0 + off, db0 + off, IDESC_QK, k > 0);
             }
-            for (int j = 0; j < x.steps; ++j, ++g) {
-                const int sb = static_cast<int>(g & 1);
-                const uint32_t spar = static_cast<uint32_t>(g >> 1) & 1u;
-                const int64_t ki = 2 * g;
-                const int e = static_cast<int>(ki % C::NS);
-                if (!mbar_wait_warp(smem_addr(&ctrl->sfree[sb]), spar ^ 1u, abort_flag) ||
-                    !mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(ki / C::NS) & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                if (tc::elect_one()) {
-                    const uint32_t kt = ring + e * C::TILE;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const uint32_t off = (k >> 2) * C::PANEL + 32 * (k & 3);
-                        const uint64_t da = tc::smem_desc(q_smem + off, 16, 1024, tc::kLayoutSw128);
-                        const uint64_t db = tc::smem_desc(kt + off, 16, 1024, tc::kLayoutSw128);
-                        tc::mma_f16(tmem + C::S_COL + sb * C::BN, da, db, IDESC_QK, k > 0);
-                    }
-                    tc::commit(smem_addr(&ctrl->sfull[sb]));
-                    tc::commit(smem_addr(&ctrl->empty[e]));
-                    if (j == x.steps - 1) tc::commit(smem_addr(&ctrl->qempty));
-                }
-                __syncwarp();
+        };
+        // O_t += P_hi V + P_lo V; keys 32c .. 32c+31 have hi at columns 32c .. +15, lo at 32c+16 .. +31
+        auto issue_pv = [&](int t, uint32_t vt, bool fresh) {
+            const uint64_t db0 = tc::smem_desc(vt, C::PANEL, 1024, tc::kLayoutSw128);
+            const uint32_t pa0 = tmem + C::S_COL + 128 * t;
+            const uint32_t d = tmem + C::O_COL + 128 * t;
+#pragma unroll 1
+            for (int i = 0; i < 16; ++i) {
+                const int part = i >> 3, k = i & 7;
+                tc::mma_f16_ts(d, pa0 + 32 * (k >> 1) + 16 * part + 8 * (k & 1), db0 + static_cast<uint64_t>(k * 128),
+                               IDESC_PV, !(fresh && i == 0));
             }
-            ++uc;
-        }
-        if (!ok) fail();
-        // Every product this warp issued has completed before tensor memory is freed.
-        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain[0]));
-        __syncwarp();
-        mbar_wait_warp(smem_addr(&ctrl->drain[0]), 0u, nullptr);
-    }
-
-    if (warp == C::WARP_PV) {
-        // ------------------------------------------------------------ value products
-        // Global step g: O += P_hi V(g) + P_lo V(g), A read from tensor memory
-        // (the P that replaced S(g)), once the softmax warps have written P(g);
-        // a unit's first step overwrites its O buffer after the epilogue has
-        // read that buffer's previous unit.
-        int64_t g = 0;
-        int uc = 0;
-        bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
-            PfUnit x;
-            uint32_t fl;
-            if (!pf_unit(a, u, x, &fl)) continue;
-            const int ob = uc & 1;
-            for (int j = 0; j < x.steps; ++j, ++g) {
-                const int64_t vi = 2 * g + 1;
-                const int e = static_cast<int>(vi % C::NS);
-                if (!mbar_wait_warp(smem_addr(&ctrl->pfull), static_cast<uint32_t>(g) & 1u, abort_flag) ||
-                    (j == 0 && !mbar_wait_warp(smem_addr(&ctrl->ofree[ob]),
-                                               (static_cast<uint32_t>(uc >> 1) & 1u) ^ 1u, abort_flag)) ||
-                    !mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(vi / C::NS) & 1u, abort_flag)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                if (tc::elect_one()) {
-                    const uint32_t vt = ring + e * C::TILE;
-                    const int sb = static_cast<int>(g & 1);
-#pragma unroll
-                    for (int part = 0; part < 2; ++part)
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            // 16 keys = 8 packed columns of P; 16 value rows
-                            const uint32_t pa = tmem + C::S_COL + sb * C::BN + part * 64 + 8 * k;
-                            const uint64_t db = tc::smem_desc(vt + k * 2048, C::PANEL, 1024, tc::kLayoutSw128);
-                            tc::mma_f16_ts(tmem + C::O_COL + ob * C::D, pa, db, IDESC_PV,
-                                           !(j == 0 && part == 0 && k == 0));
-                        }
-                    tc::commit(smem_addr(&ctrl->empty[e]));
-                    tc::commit(smem_addr(&ctrl->sfree[sb]));
-                    tc::commit(smem_addr(&ctrl->pvdone));
-                    if (j == x.steps - 1) tc::commit(smem_addr(&ctrl->ofull[ob]));
-                }
-                __syncwarp();
-            }
-            ++uc;
-        }
-        if (!ok) fail();
-        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain[1]));
-        __syncwarp();
-        mbar_wait_warp(smem_addr(&ctrl->drain[1]), 0u, nullptr);
-    }
-
-    if (warp >= C::WARP_SM0) {
-        // ------------------------------------------------------------ softmax + epilogue
-        // Two warps per tensor-memory sub-partition: warp half hf takes keys
-        // 64 hf .. 64 hf + 63 of every step (and d columns 64 hf .. of O).  The
-        // halves of a row share one reference, agreed each step from their
-        // partial maxima.
-        const int sp = warp & 3;                    // sub-partition of this warp
-        const int hf = (warp - C::WARP_SM0) >> 2;   // key half
-        const int r = 32 * sp + lane;               // tile row held by this thread (= TMEM lane)
-        const float NEG_INF = -__int_as_float(0x7f800000);
-        const uint64_t neg1 = pf_pack(-1.f, -1.f);
-        const uint64_t sl2x2 = pf_pack(a.sl2, a.sl2);
-        uint32_t xpar = 0;
-        // Both halves post a per-row value and read the other's; bounded waits.
-        // It also orders each half's tensor-memory reads of S before the other
-        // half's writes of P over the same columns.
-        auto exchange = [&](float mine, float& other) -> bool {
-            if (!mbar_wait_warp(smem_addr(&ctrl->xfree[sp]), xpar ^ 1u, abort_flag)) return false;
-            ctrl->xval[hf][r] = mine;
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->xfull[sp]));
-            if (!mbar_wait_warp(smem_addr(&ctrl->xfull[sp]), xpar, abort_flag)) return false;
-            tc::fence_after_sync();
-            other = ctrl->xval[hf ^ 1][r];
-            __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->xfree[sp]));
-            xpar ^= 1u;
-            return true;
+        };
+        auto wait_p = [&](int t, int64_t gs) {
+            return mbar_wait_warp(smem_addr(&ctrl->pfull[t]), static_cast<uint32_t>(gs) & 1u, abort_flag);
+        };
+        auto wait_ofree = [&](int t, int uc) {
+            return mbar_wait_warp(smem_addr(&ctrl->ofree[t]), (static_cast<uint32_t>(uc) & 1u) ^ 1u, abort_flag);
         };
         int64_t g = 0;
         int uc = 0;
@@ -484,45 +408,140 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
             PfUnit x;
             uint32_t fl;
             if (!pf_unit(a, u, x, &fl)) continue;
-            const int ob = uc & 1;
-            const int tq = r / a.R;        // token of the row within the tile
-            const int hq = r - tq * a.R;   // query head of the row within the group
-            const bool row_ok = tq < x.n_tok;
-            const int pos = x.pos0 + tq;   // cache position of the row's token
-            float ref = NEG_INF, l = 0.f;  // l: this half's share of the row sum
-            for (int j = 0; j < x.steps; ++j, ++g) {
-                const int sb = static_cast<int>(g & 1);
-                if (!mbar_wait_warp(smem_addr(&ctrl->sfull[sb]), static_cast<uint32_t>(g >> 1) & 1u, abort_flag)) {
+            const int n = x.steps;
+            if (!mbar_wait_warp(smem_addr(&ctrl->qfull), static_cast<uint32_t>(uc) & 1u, abort_flag) ||
+                !loaded(2 * g)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            if (tc::elect_one()) {
+                issue_qk(0, stage(2 * g));
+                tc::commit(smem_addr(&ctrl->sfull[0]));
+                issue_qk(1, stage(2 * g));
+                tc::commit(smem_addr(&ctrl->sfull[1]));
+                tc::commit(smem_addr(&ctrl->empty[(2 * g) % C::NS]));
+                if (n == 1) tc::commit(smem_addr(&ctrl->qempty));
+            }
+            __syncwarp();
+            if (!loaded(2 * g + 1) || !wait_ofree(0, uc) || !wait_p(0, g)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            if (tc::elect_one()) {
+                issue_pv(0, stage(2 * g + 1), true);
+                if (n == 1) tc::commit(smem_addr(&ctrl->ofull[0]));
+            }
+            __syncwarp();
+            for (int i = 1; i < n; ++i) {
+                const int64_t gi = g + i;
+                if (!loaded(2 * gi)) {
                     ok = false;
                     break;
                 }
                 tc::fence_after_sync();
-                uint32_t sv[64];  // this half's raw scores, then its weights (fp32 bits)
+                if (tc::elect_one()) {
+                    issue_qk(0, stage(2 * gi));  // after the product that read P_0(gi - 1) from these columns
+                    tc::commit(smem_addr(&ctrl->sfull[0]));
+                }
+                __syncwarp();
+                if ((i == 1 && !wait_ofree(1, uc)) || !wait_p(1, gi - 1)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    issue_pv(1, stage(2 * gi - 1), i == 1);
+                    tc::commit(smem_addr(&ctrl->empty[(2 * gi - 1) % C::NS]));
+                    issue_qk(1, stage(2 * gi));
+                    tc::commit(smem_addr(&ctrl->sfull[1]));
+                    tc::commit(smem_addr(&ctrl->empty[(2 * gi) % C::NS]));
+                    if (i == n - 1) tc::commit(smem_addr(&ctrl->qempty));
+                }
+                __syncwarp();
+                if (!loaded(2 * gi + 1) || !wait_p(0, gi)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                if (tc::elect_one()) {
+                    issue_pv(0, stage(2 * gi + 1), false);
+                    if (i == n - 1) tc::commit(smem_addr(&ctrl->ofull[0]));
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            const int64_t last = g + n - 1;
+            if ((n == 1 && !wait_ofree(1, uc)) || !wait_p(1, last)) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            if (tc::elect_one()) {
+                issue_pv(1, stage(2 * last + 1), n == 1);
+                tc::commit(smem_addr(&ctrl->empty[(2 * last + 1) % C::NS]));
+                tc::commit(smem_addr(&ctrl->ofull[1]));
+            }
+            __syncwarp();
+            g += n;
+            ++uc;
+        }
+        if (!ok) fail();
+        // Every product this warp issued has completed before tensor memory is freed.
+        if (tc::elect_one()) tc::commit(smem_addr(&ctrl->drain));
+        __syncwarp();
+        mbar_wait_warp(smem_addr(&ctrl->drain), 0u, nullptr);
+    }
+    } else {
+        reg_alloc<C::REG_HIGH>();
+        // ------------------------------------------------------------ softmax + epilogue
+        const int t = (warp - C::WARP_SM0) >> 2;   // query tile of this warp
+        const int sp = warp & 3;                   // sub-partition of this warp
+        const int r = 32 * sp + lane;              // tile row held by this thread (= TMEM lane)
+        const uint32_t trow = tc::tmem_addr(tmem, 32 * sp, 0);
+        const uint32_t s_col = C::S_COL + 128 * t, o_col = C::O_COL + 128 * t;
+        const float NEG_INF = -__int_as_float(0x7f800000);
+        const uint64_t neg1 = pf_pack(-1.f, -1.f);
+        const uint64_t sl2x2 = pf_pack(a.sl2, a.sl2);
+        int64_t g = 0;
+        int uc = 0;
+        bool ok = true;
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+            PfUnit x;
+            uint32_t fl;
+            if (!pf_unit(a, u, x, &fl)) continue;
+            const int n_t = min(max(x.n_tok - t * a.TQ, 0), a.TQ);  // tokens of this tile
+            const int tq = r / a.R;        // token of the row within the tile
+            const int hq = r - tq * a.R;   // query head of the row within the group
+            const bool row_ok = tq < n_t;
+            const int pos = x.pos0 + t * a.TQ + tq;  // cache position of the row's token
+            float ref = NEG_INF, l = 0.f;
+            for (int j = 0; j < x.steps; ++j, ++g) {
+                if (!mbar_wait_warp(smem_addr(&ctrl->sfull[t]), static_cast<uint32_t>(g) & 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                uint32_t sv[128];  // the row's raw scores, then its weights (fp32 bits)
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::S_COL + sb * C::BN + 64 * hf + 32 * c), sv + 32 * c);
+                for (int c = 0; c < 4; ++c) tc::tmem_ld32(trow + s_col + 32 * c, sv + 32 * c);
                 tc::tmem_wait_ld();
 
-                // Key 128 j + 64 hf + c is visible iff it is <= pos.
-                const int lim = row_ok ? pos - C::BN * j - 64 * hf : -1;
-                if (lim < 63) {
+                // Key 128 j + c is visible iff it is <= pos.
+                const int lim = row_ok ? pos - C::BN * j : -1;
+                if (lim < 127) {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
+                    for (int c = 0; c < 128; ++c)
                         if (c > lim) sv[c] = __float_as_uint(NEG_INF);
                 }
                 float m4[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-                for (int c = 0; c < 64; c += 2)
+                for (int c = 0; c < 128; c += 2)
                     m4[(c >> 1) & 3] = pf_max3(m4[(c >> 1) & 3], __uint_as_float(sv[c]), __uint_as_float(sv[c + 1]));
-                float mo;
-                const float mp = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
-                if (!exchange(mp, mo)) {
-                    ok = false;
-                    break;
-                }
                 // Base-2 row maximum (scale > 0 keeps the order); lazy reference:
                 // weights stay <= 2^8 against it.
-                const float mx = fmaxf(mp, mo) * a.sl2;
+                const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * a.sl2;
                 float alpha = 1.f;
                 const bool move = mx > ref + static_cast<float>(C::T_LAZY);
                 if (move) {
@@ -532,44 +551,49 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                 }
                 const float rb = ref == NEG_INF ? 0.f : ref;
                 const uint64_t nrb = pf_pack(-rb, -rb);
-                uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+                // Weights and P = hi + lo (bf16 pairs) over S_t's own columns, 32 keys
+                // at a time, so a chunk's scores die as its P is stored.
+                uint64_t acc[2] = {0ull, 0ull};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float2 t = pf_unpack(
-                        pf_fma2(pf_pack(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1])), sl2x2, nrb));
-                    const float p0 = fast_exp2(t.x), p1 = fast_exp2(t.y);
-                    sv[2 * i] = __float_as_uint(p0);
-                    sv[2 * i + 1] = __float_as_uint(p1);
-                    acc[i & 3] = pf_add2(acc[i & 3], pf_pack(p0, p1));
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t hi[16], lo[16];
+#pragma unroll
+                    for (int w = 0; w < 16; ++w) {
+                        const int k = 32 * c + 2 * w;
+                        const float2 e2 =
+                            pf_unpack(pf_fma2(pf_pack(__uint_as_float(sv[k]), __uint_as_float(sv[k + 1])), sl2x2, nrb));
+                        const float p0 = fast_exp2(e2.x), p1 = fast_exp2(e2.y);
+                        acc[w & 1] = pf_add2(acc[w & 1], pf_pack(p0, p1));
+                        pf_split(p0, p1, neg1, hi[w], lo[w]);
+                    }
+                    tc::tmem_st16(trow + s_col + 32 * c, hi);
+                    tc::tmem_st16(trow + s_col + 32 * c + 16, lo);
                 }
                 {
-                    const float2 s2 = pf_unpack(pf_add2(pf_add2(acc[0], acc[1]), pf_add2(acc[2], acc[3])));
+                    const float2 s2 = pf_unpack(pf_add2(acc[0], acc[1]));
                     l += s2.x + s2.y;
                 }
+                tc::tmem_wait_st();
 
                 if (j > 0 && __any_sync(0xffffffffu, move)) {
-                    // O holds this unit's earlier steps: once the previous step's value
-                    // product is done, rescale the moved rows in place (this half's d
-                    // columns).
-                    if (!mbar_wait_warp(smem_addr(&ctrl->pvdone), static_cast<uint32_t>(g - 1) & 1u, abort_flag)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
+                    // O_t holds this unit's earlier steps; the previous step's value
+                    // product has completed (S_t of this step was committed after it):
+                    // rescale the moved rows in place.
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
+                    for (int c = 0; c < 4; ++c) {
                         uint32_t o[32];
-                        const uint32_t oa = tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 64 * hf + 32 * c);
-                        tc::tmem_ld32(oa, o);
+                        tc::tmem_ld32(trow + o_col + 32 * c, o);
                         tc::tmem_wait_ld();
 #pragma unroll
                         for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-                        tc::tmem_st32(oa, o);
+                        tc::tmem_st32(trow + o_col + 32 * c, o);
                     }
                     tc::tmem_wait_st();
                 }
                 // Value rows at or past L_b may hold anything, and 0 * NaN would poison O.
-                if (C::BN * (j + 1) > x.L) {
+                // Tile 0's warps clear them (before P_0 of the step, which both value
+                // products of the step follow).
+                if (t == 0 && C::BN * (j + 1) > x.L) {
                     const int64_t vi = 2 * g + 1;
                     const int e = static_cast<int>(vi % C::NS);
                     if (!mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(vi / C::NS) & 1u,
@@ -578,47 +602,33 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                         break;
                     }
                     if (C::BN * j + r >= x.L) {
-                        const uint32_t vrow = ring + e * C::TILE + hf * C::PANEL + r * 128;
+                        const uint32_t vrow = ring + e * C::TILE + r * 128;
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) st_shared_v4(vrow + ((c ^ (r & 7)) << 4), 0u, 0u, 0u, 0u);
+                        for (int pnl = 0; pnl < 2; ++pnl)
+#pragma unroll
+                            for (int c = 0; c < 8; ++c) st_shared_v4(vrow + pnl * C::PANEL + 16 * c, 0u, 0u, 0u, 0u);
                     }
                     pf_fence_async_smem();
                 }
-                // P = hi + lo (bf16 pairs) over S's own columns: hi of keys
-                // 64 hf .. at columns 32 hf .., lo at 64 + 32 hf .. (both halves have
-                // read their scores: the exchange above orders it).
-                {
-                    uint32_t hi[32], lo[32];
-#pragma unroll
-                    for (int w = 0; w < 32; ++w)
-                        pf_split(__uint_as_float(sv[2 * w]), __uint_as_float(sv[2 * w + 1]), neg1, hi[w], lo[w]);
-                    const uint32_t pcol = C::S_COL + sb * C::BN + 32 * hf;
-                    tc::tmem_st32(tc::tmem_addr(tmem, 32 * sp, pcol), hi);
-                    tc::tmem_st32(tc::tmem_addr(tmem, 32 * sp, pcol + 64), lo);
-                    tc::tmem_wait_st();
-                }
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull));
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->pfull[t]));
             }
             if (!ok) break;
 
-            // ---------------------------------------------------- unit end: O / l -> out
-            float lo_half;
-            if (!exchange(l, lo_half) ||
-                !mbar_wait_warp(smem_addr(&ctrl->ofull[ob]), static_cast<uint32_t>(uc >> 1) & 1u, abort_flag)) {
+            // ---------------------------------------------------- unit end: O_t / l -> out
+            if (!mbar_wait_warp(smem_addr(&ctrl->ofull[t]), static_cast<uint32_t>(uc) & 1u, abort_flag)) {
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            const float lt = l + lo_half;
-            const float inv = lt > 0.f ? 1.f / lt : 0.f;
+            const float inv = l > 0.f ? 1.f / l : 0.f;
             const int64_t orow =
-                row_ok ? (static_cast<int64_t>(x.q_row0 + tq) * a.H_Q + x.kv * a.R + hq) * C::D + 64 * hf : 0;
+                row_ok ? (static_cast<int64_t>(x.q_row0 + t * a.TQ + tq) * a.H_Q + x.kv * a.R + hq) * C::D : 0;
 #pragma unroll
-            for (int c = 0; c < 2; ++c) {
+            for (int c = 0; c < 4; ++c) {
                 uint32_t o[32];
-                tc::tmem_ld32(tc::tmem_addr(tmem, 32 * sp, C::O_COL + ob * C::D + 64 * hf + 32 * c), o);
+                tc::tmem_ld32(trow + o_col + 32 * c, o);
                 tc::tmem_wait_ld();
                 if (row_ok) {
                     if constexpr (OUT_BF16) {
@@ -646,7 +656,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
             }
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree[ob]));
+            if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree[t]));
             ++uc;
         }
         if (!ok) fail();
@@ -655,7 +665,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
     // ---------------------------------------------------------------- teardown
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == C::WARP_QK) {
+    if (warp == C::WARP_MMA) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, C::TMEM_COLS);
     }

@@ -7,6 +7,18 @@ N > H_KV the KV heads are duplicated and each rank runs MQA on one of them.
 Here the N shards run one after another as independent calls on one GPU (no
 shard waits on another) and their outputs, concatenated along the head axis,
 must match the oracle and the unsharded call.
+
+Multi-token step: the concatenated shards equal the unsharded call bit for
+bit.  Its kernel has no split-KV: a query row's scores, weights and value
+sums run over the same 128-key steps in the same order whatever other rows
+share its tile, so neither the head count of a shard nor the tile shape
+changes a single bit.
+
+Decode step: the shards agree with the unsharded call within 1e-4, not bit for
+bit.  The decode schedule cuts the whole batch's tiles into equal shares per
+CTA, so where a unit's split-KV boundaries fall (and with them the rounding of
+its partial sums and their merge) depends on the total tile count, which a
+shard changes.  Both sides are independently within the oracle tolerance.
 """
 
 import dataclasses
@@ -38,7 +50,7 @@ def test_tp_shards_reassemble_the_full_step(cuda_device, world, h_q, h_kv):
     got = torch.cat(parts, dim=1).cpu()
     assert_parity(got, oracle_full(inp, w), f"TP {world} over {h_q}/{h_kv}")
     full = run_gpu(inp, w, cuda_device)
-    assert (got - full).abs().max().item() < 1e-4
+    assert (got - full).abs().max().item() < 1e-4  # split boundaries differ (module docstring)
 
 
 @pytest.mark.parametrize("world,h_q,h_kv", [(2, 64, 8), (8, 32, 4), (4, 32, 2)])
@@ -63,4 +75,4 @@ def test_tp_prefill_shards_reassemble_the_full_step(cuda_device, world, h_q, h_k
     ref = oracle.gqa_prefill(inp["q"], inp["k"], inp["v"], inp["seq_lens"], inp["cu_q"], w.softmax_scale)
     assert_parity(got, ref, f"TP prefill {world} over {h_q}/{h_kv}")
     full = gq.gqa_prefill(d["q"], d["k"], d["v"], d["seq_lens"], d["cu_q"], max_q_len=d["max_q"]).cpu()
-    assert (got - full).abs().max().item() < 1e-4
+    assert torch.equal(got.view(torch.int32), full.view(torch.int32)), "prefill shards differ from the whole call"
