@@ -25,7 +25,7 @@ __all__ = [
     "GqaError", "Params", "gqa_decode", "gqa_decode_timed", "gqa_decode_static_workspace",
     "gqa_rope_append", "gqa_decode_fp8kv", "gqa_prefill", "FLAG_BAD_POSITION", "FLAG_BAD_QUERY_SPAN",
     "workspace_bytes", "make_workspace",
-    "read_status", "kv_cache_bytes", "library", "LIB_PATH", "FLAG_SEQ_LEN_CLAMPED",
+    "read_status", "static_workspace_status", "kv_cache_bytes", "library", "LIB_PATH", "FLAG_SEQ_LEN_CLAMPED",
     "FLAG_BAD_BLOCK", "FLAG_TIMEOUT", "PAGE_SIZE",
 ]
 
@@ -41,7 +41,7 @@ EXPORTED = (
     "gqa_decode_workspace_size", "gqa_decode", "gqa_decode_timed", "gqa_read_status",
     "gqa_kv_cache_bytes", "gqa_status_string", "gqa_version", "gqa_decode_static_workspace",
     "gqa_rope_append", "gqa_decode_fp8kv", "gqa_wait_selftest", "gqa_prefill_workspace_size",
-    "gqa_prefill",
+    "gqa_prefill", "gqa_static_workspace_status",
 )
 
 
@@ -100,6 +100,8 @@ def library() -> ctypes.CDLL:
             lib.gqa_decode_static_workspace.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_float, vp,
                                                         vp]
             lib.gqa_decode_static_workspace.restype = ctypes.c_int
+            lib.gqa_static_workspace_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32), ctypes.c_int]
+            lib.gqa_static_workspace_status.restype = ctypes.c_int
             lib.gqa_rope_append.argtypes = [pp, vp, vp, vp, vp, vp, ctypes.c_double, ctypes.c_int, vp,
                                             vp, vp, vp, vp, vp]
             lib.gqa_rope_append.restype = ctypes.c_int
@@ -485,6 +487,24 @@ def read_status(workspace, stream=None, clear=False) -> int:
                                    int(bool(clear)))
     if st != 0:
         raise GqaError(st, "gqa_read_status")
+    return int(flags.value)
+
+
+def static_workspace_status(stream=None, clear=False, device=None) -> int:
+    """GQA_FLAG_* bits accumulated in the built-in workspace that
+    gqa_decode_static_workspace uses on the current device (synchronises the
+    stream); ``clear`` resets them."""
+    import torch
+
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    flags = ctypes.c_uint32(0)
+    with torch.cuda.device(device):
+        st = library().gqa_static_workspace_status(ctypes.c_void_p(stream.cuda_stream), ctypes.byref(flags),
+                                                   int(bool(clear)))
+    if st != 0:
+        raise GqaError(st, "gqa_static_workspace_status")
     return int(flags.value)
 
 

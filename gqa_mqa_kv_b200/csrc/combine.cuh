@@ -1,19 +1,22 @@
-// combine.cuh -- log-sum-exp merge of split-KV partials.
+// combine.cuh -- log-sum-exp merge of split-KV partials, done inside the
+// split kernels by the last writer of a split unit.
 //
 // A unit (sequence b, KV head kv) that the tile schedule cut across CTAs
-// c_a..c_b has one partial per CTA: o_j (already divided by its own softmax
+// ca..cb has one partial per CTA: o_j (already divided by its own softmax
 // denominator) and lse_j = m_j + log2 l_j in base-2 score units.  The merged
 // result is out = sum_j 2^(lse_j - M) o_j / sum_j 2^(lse_j - M) with
 // M = max_j lse_j, the split form of the softmax in "Grouped-Query Attention
 // (GQA) and Multi-Query Attention (MQA): Mathematical Foundations, ...",
-// section 2 (Head_i).  Units whose tiles stayed in one CTA were finished by
-// the split kernel; sequences with L_b = 0 get out = 0 here.
+// section 2 (Head_i).
 //
-// Each CTA owns up to kCombineSpan (head, d) outputs of one unit, every
-// thread kCombineEPT of them; the partials' log-sum-exps are staged in shared
-// memory kCombineChunk at a time and folded in with a running maximum, so any
-// number of partials works and every partial load of a chunk is independent
-// of the others.
+// The warps that write a CTA's partial only arrive on a CTA-local mbarrier
+// (release at CTA scope).  A dedicated merge warp of the CTA waits on it,
+// publishes the partial at GPU scope (a fence, cumulative over the writes it
+// has observed, then a ticket from the unit's counter) and, holding the last
+// ticket, merges the unit.  The streaming warps therefore never wait on a
+// GPU-scope fence or an atomic round trip.  The sums run over j = 0 ..
+// n_parts-1 in that order from the stored values, so the result does not
+// depend on which CTA merges.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -23,11 +26,6 @@
 
 namespace gqa {
 
-constexpr int kCombineThreads = 256;
-constexpr int kCombineEPT = 4;                                    // outputs per thread
-constexpr int kCombineSpan = kCombineThreads * kCombineEPT;      // outputs per CTA
-constexpr int kCombineChunk = 8;                                  // partials staged per pass
-
 template <bool OUT_BF16>
 __device__ __forceinline__ void store_out(void* out, int64_t i, float x) {
     if constexpr (OUT_BF16)
@@ -36,117 +34,168 @@ __device__ __forceinline__ void store_out(void* out, int64_t i, float x) {
         static_cast<float*>(out)[i] = x;
 }
 
-// Grid: (B * H_KV) units x ceil(R * D / kCombineSpan) parts; part z of a unit
-// owns its outputs [z * kCombineSpan, (z + 1) * kCombineSpan) in (head, d) order.
+// Warp-collective: publishes the partial this CTA's writers have finished
+// (observed through a CTA-scope barrier) and takes a ticket from *cnt; true in
+// every lane for the last of `expected` tickets (loads of the other partials
+// are ordered after that observation).
+__device__ __forceinline__ bool merge_ticket(uint32_t* cnt, int expected) {
+    __threadfence();
+    uint32_t old = 0;
+    if ((threadIdx.x & 31) == 0) old = atomicAdd(cnt, 1u);
+    old = __shfl_sync(0xffffffffu, old, 0);
+    const bool last = old == static_cast<uint32_t>(expected - 1);
+    if (last) __threadfence();
+    return last;
+}
+
+// Warp-collective merge of a split unit's R x D outputs (written at
+// out[row0 + h D + d]) from its partials, which other SMs wrote during this
+// grid and are therefore read at L2 (ld.global.cg).  Element e = lane + 32 k
+// is head e / (D/4), dimensions 4 (e % (D/4)) .. +3.  A block of KG elements
+// x JG partials issues all of its loads before using any, so it costs one L2
+// round trip; partials are folded in with a running maximum, so any number
+// of them works.
 template <int D, bool OUT_BF16>
-__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const KernelArgs a, int grid) {
-    constexpr int HPC = kCombineSpan / D;  // heads per part
-    __shared__ float s_lse[kCombineChunk][HPC];
-    __shared__ int64_t red_total[kCombineThreads / 32], red_before[kCombineThreads / 32];
-
-    grid_launch_dependents();
-    const int parts = (a.R * D + kCombineSpan - 1) / kCombineSpan;
-    const int unit = blockIdx.x / parts;
-    const int part = blockIdx.x % parts;
-    const int b = unit / a.H_KV;
-    const int kv = unit % a.H_KV;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int R = a.R;
-    const int r0 = part * HPC;                       // first head of this part
-    const int nr = min(HPC, R - r0);                 // heads in this part
-
-    // seq_lens were final before the split kernel read them, so the tile
-    // arithmetic may run while the split grid is still finishing.
-    int64_t total = 0, before = 0;
-    for (int i = threadIdx.x; i < a.B; i += blockDim.x) {
-        const int64_t c = static_cast<int64_t>(a.H_KV) * tiles_of(seq_len_at(a, i));
-        total += c;
-        if (i < b) before += c;
-    }
-    total = warp_sum_i64(total);
-    before = warp_sum_i64(before);
-    if (lane == 0) {
-        red_total[warp] = total;
-        red_before[warp] = before;
-    }
-    __syncthreads();
-    total = before = 0;
-#pragma unroll
-    for (int i = 0; i < kCombineThreads / 32; ++i) {
-        total += red_total[i];
-        before += red_before[i];
-    }
-    const int n_b = tiles_of(seq_len_at(a, b));
-    const int64_t out_base = (static_cast<int64_t>(b) * a.H_Q + static_cast<int64_t>(kv) * R + r0) * D;
-
-    if (n_b == 0) {
-        grid_dependency_wait();
-        for (int idx = threadIdx.x; idx < nr * D; idx += blockDim.x) store_out<OUT_BF16>(a.out, out_base + idx, 0.f);
-        return;
-    }
-    const int g = effective_grid(total, grid);
-    const int64_t s_u = before + static_cast<int64_t>(kv) * n_b;
-    const int64_t ca = owner_of_tile(s_u, total, g);
-    const int64_t cb = owner_of_tile(s_u + n_b - 1, total, g);
-    if (ca == cb) return;  // finished by the split kernel
-    const int n_parts = static_cast<int>(cb - ca + 1);
-    const int64_t slot0 = cta_first_tile(ca, total, g) < s_u ? 2 * ca + 1 : 2 * ca;
-
-    grid_dependency_wait();  // partials of the split grid are complete and visible from here
-
+__device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, const int64_t row0) {
+    constexpr int KG = 4, JG = 4, Q = D / 4;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    float m[kCombineEPT], sum[kCombineEPT], acc[kCombineEPT];
+    const int lane = threadIdx.x & 31;
+    const int E = a.R * Q;
+    for (int e0 = 0; e0 < E; e0 += 32 * KG) {
+        float m[KG], l[KG];
+        float4 acc[KG];
 #pragma unroll
-    for (int e = 0; e < kCombineEPT; ++e) {
-        m[e] = NEG_INF;
-        sum[e] = 0.f;
-        acc[e] = 0.f;
-    }
-    for (int j0 = 0; j0 < n_parts; j0 += kCombineChunk) {
-        const int nj = min(kCombineChunk, n_parts - j0);
-        __syncthreads();  // previous chunk's s_lse fully consumed
-        for (int i = threadIdx.x; i < nj * nr; i += blockDim.x) {
-            const int jj = i / nr, rr = i % nr;
-            const int j = j0 + jj;
-            const int64_t slot = j == 0 ? slot0 : 2 * (ca + j);
-            s_lse[jj][rr] = a.ws_lse[slot * R + r0 + rr];
+        for (int kk = 0; kk < KG; ++kk) {
+            m[kk] = NEG_INF;
+            l[kk] = 0.f;
+            acc[kk] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        __syncthreads();
+        for (int j0 = 0; j0 < u.n_parts; j0 += JG) {
+            float ls[KG][JG];
+            float4 ov[KG][JG];
 #pragma unroll
-        for (int e = 0; e < kCombineEPT; ++e) {
-            const int idx = e * kCombineThreads + threadIdx.x;
-            if (idx >= nr * D) break;
-            const int rr = idx / D, d = idx % D;
-            float ov[kCombineChunk];
+            for (int kk = 0; kk < KG; ++kk) {
+                const int e = e0 + 32 * kk + lane;
+                const int h = e / Q, q4 = e - h * Q;
 #pragma unroll
-            for (int jj = 0; jj < kCombineChunk; ++jj) {
-                const int j = j0 + jj;
-                const int64_t slot = j == 0 ? slot0 : 2 * (ca + j);
-                ov[jj] = jj < nj ? a.ws_o[(slot * R + r0 + rr) * D + d] : 0.f;
-            }
-            float mx = m[e];
-#pragma unroll
-            for (int jj = 0; jj < kCombineChunk; ++jj)
-                if (jj < nj) mx = fmaxf(mx, s_lse[jj][rr]);
-            const float rescale = fast_exp2(m[e] - mx);  // m = -inf on the first chunk -> 0
-            sum[e] *= rescale;
-            acc[e] *= rescale;
-#pragma unroll
-            for (int jj = 0; jj < kCombineChunk; ++jj) {
-                if (jj < nj) {
-                    const float wj = fast_exp2(s_lse[jj][rr] - mx);
-                    sum[e] += wj;
-                    acc[e] = fmaf(wj, ov[jj], acc[e]);
+                for (int jj = 0; jj < JG; ++jj) {
+                    ls[kk][jj] = NEG_INF;
+                    ov[kk][jj] = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (e < E && j0 + jj < u.n_parts) {
+                        const int64_t sl = part_slot(u, j0 + jj);
+                        ls[kk][jj] = __ldcg(a.ws_lse + sl * a.R + h);
+                        ov[kk][jj] = __ldcg(reinterpret_cast<const float4*>(a.ws_o + (sl * a.R + h) * D) + q4);
+                    }
                 }
             }
-            m[e] = mx;
+#pragma unroll
+            for (int kk = 0; kk < KG; ++kk) {
+                float mx = m[kk];
+#pragma unroll
+                for (int jj = 0; jj < JG; ++jj) mx = fmaxf(mx, ls[kk][jj]);
+                if (mx == NEG_INF) continue;  // an element past the unit's outputs
+                const float sc = fast_exp2(m[kk] - mx);  // m = -inf on the first block -> 0
+                l[kk] *= sc;
+                acc[kk].x *= sc;
+                acc[kk].y *= sc;
+                acc[kk].z *= sc;
+                acc[kk].w *= sc;
+#pragma unroll
+                for (int jj = 0; jj < JG; ++jj) {
+                    const float wj = fast_exp2(ls[kk][jj] - mx);  // 2^-inf = 0 for missing partials
+                    l[kk] += wj;
+                    acc[kk].x = fmaf(wj, ov[kk][jj].x, acc[kk].x);
+                    acc[kk].y = fmaf(wj, ov[kk][jj].y, acc[kk].y);
+                    acc[kk].z = fmaf(wj, ov[kk][jj].z, acc[kk].z);
+                    acc[kk].w = fmaf(wj, ov[kk][jj].w, acc[kk].w);
+                }
+                m[kk] = mx;
+            }
+        }
+#pragma unroll
+        for (int kk = 0; kk < KG; ++kk) {
+            const int e = e0 + 32 * kk + lane;
+            if (e >= E) continue;
+            const int h = e / Q, q4 = e - h * Q;
+            const float inv = 1.f / l[kk];
+            const int64_t i = row0 + static_cast<int64_t>(h) * D + 4 * q4;
+            // 8-byte stores: out is only required to be 8-byte aligned
+            if constexpr (OUT_BF16) {
+                const __nv_bfloat162 p0 = __floats2bfloat162_rn(acc[kk].x * inv, acc[kk].y * inv);
+                const __nv_bfloat162 p1 = __floats2bfloat162_rn(acc[kk].z * inv, acc[kk].w * inv);
+                *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + i) =
+                    make_uint2(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1));
+            } else {
+                float2* dst = reinterpret_cast<float2*>(static_cast<float*>(a.out) + i);
+                dst[0] = make_float2(acc[kk].x * inv, acc[kk].y * inv);
+                dst[1] = make_float2(acc[kk].z * inv, acc[kk].w * inv);
+            }
         }
     }
-#pragma unroll
-    for (int e = 0; e < kCombineEPT; ++e) {
-        const int idx = e * kCombineThreads + threadIdx.x;
-        if (idx < nr * D) store_out<OUT_BF16>(a.out, out_base + idx, acc[e] / sum[e]);
+}
+
+// A CTA's merge jobs: its first and its last segment, each when it is cut
+// (holds a partial).  Job k is signalled on mjob[k] by the segment's writers.
+struct MergeJobs {
+    int n;
+    int slot[2];      // which of mjob[0] (first segment) / mjob[1] (last) it waits on
+    SplitUnit su[2];
+    int b[2], kv[2];
+};
+
+// Warp-collective: the jobs of this CTA's tile range [lo, hi) (lo < hi).
+__device__ __forceinline__ MergeJobs merge_jobs_of(const KernelArgs& a, const Plan& p) {
+    MergeJobs J;
+    J.n = 0;
+    // the unit holding tile lo
+    const int64_t s0 = p.lo - p.tile;
+    const bool first_cut = p.tile > 0 || s0 + p.n_b > p.hi;
+    if (first_cut) {
+        J.slot[J.n] = 0;
+        J.su[J.n] = split_unit_of(s0, p.n_b, p.n_tiles, p.g);
+        J.b[J.n] = p.b;
+        J.kv[J.n] = p.kv;
+        ++J.n;
     }
+    if (s0 + p.n_b < p.hi) {
+        // another unit holds tile hi - 1: the CTA's last segment
+        int b = 0;
+        int64_t start = 0;
+        warp_find_batch(a, p.hi - 1, &b, &start);
+        const int n_b = tiles_of(seq_len_at(a, b));
+        const int kv = static_cast<int>((p.hi - 1 - start) / n_b);
+        const int64_t su = start + static_cast<int64_t>(kv) * n_b;
+        if (su + n_b > p.hi) {
+            J.slot[J.n] = 1;
+            J.su[J.n] = split_unit_of(su, n_b, p.n_tiles, p.g);
+            J.b[J.n] = b;
+            J.kv[J.n] = kv;
+            ++J.n;
+        }
+    }
+    return J;
+}
+
+// The merge warp of a split kernel (warp-collective).  Takes the call's merge
+// epoch, clears its share of the next call's counters, writes the outputs of
+// empty sequences, then serves the CTA's merge jobs in order.  Returns false
+// when a wait for the writers gave up (the caller raises the timeout flag).
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, uint64_t* mjob, const volatile int* abort) {
+    const int lane = threadIdx.x & 31;
+    uint32_t epoch = 0;
+    if (lane == 0) epoch = merge_epoch_take(a);
+    epoch = __shfl_sync(0xffffffffu, epoch, 0);
+    uint32_t* bank = merge_bank(a, epoch, static_cast<int>(threadIdx.x) - lane, 32);
+    zero_empty_sequences<D, OUT_BF16>(a, static_cast<int>(threadIdx.x) - lane, 32);
+    if (p.lo >= p.hi) return true;
+    const MergeJobs J = merge_jobs_of(a, p);
+    for (int k = 0; k < J.n; ++k) {
+        if (!mbar_wait_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort)) return false;
+        if (merge_ticket(bank + J.su[k].ca, J.su[k].n_parts))
+            merge_unit<D, OUT_BF16>(a, J.su[k], (static_cast<int64_t>(J.b[k]) * a.H_Q + J.kv[k] * a.R) * D);
+    }
+    return true;
 }
 
 }  // namespace gqa

@@ -2,9 +2,9 @@
 //
 // Validates arguments, picks the kernel (tensor-core split kernel for bf16
 // with groups of up to 64 query heads, CUDA-core split kernel otherwise),
-// encodes the TMA tensor maps, and enqueues split + combine on the caller's
-// stream with programmatic dependent launch so the combine grid's launch
-// overlaps the split grid's tail.  No allocation, no host synchronisation.
+// encodes the TMA tensor maps, and enqueues the split kernel -- which also
+// merges the partials of units it cut across CTAs -- on the caller's stream
+// with programmatic dependent launch.  No allocation, no host synchronisation.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -27,7 +27,7 @@ namespace {
 
 using namespace gqa;
 
-constexpr size_t kHeaderBytes = 256;  // status word lives at offset 0
+constexpr size_t kHeaderBytes = 256;  // words 0..2: status flags, merge epoch, epoch readers
 constexpr int kSimtCtasPerSm = 4;
 constexpr int kMaxDevices = 64;
 
@@ -103,11 +103,17 @@ int grid_for(const gqa_decode_params* p, const DeviceInfo& dev, bool kv8 = false
     return select_kernel(p, kv8) == SplitKernel::kSimt && !kv8 ? dev.sms * kSimtCtasPerSm : dev.sms;
 }
 
+// Workspace layout: header (status word, merge epoch), two banks of merge
+// counters, then the partials ws_o [2G, R, D] and ws_lse [2G, R].
+size_t ws_o_bytes(const gqa_decode_params* p, int grid) {
+    const size_t R = static_cast<size_t>(p->H_Q / p->H_KV);
+    return round_up(2 * static_cast<size_t>(grid) * R * p->head_dim * sizeof(float), 256);
+}
+
 size_t workspace_for(const gqa_decode_params* p, int grid) {
     const size_t R = static_cast<size_t>(p->H_Q / p->H_KV);
     const size_t slots = 2 * static_cast<size_t>(grid);
-    return kHeaderBytes + round_up(slots * R * p->head_dim * sizeof(float), 256) +
-           round_up(slots * R * sizeof(float), 256);
+    return kHeaderBytes + kMergeCounterBytes + ws_o_bytes(p, grid) + round_up(slots * R * sizeof(float), 256);
 }
 
 // ------------------------------------------------------------------ TMA maps
@@ -352,9 +358,7 @@ cudaError_t launch_all(const gqa_decode_params* p, const Buffers& buf, const Ker
                      : launch_split<D, false, OUTB>(p, buf, args, dev, grid, stream, encode_ok);
     if (e != cudaSuccess) return e;
     if (ev1 && (e = cudaEventRecord(ev1, stream)) != cudaSuccess) return e;
-    const int parts = (args.R * D + kCombineSpan - 1) / kCombineSpan;
-    return launch_chained(combine_kernel<D, OUTB>, p->B * p->H_KV * parts, kCombineThreads, 0,
-                          stream, args, grid);
+    return cudaSuccess;
 }
 
 gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const void* v,
@@ -378,11 +382,11 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
     // 8-bit caches always use one CTA per SM, so gqa_decode_workspace_size's
     // answer for the same parameters is always enough.
     const int grid = kv8 ? dev.sms : grid_for(p, dev);
+    if (grid > kMergeCounters) return GQA_ERR_UNSUPPORTED;  // one merge counter per CTA
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < workspace_for(p, grid))
         return GQA_ERR_WORKSPACE;
 
     const int R = p->H_Q / p->H_KV;
-    const size_t slots = 2 * static_cast<size_t>(grid);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     KernelArgs args;
     std::memset(&args, 0, sizeof args);
@@ -399,9 +403,9 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
     args.sl2 = scale * 1.4426950408889634f;  // log2(e): exponentials are taken base 2
     args.out = out;
     args.status = reinterpret_cast<uint32_t*>(ws);
-    args.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes);
-    args.ws_lse = reinterpret_cast<float*>(
-        ws + kHeaderBytes + round_up(slots * R * p->head_dim * sizeof(float), 256));
+    args.merge = reinterpret_cast<uint32_t*>(ws + kHeaderBytes);
+    args.ws_o = reinterpret_cast<float*>(ws + kHeaderBytes + kMergeCounterBytes);
+    args.ws_lse = reinterpret_cast<float*>(ws + kHeaderBytes + kMergeCounterBytes + ws_o_bytes(p, grid));
     args.k_scale = k_scale;
     args.v_scale = v_scale;
 
@@ -429,10 +433,13 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
 // must never hand this name to a kernel: on the host it is only a stand-in,
 // and the device address comes from cudaGetSymbolAddress below.
 constexpr size_t kStaticWorkspaceBytes = size_t(8) << 20;  // 8 MiB
+static_assert(kStaticWorkspaceBytes == GQA_STATIC_WORKSPACE_BYTES,
+              "the built-in workspace and the header's stated limit must agree");
 static __device__ __align__(256) unsigned char g_static_workspace[kStaticWorkspaceBytes];
 
 // Device address of g_static_workspace on the current device, looked up once
-// per device with that device current; its status word is cleared then.
+// per device with that device current; its header and merge counters are
+// cleared then.
 gqa_status static_workspace_on_current_device(void** ptr, cudaStream_t stream) {
     static std::mutex mu;
     static void* addr[kMaxDevices] = {};
@@ -443,7 +450,8 @@ gqa_status static_workspace_on_current_device(void** ptr, cudaStream_t stream) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr)
             return GQA_ERR_CUDA;
-        if (cudaMemsetAsync(p, 0, kHeaderBytes, stream) != cudaSuccess) return GQA_ERR_CUDA;
+        // status word, merge epoch and merge counters start at zero
+        if (cudaMemsetAsync(p, 0, kHeaderBytes + kMergeCounterBytes, stream) != cudaSuccess) return GQA_ERR_CUDA;
         addr[dev] = p;
     }
     *ptr = addr[dev];
@@ -608,6 +616,14 @@ gqa_status gqa_decode_static_workspace(const gqa_decode_params* params, const vo
         return st;
     return run(params, q, k_cache, v_cache, seq_lens, block_table, scale, out, ws,
                kStaticWorkspaceBytes, stream, nullptr, nullptr);
+}
+
+gqa_status gqa_static_workspace_status(void* stream, uint32_t* flags, int clear) {
+    if (flags == nullptr) return GQA_ERR_INVALID;
+    void* ws = nullptr;
+    const gqa_status st = static_workspace_on_current_device(&ws, static_cast<cudaStream_t>(stream));
+    if (st != GQA_OK) return st;
+    return gqa_read_status(ws, stream, flags, clear);
 }
 
 gqa_status gqa_rope_append(const gqa_decode_params* params, const void* q, const void* k_new,

@@ -14,10 +14,15 @@
 // "segment" -- a (sequence, KV head, KV split) triple of the split-KV method.
 // A segment that covers its whole unit writes the final output; otherwise it
 // writes a partial (normalised o, log2-sum-exp) into one of two workspace
-// slots of its CTA: 2c for the CTA's first segment, 2c+1 for its last.  The
-// combine kernel finds the partials of a unit from the same arithmetic.
+// slots of its CTA: 2c for the CTA's first segment, 2c+1 for its last.  A
+// unit cut across CTAs c_a..c_b has one partial per CTA; c_a is unique to it
+// (only a CTA's last segment can continue past its range), so c_a indexes its
+// merge counter.  Each writer arrives on that counter after its partial is
+// visible, and the last of the unit's writers merges all partials (found from
+// the same arithmetic) into the output -- no separate combine launch.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <stdint.h>
 
 namespace gqa {
@@ -28,6 +33,15 @@ constexpr uint32_t kFlagBadBlock = 2u; // GQA_FLAG_BAD_BLOCK
 constexpr uint32_t kFlagTimeout = 4u;  // GQA_FLAG_TIMEOUT
 constexpr uint32_t kFlagBadPosition = 8u;  // GQA_FLAG_BAD_POSITION
 constexpr uint32_t kFlagBadSpan = 16u;     // GQA_FLAG_BAD_QUERY_SPAN
+
+// Merge counters: two banks of kMergeCounters words after the 256-byte
+// workspace header.  Header words: [0] status flags, [1] merge epoch, [2] CTAs
+// of the running call that have read the epoch.  A call counts arrivals in
+// bank (epoch & 1) and zeroes the other bank, which the next call (epoch + 1)
+// uses; so a call cut short (a timed-out wait) never leaves stale counts for
+// the call after it.
+constexpr int kMergeCounters = 2048;
+constexpr size_t kMergeCounterBytes = 2 * kMergeCounters * sizeof(uint32_t);
 
 struct KernelArgs {
     const int32_t* seq_lens;     // [B]
@@ -41,7 +55,8 @@ struct KernelArgs {
     void* out;       // [B, H_Q, D]
     float* ws_o;     // [2G, R, D] partial outputs (normalised)
     float* ws_lse;   // [2G, R] partial log2-sum-exp
-    uint32_t* status;
+    uint32_t* status;  // workspace header: status word, merge epoch, epoch readers
+    uint32_t* merge;   // [2][kMergeCounters] merge counters
     int n_stages;    // tensor-core path: pipeline depth
     int q_rows;      // tensor-core path: query rows per TMA box, min(R, 16)
     int q_groups;    // tensor-core path: 16-row head groups holding real rows
@@ -148,7 +163,22 @@ struct Walk {
 struct Plan {
     int64_t lo, hi;  // global tile range of this CTA
     int b, kv, tile, n_b, L;
+    int64_t n_tiles; // N_T
+    int g;           // working CTAs, min(gridDim, N_T)
 };
+
+// One thread per CTA (its merge warp), after the grid dependency wait: this
+// call's merge epoch.  The last CTA to take it advances it for the next call; every CTA
+// has read it by then (each reads before it counts itself).
+__device__ __forceinline__ uint32_t merge_epoch_take(const KernelArgs& a) {
+    const uint32_t e = *reinterpret_cast<volatile uint32_t*>(a.status + 1);
+    __threadfence();  // the read above is complete before this CTA is counted
+    if (atomicAdd(a.status + 2, 1u) == gridDim.x - 1) {
+        a.status[2] = 0u;  // plain stores: the next call reads them after this grid has completed
+        a.status[1] = e + 1u;
+    }
+    return e;
+}
 
 // Warp-collective; lane 0 writes *plan.  Also raises the clamp flag (CTA 0).
 __device__ __forceinline__ void make_plan(const KernelArgs& a, Plan* plan) {
@@ -168,6 +198,8 @@ __device__ __forceinline__ void make_plan(const KernelArgs& a, Plan* plan) {
     if (lane == 0) {
         plan->lo = lo;
         plan->hi = hi;
+        plan->n_tiles = n_tiles;
+        plan->g = g;
         plan->b = b;
         plan->kv = plan->tile = plan->n_b = plan->L = 0;
         if (lo < hi) {
@@ -178,6 +210,58 @@ __device__ __forceinline__ void make_plan(const KernelArgs& a, Plan* plan) {
             plan->n_b = n_b;
             plan->kv = static_cast<int>(local / n_b);
             plan->tile = static_cast<int>(local % n_b);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- split units
+
+// The unit whose first global tile is s_u and which has n_b tiles, as the
+// schedule cut it: CTAs ca..ca+n_parts-1 each hold one partial of it.
+struct SplitUnit {
+    int64_t ca;
+    int n_parts;
+    int64_t slot0;  // workspace slot of part 0 (ca's last segment)
+};
+
+__device__ __forceinline__ SplitUnit split_unit_of(int64_t s_u, int n_b, int64_t n_tiles, int64_t g) {
+    SplitUnit u;
+    u.ca = owner_of_tile(s_u, n_tiles, g);
+    u.n_parts = static_cast<int>(owner_of_tile(s_u + n_b - 1, n_tiles, g) - u.ca + 1);
+    u.slot0 = cta_first_tile(u.ca, n_tiles, g) < s_u ? 2 * u.ca + 1 : 2 * u.ca;
+    return u;
+}
+
+// Slot of part j: part 0 is ca's last segment, every later part its CTA's first.
+__device__ __forceinline__ int64_t part_slot(const SplitUnit& u, int j) {
+    return j == 0 ? u.slot0 : 2 * (u.ca + j);
+}
+
+// This call's counter bank; the CTA's share of the other bank is zeroed here
+// (by the threads [t0, t0 + nt) of the CTA) for the next call.
+__device__ __forceinline__ uint32_t* merge_bank(const KernelArgs& a, uint32_t epoch, int t0, int nt) {
+    uint32_t* other = a.merge + ((epoch + 1u) & 1u) * kMergeCounters;
+    for (int i = blockIdx.x * nt + (static_cast<int>(threadIdx.x) - t0); i < kMergeCounters; i += gridDim.x * nt)
+        other[i] = 0u;
+    return a.merge + (epoch & 1u) * kMergeCounters;
+}
+
+// Threads [t0, t0 + nt) of the CTA write out = 0 for every sequence with
+// L_b = 0 among b = blockIdx.x, blockIdx.x + gridDim.x, ... (an empty sum).
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ void zero_empty_sequences(const KernelArgs& a, int t0, int nt) {
+    const int t = static_cast<int>(threadIdx.x) - t0;
+    for (int b = blockIdx.x; b < a.B; b += gridDim.x) {
+        if (seq_len_at(a, b) != 0) continue;
+        const int64_t base = static_cast<int64_t>(b) * a.H_Q * D;
+        const int n = a.H_Q * D;
+        // 8-byte stores: out is only required to be 8-byte aligned
+        if constexpr (OUT_BF16) {
+            for (int i = t; i < n / 4; i += nt)
+                reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(a.out) + base)[i] = make_uint2(0u, 0u);
+        } else {
+            for (int i = t; i < n / 2; i += nt)
+                reinterpret_cast<float2*>(static_cast<float*>(a.out) + base)[i] = make_float2(0.f, 0.f);
         }
     }
 }

@@ -30,6 +30,7 @@
 // in-flight copies land and returns.  Nothing traps.
 #pragma once
 
+#include "combine.cuh"
 #include "ptx.cuh"
 #include "schedule.cuh"
 
@@ -53,7 +54,8 @@ struct MmaCfg {
     static constexpr int NC = NTG * HG * TS;            // consumer warps
     static constexpr int TILE_WARPS = NTG * HG;         // consumer warps reading one tile
     static constexpr int PRODUCER = NC;                 // index of the TMA warp
-    static constexpr int THREADS = 32 * (NC + 1);
+    static constexpr int MERGE = NC + 1;                // index of the merge warp (split partials)
+    static constexpr int THREADS = 32 * (NC + 2);
     static constexpr int PANELS = D / 64;               // 128-byte-wide column panels
     static constexpr int PANEL_BYTES = kTile * 128;     // 64 tokens x 64 bf16
     // One stage: K and V tiles of 64 tokens, bf16 in 128-byte panels, or 8-bit
@@ -78,6 +80,7 @@ struct __align__(16) MmaControl {
     uint64_t qempty[2];
     uint64_t merge_full;
     uint64_t merge_free;
+    uint64_t mjob[2];  // the CTA's first / last segment partial written (merge warp's jobs)
     Plan plan;
     int abort;
 };
@@ -130,6 +133,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
         }
         mbar_init(smem_addr(&ctrl->merge_full), (C::MGN - 1) * HG);
         mbar_init(smem_addr(&ctrl->merge_free), HG);
+        for (int k = 0; k < 2; ++k) mbar_init(smem_addr(&ctrl->mjob[k]), HG);
         ctrl->abort = 0;
     }
     // Query rows a TMA box does not cover (R < ROWS) must read as zeros.
@@ -143,6 +147,14 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     fence_proxy_async_smem();
     __syncthreads();
 
+    if (warp == C::MERGE) {
+        // ------------------------------------------------------------ merge warp
+        if (!merge_warp<D, OUT_BF16>(a, ctrl->plan, ctrl->mjob, abort_flag)) {
+            *abort_flag = 1;
+            if (lane == 0) atomicOr(a.status, kFlagTimeout);
+        }
+        return;
+    }
     const int64_t lo = ctrl->plan.lo;
     const int64_t hi = ctrl->plan.hi;
     if (lo >= hi) return;
@@ -625,6 +637,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
                             if (g == 0) a.ws_lse[slot * a.R + r] = M[nt][j] + log2f(Lsum[nt][j]);
                         }
                     }
+                if (!whole) {
+                    // This warp wrote its head group's partial (all d, lse): hand it to the merge warp.
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&ctrl->mjob[first_seg ? 0 : 1]));
+                }
             }
             first_seg = false;
         }

@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
+#include "combine.cuh"
 #include "ptx.cuh"
 #include "schedule.cuh"
 
@@ -41,6 +42,8 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
     __shared__ float sm_m[kSimtWarps][HC];
     __shared__ float sm_l[kSimtWarps][HC];
     __shared__ float sm_o[kSimtWarps][HC][D];
+    __shared__ int merge_last;
+    __shared__ uint32_t s_epoch;
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -49,7 +52,10 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
     grid_dependency_wait();
     grid_launch_dependents();
     if (warp == 0) make_plan(a, &plan);
+    if (threadIdx.x == 32) s_epoch = merge_epoch_take(a);
     __syncthreads();
+    uint32_t* const bank = merge_bank(a, s_epoch, 0, blockDim.x);
+    zero_empty_sequences<D, OUT_BF16>(a, 0, blockDim.x);
     const int64_t lo = plan.lo, hi = plan.hi;
     if (lo >= hi) return;
     Walk w{plan.b, plan.kv, plan.tile, plan.n_b, plan.L};
@@ -58,6 +64,7 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
     int64_t gi = lo;
     while (gi < hi) {
         const int seg_tiles = static_cast<int>(min(static_cast<int64_t>(w.n_b - w.tile), hi - gi));
+        const int64_t s_u = gi - w.tile;  // global index of the unit's first tile
         const bool whole = (w.tile == 0) && (seg_tiles == w.n_b);
         const int64_t slot = first ? 2 * static_cast<int64_t>(blockIdx.x) : 2 * static_cast<int64_t>(blockIdx.x) + 1;
         const int t_begin = w.tile * kTile;
@@ -150,6 +157,19 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
                 }
             }
             __syncthreads();
+        }
+        if (!whole) {
+            // The CTA's partial of this unit is complete: the last of the unit's
+            // partials merges them all.
+            const SplitUnit su = split_unit_of(s_u, w.n_b, plan.n_tiles, plan.g);
+            __threadfence();
+            __syncthreads();
+            if (threadIdx.x == 0) merge_last = atomicAdd(bank + su.ca, 1u) == static_cast<uint32_t>(su.n_parts - 1);
+            __syncthreads();
+            if (merge_last && warp == 0) {
+                __threadfence();
+                merge_unit<D, OUT_BF16>(a, su, (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R) * D);
+            }
         }
         first = false;
         gi += seg_tiles;

@@ -50,6 +50,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include "combine.cuh"
 #include "ptx.cuh"
 #include "schedule.cuh"
 #include "tcgen05.cuh"
@@ -77,7 +78,8 @@ struct TcCfg {
     static constexpr int HW = RP / HSPLIT;             // query columns per softmax warp
     static constexpr int NSM = 4 * HSPLIT;
     static constexpr int WARP_QK = 1, WARP_PV = 2, WARP_SM0 = 3;
-    static constexpr int THREADS = 32 * (3 + NSM);
+    static constexpr int WARP_MERGE = WARP_SM0 + NSM;  // merge warp (split partials)
+    static constexpr int THREADS = 32 * (4 + NSM);
     static constexpr int HALF_BYTES = kTile * 128;     // one 64-row TMA box of 128-byte rows
     static constexpr int PANEL_BYTES = kStepTokens * 128;  // 128 token rows x 128 bytes
     static constexpr int KV_BYTES = KV8 ? PANEL_BYTES : 2 * PANEL_BYTES;  // one of K, V for a step
@@ -118,6 +120,7 @@ struct __align__(16) TcControl {
     uint64_t ofull, ofree;          // O^T of a segment complete / read by the epilogue
     uint64_t xch;                   // softmax-warp exchange (count 4)
     uint64_t drain[2];              // final completion of each issuing warp's products
+    uint64_t mjob[2];               // the CTA's first / last segment partial written (merge warp's jobs)
     Plan plan;
     uint32_t tmem_base;
     int abort;
@@ -243,6 +246,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         mbar_init(smem_addr(&ctrl->ofull), 1);
         mbar_init(smem_addr(&ctrl->ofree), C::NSM);
         mbar_init(smem_addr(&ctrl->xch), C::NSM);
+        for (int k = 0; k < 2; ++k) mbar_init(smem_addr(&ctrl->mjob[k]), C::NSM);
         ctrl->abort = 0;
     }
     // Query rows past H_Q come back from TMA as zeros; the P^T buffers start
@@ -865,14 +869,19 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         }
                     }
                 }
-                if (!whole && sp == 0 && lane == 0) {
-#pragma unroll
-                    for (int h = 0; h < HW; ++h)
-                        if (h0 + h < a.R) a.ws_lse[slot * a.R + h0 + h] = m[h] + log2f(lt[h]);
-                }
                 tc::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree));
+                if (lane == 0) mbar_arrive(smem_addr(&ctrl->ofree));  // O^T read: the next segment may start
+                if (!whole) {
+                    if (sp == 0 && lane == 0) {
+#pragma unroll
+                        for (int h = 0; h < HW; ++h)
+                            if (h0 + h < a.R) a.ws_lse[slot * a.R + h0 + h] = m[h] + log2f(lt[h]);
+                    }
+                    // this warp's share of the partial is written: hand it to the merge warp
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_addr(&ctrl->mjob[seg == 0 ? 0 : 1]));
+                }
             }
             st = (st + nsub) % NS;
             j += nsub;
@@ -880,6 +889,11 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             if (nsub > 1) advance_step(w, a, gi, n_of[1], hi);
         }
         if (!ok) fail();
+    }
+
+    if (warp == C::WARP_MERGE) {
+        // ------------------------------------------------------------ merge warp
+        if (!merge_warp<C::D, OUT_BF16>(a, ctrl->plan, ctrl->mjob, abort_flag)) fail();
     }
 
     // ---------------------------------------------------------------- teardown

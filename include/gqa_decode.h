@@ -217,12 +217,30 @@ gqa_status gqa_decode_timed(const gqa_decode_params* params, const void* q, cons
  *  - Every call on a device shares the one array, and it keeps the last
  *    call's contents.  Calls whose kernels overlap on the GPU (different
  *    streams, or different host threads) race on it: order them.
+ *  - Device-side problems (clamped seq_lens, out-of-range pages, a pipeline
+ *    wait that gave up) are flagged in the array's status word exactly as in
+ *    a caller's workspace; read and clear them with
+ *    gqa_static_workspace_status.  The flags accumulate until cleared.
+ *  - The looked-up address is kept for the life of the process: after
+ *    cudaDeviceReset (or anything else that destroys the device's primary
+ *    context) this entry point must not be called again on that device.
  */
 #define GQA_STATIC_WORKSPACE_BYTES (8u << 20)
 gqa_status gqa_decode_static_workspace(const gqa_decode_params* params, const void* q,
                                        const void* k_cache, const void* v_cache,
                                        const int32_t* seq_lens, const int32_t* block_table,
                                        float scale, void* out, void* stream);
+
+/*
+ * The status word of gqa_decode_static_workspace's built-in array on the
+ * CURRENT device: like gqa_read_status, it synchronises `stream`, writes the
+ * accumulated GQA_FLAG_* bits to *flags and clears them when `clear` is
+ * non-zero.  Allocates nothing.  On a device where gqa_decode_static_workspace
+ * has not run yet it performs that call's one-time set-up (address lookup and
+ * a cleared status word) and reports 0.  The pages this library follows have
+ * no counterpart to it.
+ */
+gqa_status gqa_static_workspace_status(void* stream, uint32_t* flags, int clear);
 
 /*
  * The step before gqa_decode for a new token: rotary position embedding of

@@ -156,6 +156,8 @@ def test_read_status_rejects_nulls(lib):
     flags = ctypes.c_uint32(0)
     assert lib.gqa_read_status(None, None, ctypes.byref(flags), 0) == GQA_ERR_INVALID
     assert lib.gqa_read_status(ctypes.c_void_p(256), None, None, 0) == GQA_ERR_INVALID
+    # the built-in workspace's reader checks its output pointer before touching a device
+    assert lib.gqa_static_workspace_status(None, None, 0) == GQA_ERR_INVALID
 
 
 def test_binding_refuses_host_tensors():

@@ -242,6 +242,34 @@ def test_repeated_calls_are_bitwise_identical(cuda_device):
     assert torch.equal(a.view(torch.int32), b.view(torch.int32))
 
 
+@pytest.mark.parametrize("kernel,h_q", [("mma_sync", 8), ("tcgen05", 32), ("auto", 128)])
+def test_one_sequence_cut_across_every_cta(cuda_device, kernel, h_q):
+    # One unit spread over all CTAs: every CTA holds a partial of it and the last
+    # writer merges up to a grid's worth of partials inside the split kernel.
+    w = small("llama2_70b_ragged", B=1, H_Q=h_q, H_KV=1, seq_len=148 * 64 * 3 + 17, ragged=False)
+    inp = make_inputs(w)
+    assert_parity(run_gpu(inp, w, cuda_device, kernel=kernel), oracle_full(inp, w), f"one sequence, {kernel}")
+
+
+def test_merge_counters_over_many_calls_on_one_workspace(cuda_device):
+    # Successive calls alternate between the two banks of merge counters; each
+    # call's batch is cut differently, and every result must match the oracle.
+    base = small("llama2_70b_ragged", B=5, seq_len=3000)
+    ws = None
+    for i in range(5):
+        w = dataclasses.replace(base, seed=700 + i)
+        inp = make_inputs(w)
+        inp["seq_lens"][i % w.B] = 0  # an empty sequence somewhere in every call
+        d = to_device(inp, cuda_device)
+        if ws is None:
+            ws = torch.zeros(gq.workspace_bytes(gq.make_params(d["q"], d["k"], d["seq_lens"])), dtype=torch.uint8,
+                             device=cuda_device)
+        out = torch.full(d["q"].shape, float("nan"), device=cuda_device)
+        gq.gqa_decode(d["q"], d["k"], d["v"], d["seq_lens"], scale=w.softmax_scale, out=out, workspace=ws)
+        assert_parity(out.cpu(), oracle_full(inp, w), f"call {i}")
+    assert gq.read_status(ws) == 0
+
+
 # ------------------------------------------------------------ full benchmark sizes, sampled
 
 def sampled_pairs(w, lens, per_seq=4, seed=0):
@@ -261,7 +289,8 @@ def check_sampled(out, inp, w, pairs):
     assert_parity(got, ref, f"{w.name} sampled")
 
 
-@pytest.mark.parametrize("name", ["llama2_70b_ragged", "paged_long", "sweep_hkv32", "sweep_hkv1"])
+@pytest.mark.parametrize("name", ["llama2_70b_ragged", "paged_long", "sweep_hkv32", "sweep_hkv8", "sweep_hkv4",
+                                  "sweep_hkv1"])
 def test_full_size_sampled(cuda_device, name):
     w = WORKLOADS[name]
     inp = make_inputs(w)
