@@ -50,18 +50,22 @@ __device__ __forceinline__ bool merge_ticket(uint32_t* cnt, int expected) {
 
 // Warp-collective merge of a split unit's R x D outputs (written at
 // out[row0 + h D + d]) from its partials, which other SMs wrote during this
-// grid and are therefore read at L2 (ld.global.cg).  Element e = lane + 32 k
-// is head e / (D/4), dimensions 4 (e % (D/4)) .. +3.  A block of KG elements
+// grid and are therefore read at L2 (ld.global.cg).  Element e is head
+// e / (D/4), dimensions 4 (e % (D/4)) .. +3.  A block of KG elements
 // x JG partials issues all of its loads before using any, so it costs one L2
 // round trip; partials are folded in with a running maximum, so any number
 // of them works.
+// Warp `part` of `parts` cooperating warps takes elements part * 32 + lane +
+// 32 parts k.
 template <int D, bool OUT_BF16>
-__device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, const int64_t row0) {
+__device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, const int64_t row0, const int part,
+                                        const int parts) {
     constexpr int KG = 4, JG = 4, Q = D / 4;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    const int lane = threadIdx.x & 31;
+    const int lane = (threadIdx.x & 31) + 32 * part;
+    const int stride = 32 * parts;
     const int E = a.R * Q;
-    for (int e0 = 0; e0 < E; e0 += 32 * KG) {
+    for (int e0 = 0; e0 < E; e0 += stride * KG) {
         float m[KG], l[KG];
         float4 acc[KG];
 #pragma unroll
@@ -75,7 +79,7 @@ __device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, 
             float4 ov[KG][JG];
 #pragma unroll
             for (int kk = 0; kk < KG; ++kk) {
-                const int e = e0 + 32 * kk + lane;
+                const int e = e0 + stride * kk + lane;
                 const int h = e / Q, q4 = e - h * Q;
 #pragma unroll
                 for (int jj = 0; jj < JG; ++jj) {
@@ -114,7 +118,7 @@ __device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, 
         }
 #pragma unroll
         for (int kk = 0; kk < KG; ++kk) {
-            const int e = e0 + 32 * kk + lane;
+            const int e = e0 + stride * kk + lane;
             if (e >= E) continue;
             const int h = e / Q, q4 = e - h * Q;
             const float inv = 1.f / l[kk];
@@ -139,6 +143,7 @@ __device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, 
 struct MergeJobs {
     int n;
     int slot[2];      // which of mjob[0] (first segment) / mjob[1] (last) it waits on
+    bool tail[2];     // the job is the CTA's last segment (its writers are then done streaming)
     SplitUnit su[2];
     int b[2], kv[2];
 };
@@ -152,6 +157,7 @@ __device__ __forceinline__ MergeJobs merge_jobs_of(const KernelArgs& a, const Pl
     const bool first_cut = p.tile > 0 || s0 + p.n_b > p.hi;
     if (first_cut) {
         J.slot[J.n] = 0;
+        J.tail[J.n] = s0 + p.n_b >= p.hi;
         J.su[J.n] = split_unit_of(s0, p.n_b, p.n_tiles, p.g);
         J.b[J.n] = p.b;
         J.kv[J.n] = p.kv;
@@ -167,6 +173,7 @@ __device__ __forceinline__ MergeJobs merge_jobs_of(const KernelArgs& a, const Pl
         const int64_t su = start + static_cast<int64_t>(kv) * n_b;
         if (su + n_b > p.hi) {
             J.slot[J.n] = 1;
+            J.tail[J.n] = true;
             J.su[J.n] = split_unit_of(su, n_b, p.n_tiles, p.g);
             J.b[J.n] = b;
             J.kv[J.n] = kv;
@@ -178,10 +185,15 @@ __device__ __forceinline__ MergeJobs merge_jobs_of(const KernelArgs& a, const Pl
 
 // The merge warp of a split kernel (warp-collective).  Takes the call's merge
 // epoch, clears its share of the next call's counters, writes the outputs of
-// empty sequences, then serves the CTA's merge jobs in order.  Returns false
-// when a wait for the writers gave up (the caller raises the timeout flag).
+// empty sequences, then serves the CTA's merge jobs in order.  A job of the
+// CTA's last segment is merged together with that segment's `helpers` warps,
+// which have finished streaming by then: the ticket's outcome goes to *last
+// and they are released through *assist (they call merge_assist).  Returns
+// false when a wait for the writers gave up (the caller raises the timeout
+// flag; helpers time out on *assist in turn).
 template <int D, bool OUT_BF16>
-__device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, uint64_t* mjob, const volatile int* abort) {
+__device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, uint64_t* mjob, uint64_t* assist,
+                                           volatile int* last, int helpers, const volatile int* abort) {
     const int lane = threadIdx.x & 31;
     uint32_t epoch = 0;
     if (lane == 0) epoch = merge_epoch_take(a);
@@ -192,8 +204,33 @@ __device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, u
     const MergeJobs J = merge_jobs_of(a, p);
     for (int k = 0; k < J.n; ++k) {
         if (!mbar_wait_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort)) return false;
-        if (merge_ticket(bank + J.su[k].ca, J.su[k].n_parts))
-            merge_unit<D, OUT_BF16>(a, J.su[k], (static_cast<int64_t>(J.b[k]) * a.H_Q + J.kv[k] * a.R) * D);
+        const bool mine = merge_ticket(bank + J.su[k].ca, J.su[k].n_parts);
+        const int64_t row0 = (static_cast<int64_t>(J.b[k]) * a.H_Q + J.kv[k] * a.R) * D;
+        if (J.tail[k]) {
+            if (lane == 0) {
+                *last = mine ? 1 : 0;
+                mbar_arrive(smem_addr(assist));
+            }
+            if (mine) merge_unit<D, OUT_BF16>(a, J.su[k], row0, helpers, helpers + 1);
+        } else if (mine) {
+            merge_unit<D, OUT_BF16>(a, J.su[k], row0, 0, 1);
+        }
+    }
+    return true;
+}
+
+// A writer warp of the CTA's last segment, when that segment was cut, after
+// streaming: waits for the merge warp's ticket and, if it was the unit's last,
+// merges share `part` of `parts` (the merge warp takes the last share).
+template <int D, bool OUT_BF16>
+__device__ __forceinline__ bool merge_assist(const KernelArgs& a, uint64_t* assist, const volatile int* last,
+                                             int b, int kv, int64_t s_u, int n_b, int64_t n_tiles, int g, int part,
+                                             int parts, const volatile int* abort) {
+    if (!mbar_wait_warp(smem_addr(assist), 0u, abort)) return false;
+    if (*last) {
+        __threadfence();
+        merge_unit<D, OUT_BF16>(a, split_unit_of(s_u, n_b, n_tiles, g),
+                                (static_cast<int64_t>(b) * a.H_Q + kv * a.R) * D, part, parts);
     }
     return true;
 }

@@ -81,6 +81,8 @@ struct __align__(16) MmaControl {
     uint64_t merge_full;
     uint64_t merge_free;
     uint64_t mjob[2];  // the CTA's first / last segment partial written (merge warp's jobs)
+    uint64_t assist;   // the merge warp's ticket for the last segment is known
+    int merge_last;    // ... and it was the unit's last: the consumers help merge
     Plan plan;
     int abort;
 };
@@ -134,6 +136,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
         mbar_init(smem_addr(&ctrl->merge_full), (C::MGN - 1) * HG);
         mbar_init(smem_addr(&ctrl->merge_free), HG);
         for (int k = 0; k < 2; ++k) mbar_init(smem_addr(&ctrl->mjob[k]), HG);
+        mbar_init(smem_addr(&ctrl->assist), 1);
         ctrl->abort = 0;
     }
     // Query rows a TMA box does not cover (R < ROWS) must read as zeros.
@@ -149,7 +152,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
 
     if (warp == C::MERGE) {
         // ------------------------------------------------------------ merge warp
-        if (!merge_warp<D, OUT_BF16>(a, ctrl->plan, ctrl->mjob, abort_flag)) {
+        if (!merge_warp<D, OUT_BF16>(a, ctrl->plan, ctrl->mjob, &ctrl->assist, &ctrl->merge_last, C::NC,
+                                     abort_flag)) {
             *abort_flag = 1;
             if (lane == 0) atomicOr(a.status, kFlagTimeout);
         }
@@ -258,6 +262,9 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
     uint32_t ph = 0, qph = 0, mfull_ph = 0, mfree_ph = 0;
     bool first_seg = true;
     int seg_start_tile = 0;
+    bool tail_cut = false;  // the CTA's last segment so far was cut (its unit is merged)
+    int tail_b = 0, tail_kv = 0, tail_nb = 0;
+    int64_t tail_su = 0;
     uint32_t qb[C::Q_IN_REGS ? KS : 1][NT][2];  // B fragments of Q^T (k-step, 8-head tile)
     int seg_q = 0;                                  // Q-ring slot of the current segment
     float o[KS][NT][4];      // O^T accumulators, per 16-row block of d and 8-head tile
@@ -540,6 +547,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
                     l[nt][j] += __shfl_xor_sync(0xffffffffu, l[nt][j], 16);
                 }
             const bool whole = (seg_start_tile == 0) && last_tile;
+            tail_cut = !whole;
+            tail_b = w.b;
+            tail_kv = w.kv;
+            tail_nb = w.n_b;
+            tail_su = gi - w.tile;
             if (mg > 0) {
                 if (!mbar_wait_warp(smem_addr(&ctrl->merge_free), mfree_ph ^ 1u, abort_flag)) { fail(); break; }
                 mfree_ph ^= 1u;
@@ -647,6 +659,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, HG, KV8>::THREADS, 1)
         }
         if (gi + 1 < hi) w.advance(a);
     }
+    // The CTA's last segment was cut: help the merge warp merge its unit.
+    if (tail_cut && !*abort_flag &&
+        !merge_assist<D, OUT_BF16>(a, &ctrl->assist, &ctrl->merge_last, tail_b, tail_kv, tail_su, tail_nb,
+                                   ctrl->plan.n_tiles, ctrl->plan.g, warp, C::NC + 1, abort_flag))
+        fail();
 }
 
 }  // namespace gqa

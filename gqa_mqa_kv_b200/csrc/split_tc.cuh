@@ -121,6 +121,8 @@ struct __align__(16) TcControl {
     uint64_t xch;                   // softmax-warp exchange (count 4)
     uint64_t drain[2];              // final completion of each issuing warp's products
     uint64_t mjob[2];               // the CTA's first / last segment partial written (merge warp's jobs)
+    uint64_t assist;                // the merge warp's ticket for the last segment is known
+    int merge_last;                 // ... and it was the unit's last: the softmax warps help merge
     Plan plan;
     uint32_t tmem_base;
     int abort;
@@ -247,6 +249,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         mbar_init(smem_addr(&ctrl->ofree), C::NSM);
         mbar_init(smem_addr(&ctrl->xch), C::NSM);
         for (int k = 0; k < 2; ++k) mbar_init(smem_addr(&ctrl->mjob[k]), C::NSM);
+        mbar_init(smem_addr(&ctrl->assist), 1);
         ctrl->abort = 0;
     }
     // Query rows past H_Q come back from TMA as zeros; the P^T buffers start
@@ -480,6 +483,9 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         float m[HW], l[HW];
         uint32_t xpar = 0, qph = 0;
         int qs = 0, qcur = 0, seg = -1, seg_start_tile = 0, st = 0;
+        bool tail_cut = false;  // the CTA's last segment so far was cut (its unit is merged)
+        int tail_b = 0, tail_kv = 0, tail_nb = 0;
+        int64_t tail_su = 0;
         float vfac = 1.f, qf_uniform = a.sl2;
         bool ok = true;
 
@@ -882,6 +888,11 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_addr(&ctrl->mjob[seg == 0 ? 0 : 1]));
                 }
+                tail_cut = !whole;
+                tail_b = w.b;
+                tail_kv = w.kv;
+                tail_nb = w.n_b;
+                tail_su = gi - w.tile;
             }
             st = (st + nsub) % NS;
             j += nsub;
@@ -889,11 +900,18 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
             if (nsub > 1) advance_step(w, a, gi, n_of[1], hi);
         }
         if (!ok) fail();
+        // The CTA's last segment was cut: help the merge warp merge its unit.
+        if (ok && tail_cut &&
+            !merge_assist<C::D, OUT_BF16>(a, &ctrl->assist, &ctrl->merge_last, tail_b, tail_kv, tail_su, tail_nb,
+                                          ctrl->plan.n_tiles, ctrl->plan.g, wi, C::NSM + 1, abort_flag))
+            fail();
     }
 
     if (warp == C::WARP_MERGE) {
         // ------------------------------------------------------------ merge warp
-        if (!merge_warp<C::D, OUT_BF16>(a, ctrl->plan, ctrl->mjob, abort_flag)) fail();
+        if (!merge_warp<C::D, OUT_BF16>(a, ctrl->plan, ctrl->mjob, &ctrl->assist, &ctrl->merge_last, C::NSM,
+                                        abort_flag))
+            fail();
     }
 
     // ---------------------------------------------------------------- teardown
