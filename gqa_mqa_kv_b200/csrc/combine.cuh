@@ -203,7 +203,7 @@ __device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, u
     if (p.lo >= p.hi) return true;
     const MergeJobs J = merge_jobs_of(a, p);
     for (int k = 0; k < J.n; ++k) {
-        if (!mbar_wait_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort)) return false;
+        if (!mbar_wait_sleepy_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort, 500)) return false;
         const bool mine = merge_ticket(bank + J.su[k].ca, J.su[k].n_parts);
         const int64_t row0 = (static_cast<int64_t>(J.b[k]) * a.H_Q + J.kv[k] * a.R) * D;
         if (J.tail[k]) {
@@ -226,7 +226,7 @@ template <int D, bool OUT_BF16>
 __device__ __forceinline__ bool merge_assist(const KernelArgs& a, uint64_t* assist, const volatile int* last,
                                              int b, int kv, int64_t s_u, int n_b, int64_t n_tiles, int g, int part,
                                              int parts, const volatile int* abort) {
-    if (!mbar_wait_warp(smem_addr(assist), 0u, abort)) return false;
+    if (!mbar_wait_sleepy_warp(smem_addr(assist), 0u, abort, 100)) return false;
     if (*last) {
         __threadfence();
         merge_unit<D, OUT_BF16>(a, split_unit_of(s_u, n_b, n_tiles, g),

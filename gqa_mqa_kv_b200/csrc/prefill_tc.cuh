@@ -27,8 +27,8 @@
 //                   rescaled in tensor memory then).  P replaces S_t in its
 //                   own columns as bf16 hi and lo parts: keys 32c .. 32c+31
 //                   go to columns 32c .. 32c+15 (hi, two keys per column) and
-//                   32c+16 .. 32c+31 (lo), so the product keeps ~16 bits of
-//                   every weight.
+//                   32c+16 .. 32c+31 (lo), both truncated, so the product
+//                   keeps ~15 bits of every weight.
 //   O_t += P V      tcgen05.mma, M = 128, N = d = 128, K = 128 keys, once on
 //                   the hi part and once on the lo part; A = P read from
 //                   tensor memory, B = the value rows read MN-major; O_t in
@@ -50,6 +50,8 @@
 #pragma once
 
 #include <cuda_bf16.h>
+
+#include <utility>
 
 #include "ptx.cuh"
 #include "schedule.cuh"
@@ -186,17 +188,39 @@ __device__ __forceinline__ float pf_max3(float a, float b, float c) {
     return d;
 }
 
-// p0, p1 -> bf16 hi parts (truncated: the top 16 bits of each fp32) and bf16
-// lo parts (round to nearest of the exact remainder); hi + lo is within
-// 2^-15 of each weight.  p0 lands in the low half of each packed word.
+// p0, p1 -> bf16 hi parts and bf16 lo parts, both by truncation: hi = the
+// top 16 bits of each fp32, lo = the top 16 bits of the exact remainder
+// p - hi, so hi + lo is within 2^-14 of each weight.  Bit operations only: a
+// float-to-bf16 conversion would use the unit that also computes the
+// exponentials.  p0 lands in the low half of each packed word.
 __device__ __forceinline__ void pf_split(float p0, float p1, uint64_t neg1, uint32_t& hi, uint32_t& lo) {
     const uint32_t a = __float_as_uint(p0), b = __float_as_uint(p1);
     hi = __byte_perm(a, b, 0x7632);
     const uint64_t rem = pf_fma2(pf_pack(__uint_as_float(a & 0xffff0000u), __uint_as_float(b & 0xffff0000u)), neg1,
                                  pf_pack(p0, p1));
     const float2 r = pf_unpack(rem);
-    const __nv_bfloat162 l2 = __floats2bfloat162_rn(r.x, r.y);
-    lo = *reinterpret_cast<const uint32_t*>(&l2);
+    lo = __byte_perm(__float_as_uint(r.x), __float_as_uint(r.y), 0x7632);
+}
+
+// S = Q K^T as 8 products of K = 16 (two 64-column panels of d, four 32-byte
+// slices each), offsets fixed at compile time.
+template <int... K>
+__device__ __forceinline__ void pf_issue_qk(uint32_t d, uint64_t da, uint64_t db, std::integer_sequence<int, K...>) {
+    constexpr uint32_t IDESC = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 128, PfCfg::BN);
+    (tc::mma_f16_off<static_cast<uint32_t>(((K >> 2) * PfCfg::PANEL + 32 * (K & 3)) >> 4)>(d, da, db, IDESC, K > 0),
+     ...);
+}
+
+// O += P_hi V + P_lo V as 16 products of K = 16 keys: product i is part i / 8
+// (hi, lo) of keys 16 (i % 8) .. +15 -- P columns 32 (k / 2) + 16 part +
+// 8 (k % 2) -- against value rows 16 k .. +15 (2048 bytes each).
+template <int... I>
+__device__ __forceinline__ void pf_issue_pv(uint32_t d, uint32_t pa, uint64_t db, bool fresh,
+                                            std::integer_sequence<int, I...>) {
+    constexpr uint32_t IDESC = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 1, 128, PfCfg::D);
+    (tc::mma_f16_ts_off<static_cast<uint32_t>(32 * ((I & 7) >> 1) + 16 * (I >> 3) + 8 * (I & 1)),
+                        static_cast<uint32_t>((I & 7) * 128)>(d, pa, db, IDESC, I > 0 || !fresh),
+     ...);
 }
 
 // Warpgroup-wide register budget changes (every warp of the warpgroup executes them).
@@ -217,8 +241,6 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
     static_assert(sizeof(PfControl) <= C::CTRL_BYTES, "control block overflows its slot");
     static_assert(128 * C::REG_LOW + 256 * C::REG_HIGH <= C::THREADS * C::REG_LAUNCH,
                   "the register split must fit the registers the block is launched with");
-    constexpr uint32_t IDESC_QK = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 0, 128, C::BN);
-    constexpr uint32_t IDESC_PV = tc::instr_desc(tc::kFmtBF16, tc::kFmtBF16, 0, 1, 128, C::D);
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_addr(smem_raw);
@@ -280,7 +302,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         // K/V rows are read again by the sequence's other units: keep them in L2.
         const uint64_t pol_kv = policy_evict_last();
         const uint64_t pol_q = policy_evict_first();
-        int64_t ld = 0;  // K/V loads issued: K of step g is load 2g, V is 2g + 1
+        uint32_t ld = 0;  // K/V loads issued: K of step g is load 2g, V is 2g + 1 (a CTA runs < 2^31 steps)
         int uc = 0;      // units issued
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -355,8 +377,8 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         if (!ok) {
             fail();
             // Let copies already in flight land before the CTA's shared memory goes away.
-            const int64_t first = ld > C::NS ? ld - C::NS : 0;
-            for (int64_t i = first; i < ld; ++i)
+            const uint32_t first = ld > C::NS ? ld - C::NS : 0;
+            for (uint32_t i = first; i < ld; ++i)
                 mbar_wait(smem_addr(&ctrl->full[i % C::NS]), static_cast<uint32_t>((i / C::NS) & 1), nullptr);
             if (uc > 0) mbar_wait(smem_addr(&ctrl->qfull), static_cast<uint32_t>(uc - 1) & 1u, nullptr);
         }
@@ -365,43 +387,34 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
     if (warp == C::WARP_MMA) {
         // ------------------------------------------------------------ tensor-core issue
         // Global step g of this CTA: K(g) is ring load 2g, V(g) load 2g + 1.
-        auto stage = [&](int64_t li) { return ring + static_cast<uint32_t>(li % C::NS) * C::TILE; };
-        auto loaded = [&](int64_t li) {
+        auto stage = [&](uint32_t li) { return ring + (li % C::NS) * C::TILE; };
+        auto loaded = [&](uint32_t li) {
             return mbar_wait_warp(smem_addr(&ctrl->full[li % C::NS]), static_cast<uint32_t>((li / C::NS) & 1),
                                   abort_flag);
         };
         // S_t = Q_t K^T (8 products of K = 16).  Descriptor start addresses are
         // advanced by adding (offset >> 4) to the descriptor: every operand lies
-        // below 256 KB, so the 14-bit address field never carries.
+        // below 256 KB, so the 14-bit address field never carries.  The issue
+        // sequences are straight-line code with compile-time offsets: one thread
+        // issues every product of the CTA, and run-time address arithmetic per
+        // product would make the issue itself the bottleneck.
         auto issue_qk = [&](int t, uint32_t kt) {
-            const uint64_t da0 = tc::smem_desc(q_smem + t * C::TILE, 16, 1024, tc::kLayoutSw128);
-            const uint64_t db0 = tc::smem_desc(kt, 16, 1024, tc::kLayoutSw128);
-            const uint32_t d = tmem + C::S_COL + 128 * t;
-#pragma unroll 1
-            for (int k = 0; k < 8; ++k) {
-                const uint64_t off = static_cast<uint64_t>(((k >> 2) * C::PANEL + 32 * (k & 3)) >> 4);
-                tc::mma_f16(d, da0 + off, db0 + off, IDESC_QK, k > 0);
-            }
+            pf_issue_qk(tmem + C::S_COL + 128 * t, tc::smem_desc(q_smem + t * C::TILE, 16, 1024, tc::kLayoutSw128),
+                        tc::smem_desc(kt, 16, 1024, tc::kLayoutSw128), std::make_integer_sequence<int, 8>{});
         };
         // O_t += P_hi V + P_lo V; keys 32c .. 32c+31 have hi at columns 32c .. +15, lo at 32c+16 .. +31
         auto issue_pv = [&](int t, uint32_t vt, bool fresh) {
-            const uint64_t db0 = tc::smem_desc(vt, C::PANEL, 1024, tc::kLayoutSw128);
-            const uint32_t pa0 = tmem + C::S_COL + 128 * t;
-            const uint32_t d = tmem + C::O_COL + 128 * t;
-#pragma unroll 1
-            for (int i = 0; i < 16; ++i) {
-                const int part = i >> 3, k = i & 7;
-                tc::mma_f16_ts(d, pa0 + 32 * (k >> 1) + 16 * part + 8 * (k & 1), db0 + static_cast<uint64_t>(k * 128),
-                               IDESC_PV, !(fresh && i == 0));
-            }
+            pf_issue_pv(tmem + C::O_COL + 128 * t, tmem + C::S_COL + 128 * t,
+                        tc::smem_desc(vt, C::PANEL, 1024, tc::kLayoutSw128), fresh,
+                        std::make_integer_sequence<int, 16>{});
         };
-        auto wait_p = [&](int t, int64_t gs) {
+        auto wait_p = [&](int t, uint32_t gs) {
             return mbar_wait_warp(smem_addr(&ctrl->pfull[t]), static_cast<uint32_t>(gs) & 1u, abort_flag);
         };
         auto wait_ofree = [&](int t, int uc) {
             return mbar_wait_warp(smem_addr(&ctrl->ofree[t]), (static_cast<uint32_t>(uc) & 1u) ^ 1u, abort_flag);
         };
-        int64_t g = 0;
+        uint32_t g = 0;  // steps of this CTA so far (a CTA runs < 2^31 steps)
         int uc = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -435,7 +448,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
             }
             __syncwarp();
             for (int i = 1; i < n; ++i) {
-                const int64_t gi = g + i;
+                const uint32_t gi = g + i;
                 if (!loaded(2 * gi)) {
                     ok = false;
                     break;
@@ -472,7 +485,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                 __syncwarp();
             }
             if (!ok) break;
-            const int64_t last = g + n - 1;
+            const uint32_t last = g + n - 1;
             if ((n == 1 && !wait_ofree(1, uc)) || !wait_p(1, last)) {
                 ok = false;
                 break;
@@ -504,7 +517,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         const float NEG_INF = -__int_as_float(0x7f800000);
         const uint64_t neg1 = pf_pack(-1.f, -1.f);
         const uint64_t sl2x2 = pf_pack(a.sl2, a.sl2);
-        int64_t g = 0;
+        uint32_t g = 0;
         int uc = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
@@ -594,7 +607,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
                 // Tile 0's warps clear them (before P_0 of the step, which both value
                 // products of the step follow).
                 if (t == 0 && C::BN * (j + 1) > x.L) {
-                    const int64_t vi = 2 * g + 1;
+                    const uint32_t vi = 2 * g + 1;
                     const int e = static_cast<int>(vi % C::NS);
                     if (!mbar_wait_warp(smem_addr(&ctrl->full[e]), static_cast<uint32_t>(vi / C::NS) & 1u,
                                         abort_flag)) {

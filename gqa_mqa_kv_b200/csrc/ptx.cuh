@@ -72,6 +72,27 @@ __device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, con
     }
 }
 
+// For a warp that waits long and is not on the critical path (a CTA's merge
+// warp waits for most of the kernel): polls every ~sleep_ns, so it does not
+// take issue slots from the streaming warps of its sub-partition.  Same
+// limits and result as mbar_wait_for.
+__device__ __forceinline__ bool mbar_wait_sleepy(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                                 uint32_t sleep_ns) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_timer_ns();
+    while (true) {
+        __nanosleep(sleep_ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (abort != nullptr && *abort) return false;
+        if (global_timer_ns() - t0 > kWaitTimeoutNs) return false;
+    }
+}
+
+__device__ __forceinline__ bool mbar_wait_sleepy_warp(uint32_t bar, uint32_t parity, const volatile int* abort,
+                                                      uint32_t sleep_ns) {
+    return __all_sync(0xffffffffu, mbar_wait_sleepy(bar, parity, abort, sleep_ns));
+}
+
 // The kernels' wait: limit kWaitTimeoutNs.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const volatile int* abort) {
     return mbar_wait_for(bar, parity, abort, kWaitTimeoutNs);

@@ -183,6 +183,34 @@ __device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a, uint64_t b, 
         : "memory");
 }
 
+// mma_f16 / mma_f16_ts with compile-time offsets added inside the asm: OFF
+// (16-byte units) to both shared-memory descriptors, or A_COL to the A
+// tensor-memory address and B_OFF to the B descriptor.  An unrolled issue
+// sequence then keeps no per-product address in registers.
+template <uint32_t OFF>
+__device__ __forceinline__ void mma_f16_off(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 ad, bd;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "add.s64 ad, %1, %5;\n\t"
+        "add.s64 bd, %2, %5;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], ad, bd, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(static_cast<uint32_t>(acc)), "n"(OFF)
+        : "memory");
+}
+
+template <uint32_t A_COL, uint32_t B_OFF>
+__device__ __forceinline__ void mma_f16_ts_off(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t.reg .b64 bd;\n\t.reg .b32 at;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "add.u32 at, %1, %5;\n\t"
+        "add.s64 bd, %2, %6;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [at], bd, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(static_cast<uint32_t>(acc)), "n"(A_COL), "n"(B_OFF)
+        : "memory");
+}
+
 // Arrives once on the mbarrier when every tcgen05 operation this thread has
 // issued so far has completed.
 __device__ __forceinline__ void commit(uint32_t bar) {
