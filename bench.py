@@ -46,6 +46,7 @@ PREFILL_METRIC = "prefill-attention achieved TFLOP/s (causal, algorithmic 4 d pe
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # B200 HBM3e, DGX figure (7.7 TB/s on HGX)
 FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_BF16_TFLOPS_SUSTAINED = 1400.0  # the recipe's sustained figure under the power cap
 CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -131,13 +132,18 @@ def hbm_peak():
 
 
 def tensor_peak():
-    """Dense bf16 TFLOP/s: the burst figure (a kernel timed alone)."""
+    """Dense bf16 TFLOP/s: (burst, sustained, kind).  The burst figure is for a
+    kernel timed alone; the sustained one (a seconds-long GEMM loop under the
+    1 kW power cap) for a kernel that runs continuously, as the multi-token
+    bench does (a soak, then back-to-back steps)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
-            return float(json.load(f)["bf16_tflops"]), "measured"
+            d = json.load(f)
+        burst = float(d["bf16_tflops"])
+        return burst, float(d.get("bf16_tflops_sustained", burst)), "measured"
     except Exception:
-        return FALLBACK_BF16_TFLOPS, "fallback"
+        return FALLBACK_BF16_TFLOPS, FALLBACK_BF16_TFLOPS_SUSTAINED, "fallback"
 
 
 class ClockSampler:
@@ -739,7 +745,10 @@ def run_ours_prefill(args):
                             lambda s: call(qq=q_sets[s], oo=out_sets[s]), out_sets, out_host,
                             max(1, min(args.e2e_steps, 20)), 2, dist)
 
-    peak, peak_kind = tensor_peak()
+    burst, sustained, peak_kind = tensor_peak()
+    # The kernel runs back to back for seconds (soak, then the timed steps), so it
+    # is in the sustained, power-capped regime; the clocks record shows it.
+    peak = sustained
     ms_per_step = elapsed_ms / args.steps
     achieved = flops / (kernel_ms * 1e-3) / 1e12
     line = {
@@ -757,7 +766,9 @@ def run_ours_prefill(args):
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(w.name),
                      "kernel": "prefill_tc_kernel (the whole call)", "kernel_us": kernel_ms * 1e3,
-                     "peak_note": f"{peak_kind} dense bf16 GEMM TFLOP/s (burst)",
+                     "peak_note": (f"{peak_kind} dense bf16 GEMM TFLOP/s, sustained (the kernel runs back to back "
+                                   "for seconds under the power cap); frac_vs_burst divides by the burst figure"),
+                     "peak_burst": burst, "frac_vs_burst": achieved / burst,
                      "tensor_work_note": "the value product runs twice (bf16 hi and lo parts of P): "
                                          "tensor-core work is 1.5x the algorithmic FLOPs"},
         "device_status_flags": status,

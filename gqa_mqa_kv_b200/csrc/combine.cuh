@@ -203,7 +203,7 @@ __device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, u
     if (p.lo >= p.hi) return true;
     const MergeJobs J = merge_jobs_of(a, p);
     for (int k = 0; k < J.n; ++k) {
-        if (!mbar_wait_sleepy_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort, 500)) return false;
+        if (!mbar_wait_sleepy_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort, 200)) return false;
         const bool mine = merge_ticket(bank + J.su[k].ca, J.su[k].n_parts);
         const int64_t row0 = (static_cast<int64_t>(J.b[k]) * a.H_Q + J.kv[k] * a.R) * D;
         if (J.tail[k]) {
