@@ -153,6 +153,21 @@ __device__ __forceinline__ bool pf_unit(const PrefillArgs& a, int u, PfUnit& x, 
     return true;
 }
 
+// The unit a CTA takes in its k-th round, or -1 when it has none left.
+// Round k covers units [k G, k G + G) of the heaviest-first order
+// (G = gridDim.x); even rounds hand them to the CTAs left to right and odd
+// rounds right to left, so the per-CTA sums even out over each pair of rounds
+// although unit costs fall steadily along the order (a fixed cyclic order
+// leaves the first CTAs 6-13% more work than the average).  Only the last
+// round can be short, so a CTA with no unit in round k has none after it, and
+// the round of a unit u is u / G.
+__device__ __forceinline__ int pf_order(int k, int n_units) {
+    const int G = static_cast<int>(gridDim.x);
+    const int i = (k & 1) ? G - 1 - static_cast<int>(blockIdx.x) : static_cast<int>(blockIdx.x);
+    const int64_t u = static_cast<int64_t>(k) * G + i;
+    return u < n_units ? static_cast<int>(u) : -1;
+}
+
 __device__ __forceinline__ void pf_fence_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
@@ -305,7 +320,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         uint32_t ld = 0;  // K/V loads issued: K of step g is load 2g, V is 2g + 1 (a CTA runs < 2^31 steps)
         int uc = 0;      // units issued
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        for (int u = pf_order(0, n_units); u >= 0 && ok; u = pf_order(u / gridDim.x + 1, n_units)) {
             PfUnit x;
             uint32_t fl;
             const bool has = pf_unit(a, u, x, &fl);
@@ -417,7 +432,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         uint32_t g = 0;  // steps of this CTA so far (a CTA runs < 2^31 steps)
         int uc = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        for (int u = pf_order(0, n_units); u >= 0 && ok; u = pf_order(u / gridDim.x + 1, n_units)) {
             PfUnit x;
             uint32_t fl;
             if (!pf_unit(a, u, x, &fl)) continue;
@@ -520,7 +535,7 @@ __global__ void __launch_bounds__(PfCfg::THREADS, 1)
         uint32_t g = 0;
         int uc = 0;
         bool ok = true;
-        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x) {
+        for (int u = pf_order(0, n_units); u >= 0 && ok; u = pf_order(u / gridDim.x + 1, n_units)) {
             PfUnit x;
             uint32_t fl;
             if (!pf_unit(a, u, x, &fl)) continue;
