@@ -57,8 +57,20 @@ __device__ __forceinline__ bool merge_ticket(uint32_t* cnt, int expected) {
 // of them works.
 // Warp `part` of `parts` cooperating warps takes elements part * 32 + lane +
 // 32 parts k.
+// The arguments are plain values: a reference to the kernel's argument block
+// would make the compiler keep that block in local memory, and every read of
+// it in the streaming loops would become a local load.
+struct MergeIO {
+    const float* ws_o;
+    const float* ws_lse;
+    void* out;
+    int R;
+};
+
+__device__ __forceinline__ MergeIO merge_io(const KernelArgs& a) { return MergeIO{a.ws_o, a.ws_lse, a.out, a.R}; }
+
 template <int D, bool OUT_BF16>
-__device__ __noinline__ void merge_unit(const KernelArgs& a, const SplitUnit u, const int64_t row0, const int part,
+__device__ __noinline__ void merge_unit(const MergeIO a, const SplitUnit u, const int64_t row0, const int part,
                                         const int parts) {
     constexpr int KG = 4, JG = 4, Q = D / 4;
     const float NEG_INF = -__int_as_float(0x7f800000);
@@ -202,7 +214,10 @@ __device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, u
     zero_empty_sequences<D, OUT_BF16>(a, static_cast<int>(threadIdx.x) - lane, 32);
     if (p.lo >= p.hi) return true;
     const MergeJobs J = merge_jobs_of(a, p);
-    for (int k = 0; k < J.n; ++k) {
+    // k unrolled: J's arrays stay in registers
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        if (k >= J.n) break;
         if (!mbar_wait_sleepy_warp(smem_addr(&mjob[J.slot[k]]), 0u, abort, 200)) return false;
         const bool mine = merge_ticket(bank + J.su[k].ca, J.su[k].n_parts);
         const int64_t row0 = (static_cast<int64_t>(J.b[k]) * a.H_Q + J.kv[k] * a.R) * D;
@@ -211,9 +226,9 @@ __device__ __forceinline__ bool merge_warp(const KernelArgs& a, const Plan& p, u
                 *last = mine ? 1 : 0;
                 mbar_arrive(smem_addr(assist));
             }
-            if (mine) merge_unit<D, OUT_BF16>(a, J.su[k], row0, helpers, helpers + 1);
+            if (mine) merge_unit<D, OUT_BF16>(merge_io(a), J.su[k], row0, helpers, helpers + 1);
         } else if (mine) {
-            merge_unit<D, OUT_BF16>(a, J.su[k], row0, 0, 1);
+            merge_unit<D, OUT_BF16>(merge_io(a), J.su[k], row0, 0, 1);
         }
     }
     return true;
@@ -229,7 +244,7 @@ __device__ __forceinline__ bool merge_assist(const KernelArgs& a, uint64_t* assi
     if (!mbar_wait_sleepy_warp(smem_addr(assist), 0u, abort, 100)) return false;
     if (*last) {
         __threadfence();
-        merge_unit<D, OUT_BF16>(a, split_unit_of(s_u, n_b, n_tiles, g),
+        merge_unit<D, OUT_BF16>(merge_io(a), split_unit_of(s_u, n_b, n_tiles, g),
                                 (static_cast<int64_t>(b) * a.H_Q + kv * a.R) * D, part, parts);
     }
     return true;

@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
             __syncthreads();
             if (merge_last && warp == 0) {
                 __threadfence();
-                merge_unit<D, OUT_BF16>(a, su, (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R) * D, 0, 1);
+                merge_unit<D, OUT_BF16>(merge_io(a), su, (static_cast<int64_t>(w.b) * a.H_Q + w.kv * a.R) * D, 0, 1);
             }
         }
         first = false;
