@@ -10,6 +10,7 @@
 
 #include <atomic>
 #include <cmath>
+#include <algorithm>
 #include <cstring>
 #include <mutex>
 #include <set>
@@ -99,8 +100,15 @@ SplitKernel select_kernel(const gqa_decode_params* p, bool kv8) {
     }
 }
 
+// CTAs of a split launch: one per SM (tensor-core kernels) or kSimtCtasPerSm per
+// SM (CUDA-core kernel), but never more than the step can have tiles,
+// B H_KV ceil(max_seq_len / 64): a CTA without tiles would still take the
+// merge epoch and clear its share of the counters, which costs a tiny step
+// more than its work.
 int grid_for(const gqa_decode_params* p, const DeviceInfo& dev, bool kv8 = false) {
-    return select_kernel(p, kv8) == SplitKernel::kSimt && !kv8 ? dev.sms * kSimtCtasPerSm : dev.sms;
+    const int full = select_kernel(p, kv8) == SplitKernel::kSimt && !kv8 ? dev.sms * kSimtCtasPerSm : dev.sms;
+    const int64_t most = static_cast<int64_t>(p->B) * p->H_KV * ((static_cast<int64_t>(p->max_seq_len) + 63) / 64);
+    return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(full, most)));
 }
 
 // Workspace layout: header (status word, merge epoch), two banks of merge
@@ -379,9 +387,9 @@ gqa_status run(const gqa_decode_params* p, const void* q, const void* k, const v
 
     DeviceInfo dev;
     if ((st = device_info(&dev)) != GQA_OK) return st;
-    // 8-bit caches always use one CTA per SM, so gqa_decode_workspace_size's
-    // answer for the same parameters is always enough.
-    const int grid = kv8 ? dev.sms : grid_for(p, dev);
+    // 8-bit caches use at most one CTA per SM, never more than the bf16 choice
+    // for the same parameters, so gqa_decode_workspace_size's answer is enough.
+    const int grid = kv8 ? std::min(dev.sms, grid_for(p, dev, true)) : grid_for(p, dev);
     if (grid > kMergeCounters) return GQA_ERR_UNSUPPORTED;  // one merge counter per CTA
     if (workspace == nullptr || !aligned(workspace, 256) || workspace_bytes < workspace_for(p, grid))
         return GQA_ERR_WORKSPACE;

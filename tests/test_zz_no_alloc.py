@@ -135,7 +135,9 @@ def test_fixed_workspace_reports_out_of_range_pages(cuda_device):
 
 
 def test_fixed_workspace_refuses_problems_that_do_not_fit(cuda_device):
-    w = dataclasses.replace(WORKLOADS["llama3_8b"], name="wide", B=2, H_Q=1024, H_KV=1, seq_len=64)
+    # 1024 query heads per KV head, and enough tiles (2 x 1024) to use every CTA of the
+    # grid: the partial slots alone (two per CTA, 1024 x 128 floats each) far exceed 8 MiB
+    w = dataclasses.replace(WORKLOADS["llama3_8b"], name="wide", B=2, H_Q=1024, H_KV=1, seq_len=65536)
     d = to_device(make_inputs(w), cuda_device)
     out = torch.full(d["q"].shape, 7.0, dtype=torch.float32, device=cuda_device)
     assert call_static(d, False, out, 1.0 / math.sqrt(w.D)) == GQA_ERR_WORKSPACE
