@@ -92,10 +92,10 @@ SplitKernel select_kernel(const gqa_decode_params* p, bool kv8) {
         case GQA_KERNEL_MMA_SYNC: return mma_ok ? SplitKernel::kMmaSync : SplitKernel::kNone;
         default:
             // Measured on one B200: tcgen05 wins for 8-bit caches and for bf16 groups of
-            // 17..32 heads (MQA at R = 32: 48 vs 51 us); mma.sync for R <= 16 (R = 16:
-            // 56 vs 63 us) and the HBM-bound narrow groups.
+            // 9..32 heads (R = 16: 53.3 vs 55.6 us); mma.sync for the HBM-bound groups of
+            // up to 8 heads (R = 8: 93.0 vs 94.0 us, R = 4: 51.0 vs 52.6 us).
             if (kv8) return tc_ok ? SplitKernel::kTcgen05 : SplitKernel::kSimt;
-            if (tc_ok && R > 16) return SplitKernel::kTcgen05;
+            if (tc_ok && R > 8) return SplitKernel::kTcgen05;
             return mma_ok ? SplitKernel::kMmaSync : SplitKernel::kSimt;
     }
 }

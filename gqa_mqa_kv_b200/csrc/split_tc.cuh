@@ -97,7 +97,11 @@ struct TcCfg {
     static constexpr int NP = (!KV8 && RP == 32) ? 1 : 2;
     static constexpr int MAX_STAGES = 8;
     static constexpr int T_LAZY = 8;                   // reference slack, base 2
-    static constexpr bool PAIR = HW <= 16 && NP == 2;  // softmax warps take two steps per pass
+    // Softmax warps take two steps per pass with 8-bit caches, where halving the
+    // per-step exchanges pays (8-bit 70B-shaped batch 200-205 vs 208 us); for bf16
+    // the doubled loop costs more in instruction fetch than it saves (R = 16
+    // MQA-like sweep 53 vs 61 us).
+    static constexpr bool PAIR = KV8 && HW <= 16 && NP == 2;
     // fixed region after the stage ring; every piece 1024-aligned
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_QT = OFF_Q + NQ * QSLOT_BYTES;

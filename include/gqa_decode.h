@@ -75,7 +75,7 @@ typedef enum gqa_rope_pairing {
 /* Which split kernel serves a call (both compute the same result). */
 typedef enum gqa_kernel {
     GQA_KERNEL_AUTO = 0,     /* head_dim 128: tcgen05 for 8-bit caches (R <= 32) and for bf16 with
-                                17 <= R <= 32; mma.sync for the other bf16 groups (R <= 64);
+                                9 <= R <= 32; mma.sync for the other bf16 groups (R <= 64);
                                 CUDA cores otherwise */
     GQA_KERNEL_MMA_SYNC = 1, /* warp-level mma.sync kernel: bf16 cache with R <= 64, or an 8-bit
                                 cache with head_dim 128 and R <= 8 */
