@@ -30,6 +30,30 @@ __device__ __forceinline__ float to_f32<__nv_fp8_e4m3>(__nv_fp8_e4m3 x) { return
 constexpr int kSimtWarps = 4;
 constexpr int kSimtHeads = 8;
 
+// Token tok's key and value rows of KV head w.kv (this lane's D/32 elements);
+// an out-of-range page reads as zeros and raises the flag.
+template <typename TKV, int D, bool PAGED>
+__device__ __forceinline__ void simt_load_row(const KernelArgs& a, const TKV* __restrict__ k,
+                                              const TKV* __restrict__ v, const Walk& w, int tok,
+                                              float (&kr)[D / 32], float (&vr)[D / 32]) {
+    const int lane = threadIdx.x & 31;
+    int64_t row;
+    bool live = true;
+    if constexpr (PAGED) {
+        const int page = __ldg(a.block_table + static_cast<int64_t>(w.b) * a.max_blocks + tok / kTile);
+        live = page >= 0 && page < a.num_blocks;
+        if (!live && lane == 0) atomicOr(a.status, kFlagBadBlock);
+        row = (static_cast<int64_t>(live ? page : 0) * kTile + tok % kTile) * a.H_KV + w.kv;
+    } else {
+        row = (static_cast<int64_t>(w.b) * a.S_max + tok) * a.H_KV + w.kv;
+    }
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) {
+        kr[i] = live ? to_f32(k[row * D + lane + 32 * i]) : 0.f;
+        vr[i] = live ? to_f32(v[row * D + lane + 32 * i]) : 0.f;
+    }
+}
+
 // TQ: element type of q; TKV: element type of the cache (fp32, bf16 or E4M3
 // bytes, the latter multiplied by per-KV-head k_scale / v_scale).
 template <typename TQ, typename TKV, int D, bool PAGED, bool OUT_BF16>
@@ -86,23 +110,14 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
                 m[j] = NEG_INF;
                 l[j] = 0.f;
             }
+            // The next token's rows are loaded before this token's arithmetic, so a
+            // warp waits on memory once per token pair of loads instead of per token.
+            float kr[DPL], vr[DPL];
+            if (t_begin + warp < t_end) simt_load_row<TKV, D, PAGED>(a, k, v, w, t_begin + warp, kr, vr);
             for (int tok = t_begin + warp; tok < t_end; tok += kSimtWarps) {
-                float kr[DPL], vr[DPL];
-                int64_t row;
-                bool live = true;
-                if constexpr (PAGED) {
-                    const int page = __ldg(a.block_table + static_cast<int64_t>(w.b) * a.max_blocks + tok / kTile);
-                    live = page >= 0 && page < a.num_blocks;
-                    if (!live && lane == 0) atomicOr(a.status, kFlagBadBlock);
-                    row = (static_cast<int64_t>(live ? page : 0) * kTile + tok % kTile) * a.H_KV + w.kv;
-                } else {
-                    row = (static_cast<int64_t>(w.b) * a.S_max + tok) * a.H_KV + w.kv;
-                }
-#pragma unroll
-                for (int i = 0; i < DPL; ++i) {
-                    kr[i] = live ? to_f32(k[row * D + lane + 32 * i]) : 0.f;  // a bad page reads as zeros
-                    vr[i] = live ? to_f32(v[row * D + lane + 32 * i]) : 0.f;
-                }
+                float kn[DPL], vn[DPL];
+                const bool more = tok + kSimtWarps < t_end;
+                if (more) simt_load_row<TKV, D, PAGED>(a, k, v, w, tok + kSimtWarps, kn, vn);
 #pragma unroll
                 for (int j = 0; j < HC; ++j) {
                     float s = 0.f;
@@ -118,6 +133,13 @@ __global__ void __launch_bounds__(32 * kSimtWarps)
 #pragma unroll
                     for (int i = 0; i < DPL; ++i) o[j][i] = fmaf(p, vr[i], o[j][i] * al);
                     m[j] = mn;
+                }
+                if (more) {
+#pragma unroll
+                    for (int i = 0; i < DPL; ++i) {
+                        kr[i] = kn[i];
+                        vr[i] = vn[i];
+                    }
                 }
             }
 #pragma unroll
