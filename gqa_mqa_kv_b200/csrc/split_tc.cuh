@@ -154,6 +154,11 @@ __device__ __forceinline__ Step step_at(const Walk& w, int64_t gi, int64_t lo, i
 }
 
 __device__ __forceinline__ void advance_step(Walk& w, const KernelArgs& a, int64_t& gi, int n, int64_t hi) {
+    if (w.tile + n < w.n_b && gi + n < hi) {  // the usual case: the next step is in the same unit
+        w.tile += n;
+        gi += n;
+        return;
+    }
     for (int i = 0; i < n; ++i) {
         if (gi + 1 < hi) w.advance(a);
         ++gi;
@@ -799,7 +804,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 // Loaded value rows past L_b may hold anything; 0 * NaN would poison O^T.
                 const bool loaded = tok < kTile * n_of[u];
                 if (h0 == 0 && tile_of[u] + n_of[u] == w.n_b && loaded && tile_of[u] * kTile + tok >= w.L) {
-                    const int stu = (st + u) % NS;
+                    const int stu = st + u < NS ? st + u : st + u - NS;
                     const uint32_t vrow = stages + stu * C::STAGE_BYTES + C::KV_BYTES + tok * 128;
 #pragma unroll
                     for (int pnl = 0; pnl < (KV8 ? 1 : 2); ++pnl)
@@ -898,7 +903,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                 tail_nb = w.n_b;
                 tail_su = gi - w.tile;
             }
-            st = (st + nsub) % NS;
+            st += nsub;  // nsub <= 2 <= NS: no division on the per-pass path
+            if (st >= NS) st -= NS;
             j += nsub;
             advance_step(w, a, gi, stp.n, hi);
             if (nsub > 1) advance_step(w, a, gi, n_of[1], hi);
