@@ -223,17 +223,35 @@ def kernel_source_hash(kind: str = "decode") -> str:
     return h.hexdigest()[:16]
 
 
+# The files each measured kernel is compiled from: its own header, the headers
+# it includes and the host file that sets up its launch.
+KERNEL_FILES = {
+    "split_mma": ["gqa_decode.cu", "split_mma.cuh", "combine.cuh", "schedule.cuh", "ptx.cuh"],
+    "split_tc": ["gqa_decode.cu", "split_tc.cuh", "tcgen05.cuh", "combine.cuh", "schedule.cuh", "ptx.cuh"],
+    "prefill_tc": ["gqa_decode.cu", "prefill_tc.cuh", "tcgen05.cuh", "schedule.cuh", "ptx.cuh"],
+}
+
+
+def kernel_files_hash(kernel: str) -> str:
+    """sha256 (first 16 hex digits) over the files one kernel is compiled from."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "gqa_mqa_kv_b200", "csrc")
+    for name in sorted(KERNEL_FILES[kernel]):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
 def recorded_traffic(workload: str):
     """DRAM bytes per launch of the workload's dominant kernel from the
     committed ncu summary, if it was taken on the current source of that
-    kernel; else None."""
+    kernel (the hash over the files that kernel is compiled from); else None."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.json")
-    kind = "prefill" if workload in PREFILL_WORKLOADS else "decode"
     try:
         with open(path) as f:
             rec = json.load(f)
         ent = rec.get(workload)
-        if ent and ent.get("kernel_source_hash") == kernel_source_hash(kind):
+        if ent and ent.get("kernel_files_hash") == kernel_files_hash(ent["kernel_family"]):
             return float(ent["dram_bytes_per_launch"])
     except Exception:
         pass
