@@ -496,6 +496,7 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
         int tail_b = 0, tail_kv = 0, tail_nb = 0;
         int64_t tail_su = 0;
         float vfac = 1.f, qf_uniform = a.sl2;
+        float qfac[KV8 ? HW : 1];  // KV8: the segment's score factor per head, qf_uniform * 2^-a
         bool ok = true;
 
         auto exchange = [&]() -> bool {
@@ -577,6 +578,8 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_addr(&ctrl->qtfull[qcur]));
                     if (!exchange()) { ok = false; break; }  // every head's 2^-a is in place
+#pragma unroll
+                    for (int h = 0; h < HW; ++h) qfac[h] = qf_uniform * X->qscale[qcur][h0 + h];
                 }
             }
             // The softmax warps take two steps of a segment per pass (one when the
@@ -625,13 +628,10 @@ __global__ void __launch_bounds__(TcCfg<RP, KV8>::THREADS, 1)
                         tc::tmem_ld8(ta + h0 + 8 * c, r1);
                         tc::tmem_ld8(ta + RP + h0 + 8 * c, r2);
                         tc::tmem_wait_ld();
-                        const float4 qa = *reinterpret_cast<const float4*>(&X->qscale[qcur][h0 + 8 * c]);
-                        const float4 qb = *reinterpret_cast<const float4*>(&X->qscale[qcur][h0 + 8 * c + 4]);
-                        const float qsc[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            s[u][8 * c + i] = (__uint_as_float(r1[i]) + __uint_as_float(r2[i]) * 0.0625f) *
-                                              (qf_uniform * qsc[i]);
+                            s[u][8 * c + i] =
+                                (__uint_as_float(r1[i]) + __uint_as_float(r2[i]) * 0.0625f) * qfac[8 * c + i];
                     }
                 }
                 // S^T buffer sb may take the step after next
