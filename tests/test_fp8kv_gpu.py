@@ -92,6 +92,28 @@ def test_fp8_full_size_sampled(cuda_device):
     assert_parity(got, ref_fp8(inp, w, pairs=pairs), "fp8 full size")
 
 
+@pytest.mark.parametrize("kernel,h_q", [("tcgen05", 8), ("tcgen05", 32), ("mma_sync", 8)])
+def test_fp8_one_sequence_cut_across_every_cta(cuda_device, kernel, h_q):
+    # One unit spread over all CTAs, with a ragged tail: every CTA holds a
+    # partial and the last writer merges a grid's worth of them.
+    w = dataclasses.replace(WORKLOADS["llama2_70b_ragged_fp8"], name="one", B=1, H_Q=h_q, H_KV=1,
+                            seq_len=148 * 64 * 3 + 17, ragged=False)
+    inp = make_inputs(w)
+    assert_parity(run_fp8(inp, w, cuda_device, kernel=kernel), ref_fp8(inp, w), f"fp8 one sequence, {kernel}")
+
+
+@pytest.mark.parametrize("name", ["paged_long_fp8", "llama3_8b_fp8"])
+def test_fp8_other_full_size_workloads_sampled(cuda_device, name):
+    w = WORKLOADS[name]
+    inp = make_inputs(w)
+    out = run_fp8(inp, w, cuda_device, paged=bool(w.page_size))
+    assert torch.all(torch.isfinite(out))
+    rng = np.random.default_rng(1)
+    pairs = [(b, int(h)) for b in range(w.B) for h in {0, w.H_Q - 1, int(rng.integers(0, w.H_Q))}]
+    got = torch.stack([out[b, h] for b, h in pairs])
+    assert_parity(got, ref_fp8(inp, w, pairs=pairs), f"{name} sampled")
+
+
 def test_fp8_requires_bf16_query(cuda_device):
     w = dataclasses.replace(WORKLOADS["llama2_70b_ragged_fp8"], B=1, seq_len=64)
     d = to_device(make_inputs(w), cuda_device)
