@@ -290,7 +290,7 @@ def check_sampled(out, inp, w, pairs):
 
 
 @pytest.mark.parametrize("name", ["llama2_70b_ragged", "paged_long", "sweep_hkv32", "sweep_hkv8", "sweep_hkv4",
-                                  "sweep_hkv1"])
+                                  "sweep_hkv2", "sweep_hkv1"])
 def test_full_size_sampled(cuda_device, name):
     w = WORKLOADS[name]
     inp = make_inputs(w)
